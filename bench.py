@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the top-k MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+                    [--preset olmoe --tokens 4096] [--no-sweep] [--no-cpu]
+
+One step = one whole layer forward (RMSNorm, router, top-k, permutation,
+grouped gate/up and down GEMMs, combine) over one batch of T synthetic tokens,
+through the C ABI (moe_layer_forward).  Default workload: the OLMoE-1B-7B-shaped
+layer (d 2048, 64 experts, top-8, expert hidden 1024, bf16) at T = 4096 prefill
+tokens.  With N > 1 (torchrun) every rank runs its own batch on its own GPU with
+replicated weights -- token data parallelism, no collective on the data path
+(weak scaling); the step time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle (the
+only reference this layer has) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_synth  # noqa: E402
+from moe_layer_fp32_b200 import roofline as R  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (decode & prefill); % of HBM / tensor-core roofline"
+KERNEL_NAMES_TC = ["rmsnorm", "router", "route_topk", "permute", "gather", "gateup_gemm",
+                   "down_gemm", "combine"]
+KERNEL_NAMES_SIMT = ["rmsnorm", "router", "route_topk", "permute", "gateup_simt", "down_simt",
+                     "combine"]
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--preset", default="olmoe")
+    p.add_argument("--tokens", type=int, default=4096)
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    return p.parse_args()
+
+
+def workload_name(sh, T):
+    names = {"olmoe": "OLMoE-1B-7B-shaped", "v2lite": "DeepSeek-V2-Lite-shaped",
+             "qwen3_int4": "Qwen3-30B-A3B-shaped (int4 experts)",
+             "qwen3_int8": "Qwen3-30B-A3B-shaped (int8 experts)", "v3": "DeepSeek-V3-shaped",
+             "tiny": "Tiny"}
+    kind = "decode" if T <= 64 else "prefill"
+    return f"{names.get(sh.name, sh.name)} MoE layer forward, {kind} T={T}"
+
+
+def config_dict(sh, T, world):
+    return {"workload": workload_name(sh, T), "T_per_gpu": T, "global_batch": T * world,
+            "d": sh.d, "E": sh.E, "k": sh.k, "f": sh.f, "n_shared": sh.n_shared,
+            "expert_dtype": sh.expert, "router_dtype": sh.router, "bias_mode": sh.bias_mode,
+            "capacity_factor": sh.capacity_factor, "renormalize": sh.renormalize,
+            "parallelism": f"replicas x{world} (token data parallel, no collective)",
+            "l2": "inputs larger than L2 (126 MB): every step streams all touched expert "
+                  "weights (%.0f MB at this batch)" % (
+                      R.expert_bytes(sh.expert, sh.d, sh.f, sh.group_size) * sh.E / 1e6)}
+
+
+# --------------------------------------------------------------------- clocks
+class Clocks:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+# --------------------------------------------------------------------- helpers
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(li, x, n_tokens, reps=1):
+    """Oracle on the first n_tokens rows of the batch (routing over that
+    sub-batch); returns seconds per call."""
+    from oracle import moe_oracle as O
+    xs = x[:n_tokens]
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        O.layer_from_inputs(li, xs)
+    return (time.perf_counter() - t0) / reps
+
+
+# --------------------------------------------------------------------- our arm
+def run_ours(args):
+    import moe_layer_fp32_b200 as M
+    world, rank, local = dist_setup(args)
+    sh = moe_synth.PRESETS[args.preset]
+    T, K, W = args.tokens, args.steps, max(args.warmup, 3)
+    dev = torch.device("cuda", local)
+    li_host = moe_synth.make_layer(sh)
+    li = li_host.to(dev)
+    x_host = moe_synth.make_x(sh, T, stream=T + 7919 * rank)
+    x = x_host.to(dev)
+    layer = M.MoELayer(li, T)            # output in the activation dtype (bf16)
+    cfg = layer.cfg
+    L = M.moe_layer_launch_count(cfg)
+    names = KERNEL_NAMES_TC if sh.expert != "f32" else KERNEL_NAMES_SIMT
+
+    # routing statistics of this batch (touched experts, kept rows) for the roofline
+    counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
+    out = layer.forward(x, counts=counts)
+    torch.cuda.synchronize()
+    cnt = counts.cpu().numpy()
+    cap = None
+    if sh.capacity_factor > 0:
+        import math
+        cap = math.ceil(float(np.float32(sh.capacity_factor)) * T * sh.k / sh.E)
+    kept = int(np.minimum(cnt, cap).sum()) if cap else int(cnt.sum())
+    touched = int((cnt > 0).sum())
+
+    for _ in range(W):
+        layer.forward(x, out)
+    barrier(world)
+
+    # profiled steps: per-kernel events on up to 256 evenly spread steps
+    n_prof = min(K, 256)
+    prof_steps = set(np.linspace(0, K - 1, n_prof).round().astype(int).tolist())
+    evs = {s: [torch.cuda.Event(enable_timing=True) for _ in range(L + 1)] for s in prof_steps}
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    start.record()
+    for s in range(K):
+        if s in prof_steps:
+            M.moe_layer_forward_profiled(cfg, layer.w, x, out, layer.ws, evs[s])
+        else:
+            layer.forward(x, out)
+    end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    assert M.moe_get_device_status(layer.ws) == 0, "device error word set"
+    ms_max = max_over_ranks(ms, world)
+    per_kernel = {n: float(np.mean([evs[s][i].elapsed_time(evs[s][i + 1]) for s in prof_steps]))
+                  for i, n in enumerate(names)}
+    tokens_total = T * K * world
+    value = tokens_total / (ms_max / 1e3)
+
+    # roofline of the dominant kernel
+    peaks = R.measured_peaks()
+    dom = max(per_kernel, key=per_kernel.get)
+    dom_ms = per_kernel[dom]
+    if dom in ("gateup_gemm", "down_gemm", "router"):
+        if dom == "gateup_gemm":
+            fl = R.gateup_flops(sh, T, kept)
+        elif dom == "down_gemm":
+            fl = 2.0 * sh.d * sh.f * (kept + sh.n_shared * T)
+        else:
+            fl = 2.0 * T * sh.d * sh.E
+        tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        ach = fl / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 2),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(ach / tc_peak, 4),
+                "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a "
+                               "seconds-long loop)",
+                "algorithmic_per_launch": fl, "avg_launch_us": round(dom_ms * 1e3, 2),
+                "traffic": read_traffic(dom, sh, T)}
+    else:
+        nb = R.layer_bytes(sh, T, touched)
+        ach = nb / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                "avg_launch_us": round(dom_ms * 1e3, 2), "traffic": None}
+    # whole-layer roofline (slower of flops at the tensor peak and bytes over HBM)
+    fl_layer = R.layer_flops(sh, T, kept)
+    by_layer = R.layer_bytes(sh, T, touched)
+    t_roof = R.roofline_time(fl_layer, by_layer,
+                             peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12,
+                             peaks["hbm_gbs"] * 1e9)
+    layer_roof = {"t_roof_us": round(t_roof * 1e6, 2), "t_step_us": round(ms_max / K * 1e3, 2),
+                  "frac": round(t_roof / (ms_max / K / 1e3), 4),
+                  "bound": "tensor" if fl_layer / (peaks.get("bf16_tflops_sustained", 1) * 1e12)
+                  > by_layer / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                  "flops": fl_layer, "bytes": by_layer, "touched_experts": touched,
+                  "kept_rows": kept}
+
+    # end to end through the C ABI with host buffers
+    e2e = run_e2e(M, layer, x_host, sh, T, min(K, 200), world)
+
+    res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+           "steps": K, "warmup": W, "ms_per_step": round(ms_max / K, 5),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded N(0,1) tokens, fan-in-scaled random expert weights)",
+           "config": config_dict(sh, T, world), "roofline": roof, "layer_roofline": layer_roof,
+           "e2e": e2e, "gpu_launches": L * K, "clocks": clk,
+           "kernels_avg_us": {k: round(v * 1e3, 2) for k, v in per_kernel.items()}}
+    if rank == 0 and world == 1 and not args.no_sweep:
+        res["sweep"] = run_sweep(M, dev)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        res["cpu_baseline"] = cpu_baseline(li_host, x_host, sh, T)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def run_e2e(M, layer, x_host, sh, T, K, world):
+    xp = x_host.pin_memory()
+    outp = torch.empty(x_host.shape, dtype=layer.out_dtype).pin_memory()
+    xd = torch.empty_like(xp, device="cuda")
+    od = torch.empty(x_host.shape, dtype=layer.out_dtype, device="cuda")
+    for _ in range(3):
+        xd.copy_(xp, non_blocking=True)
+        layer.forward(xd, od)
+        outp.copy_(od, non_blocking=True)
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        xd.copy_(xp, non_blocking=True)
+        layer.forward(xd, od)
+        outp.copy_(od, non_blocking=True)
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    return {"value": round(T * K * world / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(xp.numel() * xp.element_size()),
+            "d2h_bytes_per_step": int(outp.numel() * outp.element_size()), "steps": K}
+
+
+def run_sweep(M, dev):
+    """Decode batches of the same layer: whole-layer time, stream-launched and
+    replayed from a CUDA graph, and the fraction of the HBM roofline."""
+    sh = moe_synth.PRESETS["olmoe"]
+    li = moe_synth.make_layer(sh).to(dev)
+    peaks = R.measured_peaks()
+    out = []
+    for T in (1, 16, 64):
+        x = moe_synth.make_x(sh, T).to(dev)
+        layer = M.MoELayer(li, T)
+        counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
+        o = layer.forward(x, counts=counts)
+        torch.cuda.synchronize()
+        touched = int((counts.cpu().numpy() > 0).sum())
+        for _ in range(20):
+            layer.forward(x, o)
+        n = 500
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        s.record()
+        for _ in range(n):
+            layer.forward(x, o)
+        e.record()
+        torch.cuda.synchronize()
+        us_stream = s.elapsed_time(e) / n * 1e3
+        us_graph = None
+        try:
+            g = torch.cuda.CUDAGraph()
+            st = torch.cuda.Stream()
+            with torch.cuda.stream(st):
+                layer.forward(x, o)
+                st.synchronize()
+                with torch.cuda.graph(g, stream=st):
+                    layer.forward(x, o, stream=st)
+            for _ in range(20):
+                g.replay()
+            torch.cuda.synchronize()
+            s.record()
+            for _ in range(n):
+                g.replay()
+            e.record()
+            torch.cuda.synchronize()
+            us_graph = s.elapsed_time(e) / n * 1e3
+            del g
+        except Exception as ex:  # capture problems are reported, not hidden
+            us_graph = f"capture failed: {ex}"
+        nb = R.layer_bytes(sh, T, touched)
+        best = min(us_stream, us_graph) if isinstance(us_graph, float) else us_stream
+        out.append({"workload": workload_name(sh, T), "T": T, "touched_experts": touched,
+                    "us_per_layer_stream": round(us_stream, 2),
+                    "us_per_layer_graph": round(us_graph, 2) if isinstance(us_graph, float) else us_graph,
+                    "tokens_per_s": round(T / (best / 1e6), 1),
+                    "hbm_roofline_us": round(nb / (peaks["hbm_gbs"] * 1e9) * 1e6, 2),
+                    "hbm_frac": round(nb / (best / 1e6) / (peaks["hbm_gbs"] * 1e9), 4)})
+    return out
+
+
+def cpu_baseline(li_host, x_host, sh, T, n_tokens=512):
+    """The oracle, as it stands, on the host cores: the first n_tokens rows of
+    the same batch (routing over that sub-batch, every expert they touch)."""
+    n = min(n_tokens, T)
+    sec = time_oracle(li_host, x_host, n)
+    return {"value": round(n / sec, 2), "unit": "tokens/s", "cores": cpu_threads(),
+            "kind": "oracle", "sample": f"first {n} of the {T} tokens of the timed batch, one "
+                                        f"call ({sec:.1f} s), numpy float64"}
+
+
+# --------------------------------------------------------------------- traffic
+def read_traffic(kernel, sh, T):
+    """DRAM bytes per launch of this kernel from the committed ncu summary, if
+    that summary was taken on the current kernel source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{sh.name}_T{T}.md")
+    if not os.path.exists(path):
+        return None
+    src = os.path.join(ROOT, "moe_layer_fp32_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("common.cuh", "gemm_tc.cuh"):
+        with open(os.path.join(src, f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    vals = {}
+    with open(path) as fh:
+        for line in fh:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != digest:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# --------------------------------------------------------------------- reference arm
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    sh = moe_synth.PRESETS[args.preset]
+    T, K, W = args.tokens, args.steps, max(args.warmup, 3)
+    li = moe_synth.make_layer(sh)
+    x = moe_synth.make_x(sh, T)
+    # size each step's sample so the whole run takes a few minutes
+    probe = time_oracle(li, x, 1)
+    budget = 150.0
+    per_step = budget / (K + W)
+    n_tok = 1
+    if per_step > 2 * probe:
+        n_tok = int(min(T, max(1, (per_step / probe))))
+    for _ in range(W):
+        time_oracle(li, x, n_tok)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        time_oracle(li, x, n_tok)
+    sec = time.perf_counter() - t0
+    value = n_tok * K / sec
+    cores = cpu_threads()
+    res = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+           "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(sec / K * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded N(0,1) tokens, fan-in-scaled random expert weights)",
+           "config": config_dict(sh, T, 1),
+           "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                            "kind": "oracle",
+                            "sample": f"each step: the oracle on the first {n_tok} token(s) of "
+                                      f"the T={T} batch (routing over that sub-batch)"},
+           "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

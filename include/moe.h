@@ -1,0 +1,234 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) top-k Mixture-of-Experts FFN layer forward.
+ *
+ * The layer (inference, one GPU):
+ *
+ *   xn      = RMSNorm(x) * gamma                       (rounded to the activation dtype)
+ *   logits  = xn . W_r                                 (FP32 accumulation)
+ *   idx, g  = top-k of the FP32 logits (+ per-expert bias), softmax gates in FP32,
+ *             optionally renormalised over the selected k
+ *   counts, offsets, perm = per-expert histogram + prefix scan + stable permutation,
+ *             with an optional capacity C*T*k/E per expert (overflow dropped)
+ *   y_a     = g_a * SwiGLU_e(xn_t)                     (grouped GEMM over experts)
+ *   out     = x + sum_shared SwiGLU_s(xn) + sum_{kept a of t} y_a
+ *
+ * Sources (page title, section):
+ *   "MoE: dynamism the compiler cannot remove" -- the natural implementation
+ *     (router -> top-k -> per-expert dispatch), the capacity section (buffers of
+ *     C*T*k/E rows, overflow tokens pass through on the residual) and the grouped
+ *     GEMM section (one launch over the total work T*k; each block finds its group
+ *     from a small descriptor array).
+ *   picx.dev summary of the moe-ceilings study, Sub-study 1 -- gate probabilities
+ *     accumulated in FP32 before the top-k; the router is kept un-quantised.
+ *   "MoE Research", section 2 -- shared (always-on) experts; per-expert bias terms
+ *     for auxiliary-loss-free balancing.  Section 3 -- grouped GEMM and sorting.
+ *   "MoE at the inference level ...", Workarounds -- gather -> grouped GEMM ->
+ *     scatter; int4 / fp8 expert weights.
+ *
+ * Conventions common to every entry point:
+ *   - Every tensor pointer is DEVICE memory owned by the caller; shapes are
+ *     row-major with the last index contiguous.  The library allocates nothing
+ *     and keeps no global state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream and never synchronise the host,
+ *     except moe_get_device_status.
+ *   - Argument errors are returned synchronously (MOE_ERR_INVALID /
+ *     MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE) and nothing is launched.  A failed
+ *     launch returns MOE_ERR_CUDA.
+ *   - Errors found on the device (an expert id outside [0,E) in topk_idx, a
+ *     pipeline wait that ran out) set an int32 error word at the start of the
+ *     workspace; read it with moe_get_device_status.  Kernels never trap.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,      /* bad argument (NULL pointer, k > E, size out of range) */
+  MOE_ERR_UNSUPPORTED = 2,  /* legal but not implemented (dtype/shape combination)   */
+  MOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moe_workspace_size */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call failed                             */
+  MOE_ERR_DEVICE = 5        /* the device error word is set (moe_get_device_status)  */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_INT8 = 2, MOE_INT4 = 3 } moe_dtype;
+
+/* Per-expert router bias ("MoE Research", section 2):
+ *   NONE   : no bias.
+ *   LOGIT  : the bias is part of the router logits; it moves both the selection
+ *            and the gate probabilities.
+ *   SELECT : auxiliary-loss-free style; the bias moves the selection only and the
+ *            gates are the softmax of the unbiased logits. */
+typedef enum { MOE_BIAS_NONE = 0, MOE_BIAS_LOGIT = 1, MOE_BIAS_SELECT = 2 } moe_bias_mode;
+
+/* Layer configuration.  All fields are 32-bit so that the layout is the same
+ * from every language. */
+typedef struct moe_config {
+  int32_t T;               /* tokens in the batch, >= 1                                 */
+  int32_t d;               /* model dim, multiple of 8 (of 128 for bf16/int experts)    */
+  int32_t E;               /* routed experts, 1..512, multiple of 8 for a bf16 router   */
+  int32_t k;               /* experts per token, 1..min(E, 32)                          */
+  int32_t f;               /* expert hidden dim (multiple of 128 for bf16/int experts)  */
+  int32_t n_shared;        /* always-on shared experts, 0..8; each has hidden f         */
+  float capacity_factor;   /* <= 0: uncapped; else cap = ceil(C*T*k/E) rows per expert,
+                              computed in double; assignments ranked in flat order
+                              a = t*k + j and kept iff their rank < cap                */
+  int32_t renormalize;     /* nonzero: gates divided by their sum over the k selected  */
+  int32_t bias_mode;       /* moe_bias_mode                                             */
+  float rms_eps;           /* RMSNorm epsilon                                           */
+  int32_t act_dtype;       /* x (and the residual): MOE_BF16 or MOE_F32                 */
+  int32_t out_dtype;       /* out: MOE_BF16 or MOE_F32 (MOE_F32 when act_dtype is F32);
+                              the combine sums in FP32 and rounds once to this type    */
+  int32_t router_dtype;    /* W_r: MOE_BF16 or MOE_F32 (must equal act_dtype)           */
+  int32_t expert_dtype;    /* MOE_F32 (requires act F32) | MOE_BF16 | MOE_INT8 | MOE_INT4 */
+  int32_t group_size;      /* int4: scale group along K; must be 128                    */
+} moe_config;
+
+/* Layer weights (device pointers, caller-owned).
+ *   rms_gamma   [d] float32
+ *   w_router    [d, E]            router dtype
+ *   router_bias [E] float32, or NULL (required unless bias_mode == NONE)
+ *   w_gate/w_up [E, d, f]         F32/BF16: that type; INT8: int8; INT4: uint8 [E, d, f/2]
+ *   w_down      [E, f, d]         F32/BF16: that type; INT8: int8; INT4: uint8 [E, f, d/2]
+ *   s_gate/s_up INT8: bf16 [E, f]; INT4: bf16 [E, d/128, f]; otherwise NULL
+ *   s_down      INT8: bf16 [E, d]; INT4: bf16 [E, f/128, d]; otherwise NULL
+ *   sh_*        the same for the n_shared shared experts ([S, ...]); NULL if S == 0
+ * int8 weights are symmetric: w = q * s per output column.  int4 weights are
+ * symmetric signed 4-bit, two per byte along the contiguous dim (low nibble =
+ * even column); the weight the layer uses is bf16(q * s) with one scale per 128
+ * rows of K. */
+typedef struct moe_weights {
+  const void* rms_gamma;
+  const void* w_router;
+  const void* router_bias;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+  const void* s_gate;
+  const void* s_up;
+  const void* s_down;
+  const void* sh_gate;
+  const void* sh_up;
+  const void* sh_down;
+  const void* sh_s_gate;
+  const void* sh_s_up;
+  const void* sh_s_down;
+} moe_weights;
+
+/* Bytes of device workspace the calls below need for this configuration (worst
+ * case over routings: T*k kept slots).  0 on an invalid configuration.  The
+ * workspace needs 256-byte alignment; its first 4 bytes are the device error
+ * word.  Fixed size and fixed addresses make the calls capturable in a CUDA
+ * graph ("MoE: dynamism the compiler cannot remove", grouped GEMM section:
+ * descriptor buffers at fixed addresses with fixed maximum sizes). */
+size_t moe_workspace_size(const moe_config* cfg);
+
+/* Zero the device error word (asynchronous). */
+moe_status moe_clear_device_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Steps a1 + a2: RMSNorm and the router GEMM.
+ *   x       [T, d] act dtype          xn_out [T, d] act dtype (bf16 or fp32), or NULL
+ *   logits  [T, E] float32 (no bias)  ws: workspace (xn is kept there when xn_out is NULL)
+ * RMSNorm is computed in double per token, xn = (x * (mean(x^2) + eps)^-1/2) * gamma,
+ * and rounded once (round-to-nearest-even) to the activation dtype.  The router
+ * multiplies that rounded xn by W_r with FP32 accumulation (picx.dev summary,
+ * Sub-study 1: router kept un-quantised, gates in FP32). */
+moe_status moe_rmsnorm_router(const moe_config* cfg, const moe_weights* w, const void* x,
+                              void* xn_out, float* logits, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Step a3: softmax + top-k + bias + renormalisation, one warp per token.
+ *   logits    [T, E] float32 router logits (bias not included)
+ *   bias      [E] float32 or NULL (see moe_bias_mode)
+ *   topk_idx  [T, k] int32: selected experts by descending key (logit, plus the
+ *             bias in LOGIT/SELECT mode), ties to the lower expert index; NaN keys
+ *             order below every number
+ *   topk_gate [T, k] float32: softmax over all E (FP32), of the biased logits in
+ *             LOGIT mode and of the plain logits otherwise; renormalised over the
+ *             k selected when cfg->renormalize
+ * Deterministic; given identical logits the indices are bit-exact to any correct
+ * implementation of the rule above. */
+moe_status moe_route(const moe_config* cfg, const float* logits, const float* bias,
+                     int32_t* topk_idx, float* topk_gate, void* stream);
+
+/* Steps a4 + a5: per-expert histogram, prefix scan, capacity and the stable
+ * permutation ("MoE Research", section 3: grouped GEMM and sorting).  No global
+ * atomics; deterministic.
+ *   topk_idx    [T*k] int32 (flat assignment a = t*k + j)
+ *   counts      [E]   int32: assignments per expert before capacity
+ *   offsets     [E+1] int32: exclusive scan of kept[e] = min(counts[e], cap)
+ *   perm_assign [T*k] int32: slot s (< offsets[E]) holds assignment a; token = a / k
+ *   slot_of     [T*k] int32: slot of assignment a, or -1 when dropped by capacity
+ *   n_dropped   [1]   int32: sum_e max(0, counts[e] - cap)
+ *   ws          workspace (only its error word is used; an id outside [0,E) sets
+ *               it, and that assignment is dropped) */
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
+                       int32_t* offsets, int32_t* perm_assign, int32_t* slot_of,
+                       int32_t* n_dropped, void* ws, size_t ws_bytes, void* stream);
+
+/* Steps a6 + a7: grouped SwiGLU expert GEMMs over the permuted tokens
+ * ("MoE: dynamism the compiler cannot remove", grouped GEMM section), plus the
+ * shared experts on every token.
+ *   xn          [T, d] act dtype (normalised activations)
+ *   offsets     [E+1], perm_assign [T*k]: as written by moe_permute
+ *   topk_gate   [T*k] float32
+ *   y_assign    [T*k, d] float32: row a = g_a * SwiGLU_{e(a)}(xn_{a/k}) for every kept
+ *               assignment a; rows of dropped assignments are left untouched
+ *   y_shared    [S, T, d] float32: SwiGLU_s(xn_t), or NULL when S == 0
+ * bf16 / int experts run on the tcgen05 tensor cores (bf16 operands, FP32
+ * accumulation; the intermediate h is rounded to bf16); fp32 experts run in FP32
+ * on the CUDA cores. */
+moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* xn,
+                           const int32_t* offsets, const int32_t* perm_assign,
+                           const float* topk_gate, float* y_assign, float* y_shared,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Step a8: combine.  out[t] = residual[t] + sum_s y_shared[s, t] +
+ * sum_{j : slot_of[t*k+j] >= 0} y_assign[t*k+j], summed in FP32 in that fixed order
+ * (deterministic), rounded to the activation dtype.
+ *   residual [T, d] act dtype or NULL (then out is the MoE delta only)
+ *   out      [T, d] out dtype */
+moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32_t* slot_of,
+                       const float* y_shared, const void* residual, void* out,
+                       void* stream);
+
+/* The whole layer: a1..a8 chained on one stream, no host synchronisation.
+ *   x [T, d] act dtype, out [T, d] out dtype.  Optional outputs (NULL to skip):
+ *   logits_out [T, E] float32, topk_idx_out [T, k] int32, counts_out [E] int32. */
+moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const void* x,
+                             void* out, void* ws, size_t ws_bytes, float* logits_out,
+                             int32_t* topk_idx_out, int32_t* counts_out, void* stream);
+
+/* moe_layer_forward with per-kernel timing marks, for profiling: events[0] is
+ * recorded on `stream` before the first kernel and events[i] right after the
+ * i-th kernel (i = 1 .. moe_layer_launch_count(cfg)).  `events` holds
+ * caller-created cudaEvent_t handles (as void*); n_events must be at least
+ * moe_layer_launch_count(cfg) + 1.  No optional outputs. */
+moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* w,
+                                      const void* x, void* out, void* ws, size_t ws_bytes,
+                                      void* const* events, int32_t n_events, void* stream);
+
+/* Synchronise `stream`, then read the device error word into *code (0 = none;
+ * 1 = expert id out of range; 2 = a pipeline wait ran out).  Returns MOE_ERR_DEVICE
+ * when the word is nonzero. */
+moe_status moe_get_device_status(const void* ws, int32_t* code, void* stream);
+
+/* Static, human-readable name of a status. */
+const char* moe_status_string(moe_status s);
+
+/* Number of kernels moe_layer_forward launches for this configuration (for
+ * launch accounting); 0 on an invalid configuration. */
+int32_t moe_layer_launch_count(const moe_config* cfg);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

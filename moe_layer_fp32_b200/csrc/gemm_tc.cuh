@@ -1,0 +1,366 @@
+// Grouped GEMM on the sm_100a tensor cores (tcgen05 + TMEM, TMA-fed) for the
+// expert FFN (a6, a7) and the router at large batches (a2).
+//
+// "MoE: dynamism the compiler cannot remove", grouped GEMM section: one launch
+// over a grid sized for the total work, each block finding its group (expert)
+// from a small descriptor array -- here the per-expert offsets written by the
+// permutation, turned into a tile prefix inside every CTA, so the grid never
+// depends on the routing and no host synchronisation is needed.
+//
+// Orientation ("swap AB"): the weights are the MMA's M side and the tokens its
+// N side, C^T[n, m] = sum_k W[k, n] * X[m, k].
+//   A = weight tile, 128 output features x 64 k, loaded from W[G][K][N]
+//       (features contiguous, i.e. MN-major) as two 64-feature TMA boxes with
+//       the 128-byte swizzle.
+//   B = token tile, BN rows x 64 k, loaded from X[R][K] (K-major), 128-byte
+//       swizzle.  Rows past the end of an expert's segment belong to the next
+//       segment or fall outside the tensor (zero fill); their columns of the
+//       accumulator are simply not stored.
+// Accumulators live in TMEM (lane = feature, column = token), double buffered
+// so that the epilogue of one tile overlaps the main loop of the next.
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 allocates TMEM and
+// its lane 0 issues tcgen05.mma; warps 2..5 drain TMEM (warp w reads lanes
+// 32*(w%4) .. +31) and run the epilogue.
+//
+// Epilogues:
+//   GATEUP  two accumulators (gate, up); h = silu(gate) * up -> bf16 H row.
+//   DOWN    y * gate(assignment) -> fp32 row perm_assign[slot] of Y (un-permuted),
+//           or the shared expert's row of Ys (gate 1).
+//   ROUTER  fp32 logits[t][e] for e < n_valid.
+#pragma once
+#include <cuda.h>
+#include "common.cuh"
+#include "kernels_small.cuh"
+
+namespace moe {
+
+enum Epi : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_ROUTER = 2 };
+
+constexpr int kTcThreads = 192;
+constexpr int kMaxGroups = 512;
+
+struct TcProblem {
+  CUtensorMap tmA;            // weights [G][K][N] bf16 (dims n, k, g), box (64, 64, 1)
+  CUtensorMap tmA2;           // second weight matrix (up) for GATEUP
+  CUtensorMap tmB;            // activations [R][K] bf16 (dims k, r), box (64, BN)
+  const int32_t* offsets;     // [G+1] segments (B rows and output rows), or nullptr
+  int G;                      // groups
+  int uniform_rows;           // rows per group when offsets == nullptr
+  int b_row_base;             // when offsets == nullptr: B row of group g's row 0 is
+  int b_group_stride;         //   b_row_base + g * b_group_stride
+  int N;                      // output features
+  int K;                      // reduction length (multiple of 64)
+  void* out;                  // H (bf16) / Y / Ys / logits (fp32)
+  size_t out_row_base;        // GATEUP / shared DOWN / ROUTER: row = base + seg + m
+  int ld_out;                 // elements per output row
+  const int32_t* perm_assign; // routed DOWN: output row = perm_assign[slot]
+  const float* gate;          // routed DOWN: scale
+  int n_valid;                // features actually stored (n < n_valid)
+};
+
+struct TcParams {
+  TcProblem prob[2];
+  int n_prob;
+  int32_t* err;
+};
+
+struct TileInfo {
+  int prob, g, m0, rows, n0;
+  int b_row;          // B row of the tile's first token
+  size_t out_seg;     // output row of the tile's first token (non-routed-DOWN cases)
+  int slot0;          // routed: slot of the tile's first token
+};
+
+template <int EPI>
+struct TcShape {
+  static constexpr int NA = (EPI == EPI_GATEUP) ? 2 : 1;
+  static constexpr uint32_t A_BYTES = 128 * 64 * 2;
+};
+
+template <int EPI, int BN>
+struct TcConfig {
+  static constexpr int NA = TcShape<EPI>::NA;
+  static constexpr uint32_t A_BYTES = TcShape<EPI>::A_BYTES;
+  static constexpr uint32_t B_BYTES = BN * 64 * 2;
+  static constexpr uint32_t STAGE_BYTES = NA * A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr uint32_t ACC_COLS = NA * BN;
+  static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS;
+  static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
+                                        : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr uint32_t IDESC = idesc_bf16_mn_k(128, BN);
+  // barriers + bookkeeping after the tiles
+  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
+  static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
+  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
+  static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
+};
+
+// Decode a linear tile id.  Tiles run over problems, then (group, m-tile) in the
+// tile prefix order, then the feature tiles innermost so that neighbouring CTAs
+// share a token tile.
+MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int tile, TileInfo& ti) {
+  int pi = 0;
+  for (; pi < p.n_prob; ++pi) {
+    const TcProblem& P = p.prob[pi];
+    const int* pre = prefix + pi * (kMaxGroups + 1);
+    const int nt = (P.N + 127) / 128;
+    const int cnt = pre[P.G] * nt;
+    if (tile < cnt) break;
+    tile -= cnt;
+  }
+  const TcProblem& P = p.prob[pi];
+  const int* pre = prefix + pi * (kMaxGroups + 1);
+  const int nt = (P.N + 127) / 128;
+  const int mt = tile / nt;
+  ti.prob = pi;
+  ti.n0 = (tile % nt) * 128;
+  const int g = find_group(pre, P.G, mt);
+  ti.g = g;
+  ti.m0 = (mt - pre[g]) * BN;
+  int seg_start, seg_rows;
+  if (P.offsets) {
+    seg_start = P.offsets[g];
+    seg_rows = P.offsets[g + 1] - seg_start;
+    ti.b_row = seg_start + ti.m0;
+  } else {
+    seg_start = g * P.uniform_rows;
+    seg_rows = P.uniform_rows;
+    ti.b_row = P.b_row_base + g * P.b_group_stride + ti.m0;
+  }
+  ti.rows = min(BN, seg_rows - ti.m0);
+  ti.slot0 = seg_start + ti.m0;
+  ti.out_seg = P.out_row_base + (size_t)seg_start + ti.m0;
+}
+
+MOE_DEV int total_tiles(const TcParams& p, const int* prefix) {
+  int tot = 0;
+  for (int pi = 0; pi < p.n_prob; ++pi) {
+    const TcProblem& P = p.prob[pi];
+    tot += prefix[pi * (kMaxGroups + 1) + P.G] * ((P.N + 127) / 128);
+  }
+  return tot;
+}
+
+MOE_DEV float silu_f(float u) { return u / (1.f + expf(-u)); }
+
+template <int EPI, int BN>
+__global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant__ TcParams p) {
+  using C = TcConfig<EPI, BN>;
+  constexpr int NA = C::NA;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
+  uint64_t* tempty_bar = tfull_bar + 2;       // [2]
+  uint64_t* drain_bar = tempty_bar + 2;       // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
+  int* prefix = reinterpret_cast<int*>(
+      reinterpret_cast<uint8_t*>(smem) + STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      issued[s] = 0;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int pi = 0; pi < p.n_prob; ++pi) {
+      tma_prefetch_desc(&p.prob[pi].tmA);
+      if (NA == 2) tma_prefetch_desc(&p.prob[pi].tmA2);
+      tma_prefetch_desc(&p.prob[pi].tmB);
+    }
+  }
+  if (warp >= 2 && warp - 2 < p.n_prob) {
+    const TcProblem& P = p.prob[warp - 2];
+    group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = total_tiles(p, prefix);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, tile, ti);
+        const TcProblem& P = p.prob[ti.prob];
+        const int kblocks = P.K / 64;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag)) { ok = false; break; }
+          uint8_t* st = tiles + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          issued[stage] = (int)phase + 1;
+          tma_load_3d(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g);
+          tma_load_3d(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g);
+          if (NA == 2) {
+            tma_load_3d(st + C::A_BYTES, &P.tmA2, &full_bar[stage], ti.n0, kb * 64, ti.g);
+            tma_load_3d(st + C::A_BYTES + 8192, &P.tmA2, &full_bar[stage], ti.n0 + 64, kb * 64,
+                        ti.g);
+          }
+          tma_load_2d(st + NA * C::A_BYTES, &P.tmB, &full_bar[stage], kb * 64, ti.b_row);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, tile, ti);
+        const int kblocks = p.prob[ti.prob].K / 64;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(tiles + stage * C::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + NA * C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // A: MN-major SW128, 16 k-rows of 128 B per MMA step; the two 64-feature
+            //    halves sit 8 KB apart (leading offset), 8-row groups 1 KB apart.
+            // B: K-major SW128, 16 k = 32 B per step, 8-row groups 1 KB apart.
+            const uint64_t bd = sw128_desc(b_addr + kk * 32, 16, 1024);
+            const uint64_t ad = sw128_desc(a_addr + kk * 2048, 8192, 1024);
+            tc_mma_f16(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0);
+            if (NA == 2) {
+              const uint64_t ad2 = sw128_desc(a_addr + C::A_BYTES + kk * 2048, 8192, 1024);
+              tc_mma_f16(d_tmem + BN, ad2, bd, C::IDESC, (kb | kk) != 0);
+            }
+          }
+          tc_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull_bar[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // wait until every MMA issued above has completed before TMEM is released
+      tc_commit(drain_bar);
+      long long t0 = clock64();
+      while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kWaitCycles) {}
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      TileInfo ti;
+      decode_tile(p, prefix, BN, tile, ti);
+      const TcProblem& P = p.prob[ti.prob];
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t t_base = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      const int n = ti.n0 + row;
+      const bool n_ok = n < P.n_valid;
+#pragma unroll 1
+      for (int c = 0; c < BN / 16; ++c) {
+        if (c * 16 >= ti.rows) break;
+        float v0[16];
+        tmem_ld16(t_base + c * 16, v0);
+        float v1[16];
+        if (NA == 2) tmem_ld16(t_base + BN + c * 16, v1);
+        tmem_wait_ld();
+        if (EPI == EPI_GATEUP) {
+          __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = c * 16 + j;
+            if (m < ti.rows && n_ok)
+              H[(ti.out_seg + m) * (size_t)P.ld_out + n] = __float2bfloat16_rn(silu_f(v0[j]) * v1[j]);
+          }
+        } else if (EPI == EPI_DOWN) {
+          float* Y = reinterpret_cast<float*>(P.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = c * 16 + j;
+            if (m < ti.rows && n_ok) {
+              if (P.perm_assign) {
+                const int as = P.perm_assign[ti.slot0 + m];
+                Y[(size_t)as * P.ld_out + n] = v0[j] * P.gate[as];
+              } else {
+                Y[(ti.out_seg + m) * (size_t)P.ld_out + n] = v0[j];
+              }
+            }
+          }
+        } else {
+          float* L = reinterpret_cast<float*>(P.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = c * 16 + j;
+            if (m < ti.rows && n_ok) L[(ti.out_seg + m) * (size_t)P.ld_out + n] = v0[j];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // copies still in flight after an abort: wait (bounded) for each stage's last load
+    for (int s = 0; s < STAGES; ++s) {
+      if (issued[s]) {
+        long long t0 = clock64();
+        while (!mbar_try_wait(&full_bar[s], (uint32_t)(issued[s] - 1)) &&
+               clock64() - t0 < kWaitCycles) {}
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace moe

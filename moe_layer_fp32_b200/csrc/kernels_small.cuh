@@ -1,0 +1,508 @@
+// CUDA-core kernels of the layer: RMSNorm (a1), the split-K router for small
+// batches (a2), softmax/top-k routing (a3), histogram + scan + permutation
+// (a4/a5), the row gather that feeds the grouped GEMM, the combine (a8), and the
+// FP32 grouped SwiGLU FFN used when the expert weights are fp32.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// block reductions
+// ---------------------------------------------------------------------------
+template <typename V>
+MOE_DEV V warp_sum(V v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+MOE_DEV float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Tile prefix over the groups of a grouped problem: prefix[g] = number of
+// BM-row tiles of groups < g.  rows(g) = off[g+1] - off[g], or `uniform` rows
+// when off == nullptr.  Called by one warp; s_off is a shared scratch of G+1.
+MOE_DEV void group_tile_prefix(const int32_t* off, int G, int uniform, int BM, int* prefix) {
+  const int lane = threadIdx.x & 31;
+  int carry = 0;
+  if (lane == 0) prefix[0] = 0;
+  for (int c = 0; c < G; c += 32) {
+    int g = c + lane;
+    int rows = 0;
+    if (g < G) rows = off ? (off[g + 1] - off[g]) : uniform;
+    int v = (rows + BM - 1) / BM;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (g < G) prefix[g + 1] = carry + v;
+    carry += __shfl_sync(0xffffffffu, v, 31);
+  }
+}
+// group of tile-row `mt`: largest g with prefix[g] <= mt
+MOE_DEV int find_group(const int* prefix, int G, int mt) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= mt) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------------------
+// a1: RMSNorm, one CTA of 256 threads per token.  The sum of squares, the
+// scale and the product are taken in double and rounded once to the
+// activation type (round-to-nearest-even).
+// ---------------------------------------------------------------------------
+MOE_DEV void store_act(__nv_bfloat16* p, double v) { *p = bf16_from_double(v); }
+MOE_DEV void store_act(float* p, double v) { *p = (float)v; }
+
+template <typename TA>
+__global__ void __launch_bounds__(256) k_rmsnorm(const TA* __restrict__ x,
+                                                 const float* __restrict__ gamma,
+                                                 TA* __restrict__ xn, int d, double eps) {
+  __shared__ double red[8];
+  const size_t row = (size_t)blockIdx.x * d;
+  double s = 0.0;
+  for (int i = threadIdx.x; i < d; i += 256) {
+    double v = (double)to_f32(x[row + i]);
+    s += v * v;
+  }
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  double tot = 0.0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const double r = 1.0 / sqrt(tot / d + eps);
+  for (int i = threadIdx.x; i < d; i += 256) {
+    double v = (double)to_f32(x[row + i]);
+    store_act(&xn[row + i], (v * r) * (double)gamma[i]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a2 (small batches): router logits split over K.  CTA (blockIdx.x, blockIdx.y)
+// computes part[y][t][e] = sum_{i in slice y} xn[t][i] * W_r[i][e] for a tile of
+// TT tokens; the route kernel adds the slices in order.
+// ---------------------------------------------------------------------------
+template <typename TA, int TT>
+__global__ void __launch_bounds__(256) k_router_split(const TA* __restrict__ xn,
+                                                      const TA* __restrict__ wr,
+                                                      float* __restrict__ part, int T, int d,
+                                                      int E, int slice) {
+  extern __shared__ float xs[];   // [TT][slice]
+  const int t0 = blockIdx.x * TT;
+  const int k0 = blockIdx.y * slice;
+  const int kn = min(slice, d - k0);
+  for (int i = threadIdx.x; i < TT * slice; i += blockDim.x) {
+    int tt = i / slice, kk = i % slice;
+    float v = 0.f;
+    if (t0 + tt < T && kk < kn) v = to_f32(xn[(size_t)(t0 + tt) * d + k0 + kk]);
+    xs[i] = v;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float acc[TT];
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) acc[tt] = 0.f;
+    for (int kk = 0; kk < kn; ++kk) {
+      float w = to_f32(wr[(size_t)(k0 + kk) * E + e]);
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt) acc[tt] = fmaf(xs[tt * slice + kk], w, acc[tt]);
+    }
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt)
+      if (t0 + tt < T) part[((size_t)blockIdx.y * T + t0 + tt) * E + e] = acc[tt];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a3: softmax + top-k + bias + renormalisation, one warp per token.  Lane l
+// holds experts l, l+32, ...  Keys are FP32 (logit, plus bias in LOGIT/SELECT
+// mode); selection order is (key descending, expert ascending), NaN keys count
+// as -inf.  Gates are the FP32 softmax over all E.
+// ---------------------------------------------------------------------------
+MOE_DEV bool key_better(float ka, int ea, float kb, int eb) {
+  return ka > kb || (ka == kb && ea < eb);
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) k_route(const float* __restrict__ part, int ns, int T,
+                                               int E, int k, const float* __restrict__ bias,
+                                               int mode, int renorm, int32_t* __restrict__ idx,
+                                               float* __restrict__ gate,
+                                               float* __restrict__ logits_out) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  float key[EPL], pin[EPL];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = -INFINITY;
+    pin[i] = -INFINITY;
+    if (e < E) {
+      float l = 0.f;
+      for (int s = 0; s < ns; ++s) l += part[((size_t)s * T + t) * E + e];
+      if (logits_out) logits_out[(size_t)t * E + e] = l;
+      float b = (mode != 0 && bias) ? bias[e] : 0.f;
+      float sk = (mode != 0) ? l + b : l;
+      pin[i] = (mode == 1) ? sk : l;
+      key[i] = isnan(sk) ? -INFINITY : sk;
+      mx = fmaxf(mx, pin[i]);
+    }
+  }
+  mx = warp_max(mx);
+  float ex[EPL];
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    ex[i] = (lane + 32 * i < E) ? expf(pin[i] - mx) : 0.f;
+    sum += ex[i];
+  }
+  sum = warp_sum(sum);
+  uint32_t taken = 0;
+  int my_e = 0;
+  float my_p = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && key_better(key[i], e, bk, be)) {
+        bk = key[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (key_better(ok, oe, bk, be)) { bk = ok; be = oe; }
+    }
+    const int owner = be & 31, slot = be >> 5;
+    float pv = 0.f;
+    if (lane == owner) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (i == slot) { taken |= 1u << i; pv = ex[i] / sum; }
+    }
+    pv = __shfl_sync(0xffffffffu, pv, owner);
+    if (lane == j) { my_e = be; my_p = pv; }
+  }
+  if (renorm) {
+    float s = warp_sum(lane < k ? my_p : 0.f);
+    my_p = my_p / s;
+  }
+  if (lane < k) {
+    idx[(size_t)t * k + lane] = my_e;
+    gate[(size_t)t * k + lane] = my_p;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a4 + a5: histogram, scan, capacity and stable permutation in one CTA of
+// 1024 threads.  Warp w owns a contiguous chunk of the flat assignments; no
+// global atomics.  Pass 1 counts per (warp, expert) with __match_any_sync;
+// a per-expert scan over warps gives each warp's base rank; a block scan over
+// experts of kept = min(count, cap) gives the offsets; pass 2 assigns
+// rank = base + running count + lanes before it with the same expert.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ idx, int n, int E,
+                                                  int cap, int32_t* __restrict__ counts,
+                                                  int32_t* __restrict__ offsets,
+                                                  int32_t* __restrict__ perm_assign,
+                                                  int32_t* __restrict__ slot_of,
+                                                  int32_t* __restrict__ n_dropped,
+                                                  int32_t* err) {
+  extern __shared__ int sm[];
+  int* cnt = sm;               // [32][E]
+  int* s_off = sm + 32 * E;    // [E]
+  __shared__ int wsum[32];
+  __shared__ int s_drop;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < 32 * E; i += 1024) cnt[i] = 0;
+  if (tid == 0) s_drop = 0;
+  __syncthreads();
+  const int chunk = (((n + 31) / 32) + 31) & ~31;
+  const int beg = warp * chunk, end = min(n, beg + chunk);
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = beg; base < end; base += 32) {
+    const int a = base + lane;
+    int e = -1;
+    if (a < end) {
+      e = idx[a];
+      if (e < 0 || e >= E) { set_error(err, DEV_BAD_EXPERT); e = -1; }
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  int tot = 0;
+  if (tid < E) {
+    for (int w = 0; w < 32; ++w) {
+      int c = cnt[w * E + tid];
+      cnt[w * E + tid] = tot;
+      tot += c;
+    }
+  }
+  const int kept = (tid < E) ? min(tot, cap) : 0;
+  if (tid < E) {
+    counts[tid] = tot;
+    if (tot > kept) atomicAdd(&s_drop, tot - kept);
+  }
+  int v = kept;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  if (lane == 31) wsum[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    wsum[lane] = w;
+  }
+  __syncthreads();
+  if (tid < E) {
+    const int excl = v - kept + (warp > 0 ? wsum[warp - 1] : 0);
+    offsets[tid] = excl;
+    s_off[tid] = excl;
+    if (tid == E - 1) offsets[E] = excl + kept;
+  }
+  if (tid == 0) *n_dropped = s_drop;
+  __syncthreads();
+  for (int base = beg; base < end; base += 32) {
+    const int a = base + lane;
+    int e = -1;
+    if (a < end) {
+      e = idx[a];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    int rank = 0;
+    if (e >= 0) rank = cnt[warp * E + e] + __popc(peers & lt);
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp * E + e] += __popc(peers);
+    __syncwarp();
+    if (a < end) {
+      if (e >= 0 && rank < cap) {
+        const int s = s_off[e] + rank;
+        slot_of[a] = s;
+        perm_assign[s] = a;
+      } else {
+        slot_of[a] = -1;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gather: xp[s] = xn[perm_assign[s] / k] for s < offsets[E]; one warp per row,
+// 16-byte vectors (d * sizeof(TA) is a multiple of 16).
+// ---------------------------------------------------------------------------
+template <typename TA>
+__global__ void __launch_bounds__(256) k_gather_rows(const TA* __restrict__ xn,
+                                                     const int32_t* __restrict__ perm_assign,
+                                                     const int32_t* __restrict__ n_rows_ptr,
+                                                     int k, int d, TA* __restrict__ xp) {
+  const int n_rows = *n_rows_ptr;
+  const int vec_per_row = d * (int)sizeof(TA) / 16;
+  const int warps = gridDim.x * 8;
+  for (int s = blockIdx.x * 8 + (threadIdx.x >> 5); s < n_rows; s += warps) {
+    const int t = perm_assign[s] / k;
+    const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)s * d);
+    for (int i = threadIdx.x & 31; i < vec_per_row; i += 32) dst[i] = src[i];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a8: combine, 4 consecutive elements per thread.  out = residual + shared
+// experts (s ascending) + kept assignments (j ascending), FP32.
+// ---------------------------------------------------------------------------
+MOE_DEV void load4(const float* p, float (&v)[4]) {
+  float4 q = *reinterpret_cast<const float4*>(p);
+  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+}
+MOE_DEV void load4(const __nv_bfloat16* p, float (&v)[4]) {
+  uint2 q = *reinterpret_cast<const uint2*>(p);
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&q.x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&q.y);
+  v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
+}
+MOE_DEV void store4(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+MOE_DEV void store4(__nv_bfloat16* p, const float (&v)[4]) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 q;
+  q.x = *reinterpret_cast<uint32_t*>(&a);
+  q.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = q;
+}
+
+template <typename TA, typename TO>
+__global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y,
+                                                 const int32_t* __restrict__ slot_of,
+                                                 const float* __restrict__ ys, int S,
+                                                 const TA* __restrict__ res, TO* __restrict__ out,
+                                                 int T, int d, int k) {
+  const int q = d / 4;
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (size_t)T * q) return;
+  const int t = (int)(i / q);
+  const int c = (int)(i % q) * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (res) load4(res + (size_t)t * d + c, acc);
+  for (int s = 0; s < S; ++s) {
+    float v[4];
+    load4(ys + ((size_t)s * T + t) * d + c, v);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] += v[u];
+  }
+  for (int j = 0; j < k; ++j) {
+    const size_t a = (size_t)t * k + j;
+    if (slot_of[a] >= 0) {
+      float v[4];
+      load4(y + a * d + c, v);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] += v[u];
+    }
+  }
+  store4(out + (size_t)t * d + c, acc);
+}
+
+// ---------------------------------------------------------------------------
+// FP32 grouped SwiGLU FFN on the CUDA cores (fp32 expert weights).
+// A CTA of 128 threads takes a tile of up to RB rows of one group and 128
+// output features; each thread owns one feature.  Groups come from the routed
+// segments (offsets) followed by the shared experts (T rows each).
+// ---------------------------------------------------------------------------
+struct SimtArgs {
+  const float* xn;           // [T, d] (rows gathered through perm_assign)
+  const int32_t* offsets;    // [E+1]
+  const int32_t* perm_assign;
+  const float* gate;         // [T*k]
+  const float* wg; const float* wu; const float* wd;        // routed [E,...]
+  const float* swg; const float* swu; const float* swd;     // shared [S,...]
+  float* h;                  // [T*k + S*T, f]
+  float* y;                  // [T*k, d]
+  float* ys;                 // [S, T, d]
+  int T, d, f, k, E, S;
+};
+
+constexpr int kSimtRB = 8;
+constexpr int kSimtKC = 256;
+
+template <bool DOWN>
+__global__ void __launch_bounds__(128) k_simt_ffn(SimtArgs a) {
+  __shared__ int prefix[520];
+  __shared__ float xs[kSimtRB][kSimtKC];
+  __shared__ int rows_src[kSimtRB];
+  const int N = DOWN ? a.d : a.f;
+  const int K = DOWN ? a.f : a.d;
+  const int n_tiles = (N + 127) / 128;
+  if (threadIdx.x < 32) group_tile_prefix(a.offsets, a.E, 0, kSimtRB, prefix);
+  __syncthreads();
+  const int routed_mt = prefix[a.E];
+  const int shared_mt_per = (a.T + kSimtRB - 1) / kSimtRB;
+  const int total = (routed_mt + a.S * shared_mt_per) * n_tiles;
+  for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    const int mt = tile / n_tiles, nt = tile % n_tiles;
+    const bool shared = mt >= routed_mt;
+    int g, r0, rows;
+    if (!shared) {
+      g = find_group(prefix, a.E, mt);
+      r0 = a.offsets[g] + (mt - prefix[g]) * kSimtRB;
+      rows = min(kSimtRB, a.offsets[g + 1] - r0);
+    } else {
+      const int m2 = mt - routed_mt;
+      g = m2 / shared_mt_per;
+      r0 = (m2 % shared_mt_per) * kSimtRB;
+      rows = min(kSimtRB, a.T - r0);
+    }
+    __syncthreads();
+    if (threadIdx.x < kSimtRB) {
+      int r = threadIdx.x, src = -1;
+      if (r < rows) {
+        if (DOWN) src = shared ? a.T * a.k + g * a.T + r0 + r : r0 + r;     // row of h
+        else src = shared ? r0 + r : a.perm_assign[r0 + r] / a.k;          // row of xn
+      }
+      rows_src[r] = src;
+    }
+    const float* W;
+    if (DOWN) W = shared ? a.swd + (size_t)g * a.f * a.d : a.wd + (size_t)g * a.f * a.d;
+    else W = nullptr;
+    const float* Wg = shared ? a.swg + (size_t)g * a.d * a.f : a.wg + (size_t)g * a.d * a.f;
+    const float* Wu = shared ? a.swu + (size_t)g * a.d * a.f : a.wu + (size_t)g * a.d * a.f;
+    const int n = nt * 128 + threadIdx.x;
+    float acc0[kSimtRB], acc1[kSimtRB];
+#pragma unroll
+    for (int r = 0; r < kSimtRB; ++r) { acc0[r] = 0.f; acc1[r] = 0.f; }
+    for (int k0 = 0; k0 < K; k0 += kSimtKC) {
+      const int kn = min(kSimtKC, K - k0);
+      __syncthreads();
+      for (int i = threadIdx.x; i < kSimtRB * kSimtKC; i += 128) {
+        const int r = i / kSimtKC, kk = i % kSimtKC;
+        float v = 0.f;
+        if (rows_src[r] >= 0 && kk < kn) {
+          const float* src = DOWN ? a.h + (size_t)rows_src[r] * a.f : a.xn + (size_t)rows_src[r] * a.d;
+          v = src[k0 + kk];
+        }
+        xs[r][kk] = v;
+      }
+      __syncthreads();
+      if (n < N) {
+        for (int kk = 0; kk < kn; ++kk) {
+          if (DOWN) {
+            const float w = W[(size_t)(k0 + kk) * N + n];
+#pragma unroll
+            for (int r = 0; r < kSimtRB; ++r) acc0[r] = fmaf(xs[r][kk], w, acc0[r]);
+          } else {
+            const float wg = Wg[(size_t)(k0 + kk) * N + n];
+            const float wu = Wu[(size_t)(k0 + kk) * N + n];
+#pragma unroll
+            for (int r = 0; r < kSimtRB; ++r) {
+              acc0[r] = fmaf(xs[r][kk], wg, acc0[r]);
+              acc1[r] = fmaf(xs[r][kk], wu, acc1[r]);
+            }
+          }
+        }
+      }
+    }
+    if (n < N) {
+      for (int r = 0; r < rows; ++r) {
+        if (DOWN) {
+          if (shared) {
+            a.ys[((size_t)g * a.T + r0 + r) * a.d + n] = acc0[r];
+          } else {
+            const int as = a.perm_assign[r0 + r];
+            a.y[(size_t)as * a.d + n] = a.gate[as] * acc0[r];
+          }
+        } else {
+          const float u = acc0[r];
+          const float hv = (u / (1.f + expf(-u))) * acc1[r];
+          const size_t hrow = shared ? (size_t)a.T * a.k + (size_t)g * a.T + r0 + r : (size_t)(r0 + r);
+          a.h[hrow * a.f + n] = hv;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,608 @@
+// Host side of the C ABI declared in include/moe.h: argument validation,
+// workspace layout, TMA tensor-map encoding and the kernel launches.  All
+// launches go to the caller's stream; nothing here synchronises except
+// moe_get_device_status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <climits>
+#include <cmath>
+#include <cstring>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "kernels_small.cuh"
+#include "gemm_tc.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+inline bool tc_experts(const moe_config* c) { return c->expert_dtype != MOE_F32; }
+// the router runs on the tensor cores from this batch size up (bf16 router)
+constexpr int kTcRouterMinT = 128;
+inline bool tc_router(const moe_config* c) {
+  return c->router_dtype == MOE_BF16 && c->T >= kTcRouterMinT;
+}
+constexpr int kRouterSlice = 128;
+constexpr int kRouterTT = 8;
+inline int router_splits(const moe_config* c) {
+  if (tc_router(c)) return 1;
+  int ns = (c->d + kRouterSlice - 1) / kRouterSlice;
+  int ttiles = (c->T + kRouterTT - 1) / kRouterTT;
+  // enough CTAs to cover the SMs a couple of times, no more slices than needed
+  int want = (296 + ttiles - 1) / ttiles;
+  return ns < want ? ns : (want < 1 ? 1 : want);
+}
+inline int router_slice(const moe_config* c, int ns) {
+  int s = (c->d + ns - 1) / ns;
+  return (s + 7) / 8 * 8;
+}
+
+struct Layout {
+  size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, xp, h, y, ys, total;
+  int ns;
+};
+
+moe_status validate(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID;
+  if (c->T < 1 || c->d < 8 || c->d % 8 || c->E < 1 || c->E > kMaxGroups || c->k < 1 ||
+      c->k > c->E || c->k > 32 || c->f < 1 || c->n_shared < 0 || c->n_shared > 8)
+    return MOE_ERR_INVALID;
+  if ((long long)c->T * c->k > (1LL << 30)) return MOE_ERR_INVALID;
+  if (c->act_dtype != MOE_BF16 && c->act_dtype != MOE_F32) return MOE_ERR_INVALID;
+  if (c->out_dtype != MOE_BF16 && c->out_dtype != MOE_F32) return MOE_ERR_INVALID;
+  if (c->act_dtype == MOE_F32 && c->out_dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
+  if (c->router_dtype != c->act_dtype) return MOE_ERR_UNSUPPORTED;
+  if (c->bias_mode < MOE_BIAS_NONE || c->bias_mode > MOE_BIAS_SELECT) return MOE_ERR_INVALID;
+  if (!(c->rms_eps >= 0.f) || !std::isfinite(c->capacity_factor)) return MOE_ERR_INVALID;
+  switch (c->expert_dtype) {
+    case MOE_F32:
+      if (c->act_dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
+      break;
+    case MOE_BF16:
+      if (c->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+      if (c->d % 128 || c->f % 128 || c->E % 8) return MOE_ERR_UNSUPPORTED;
+      break;
+    case MOE_INT8:
+    case MOE_INT4:
+      return MOE_ERR_UNSUPPORTED;
+    default:
+      return MOE_ERR_INVALID;
+  }
+  return MOE_OK;
+}
+
+Layout layout(const moe_config* c) {
+  Layout L{};
+  const size_t T = c->T, d = c->d, E = c->E, k = c->k, f = c->f, S = c->n_shared;
+  const size_t act = c->act_dtype == MOE_BF16 ? 2 : 4;
+  const size_t hb = tc_experts(c) ? 2 : 4;
+  L.ns = router_splits(c);
+  size_t o = 0;
+  L.err = o;      o = align_up(o + 16);
+  L.xn = o;       o = align_up(o + T * d * act);
+  L.part = o;     o = align_up(o + (size_t)L.ns * T * E * 4);
+  L.idx = o;      o = align_up(o + T * k * 4);
+  L.gate = o;     o = align_up(o + T * k * 4);
+  L.counts = o;   o = align_up(o + E * 4);
+  L.offsets = o;  o = align_up(o + (E + 1) * 4);
+  L.perm = o;     o = align_up(o + T * k * 4);
+  L.slot = o;     o = align_up(o + T * k * 4);
+  L.dropped = o;  o = align_up(o + 16);
+  L.xp = o;       o = align_up(o + (tc_experts(c) ? T * k * d * act : 0));
+  L.h = o;        o = align_up(o + (T * k + S * T) * f * hb);
+  L.y = o;        o = align_up(o + T * k * d * 4);
+  L.ys = o;       o = align_up(o + S * T * d * 4);
+  L.total = o;
+  return L;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(ws) + off); }
+
+inline cudaStream_t S_(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Optional per-kernel timing marks: event i+1 is recorded after the i-th launch.
+struct Marks {
+  cudaEvent_t* ev = nullptr;
+  int n = 0, i = 0;
+  void mark(cudaStream_t st) {
+    if (ev && i < n) cudaEventRecord(ev[i++], st);
+  }
+};
+
+moe_status check_launch() {
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status check_ws(const moe_config* c, void* ws, size_t ws_bytes) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < layout(c).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// ----------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// weights [G][K][N] bf16, N contiguous; box 64 features x 64 k x 1
+bool map_weights(CUtensorMap* m, const void* base, int G, int K, int N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)G};
+  cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)K * N * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// activations [R][K] bf16, K contiguous; box 64 k x BN rows
+bool map_rows(CUtensorMap* m, const void* base, int R, int K, int BN) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)R};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)BN};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI, int BN>
+moe_status launch_tc(const TcParams& p, cudaStream_t st) {
+  using C = TcConfig<EPI, BN>;
+  auto kern = k_tc_gemm<EPI, BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  kern<<<num_sms(), kTcThreads, C::SMEM_BYTES, st>>>(p);
+  return check_launch();
+}
+
+template <int EPI>
+moe_status launch_tc_bn(int bn, const TcParams& p, cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_tc<EPI, 16>(p, st);
+    case 32: return launch_tc<EPI, 32>(p, st);
+    case 64: return launch_tc<EPI, 64>(p, st);
+    default: return launch_tc<EPI, 128>(p, st);
+  }
+}
+
+// token-tile width of the expert GEMMs from the mean rows per expert
+int pick_bn(const moe_config* c) {
+  double mean = (double)c->T * c->k / c->E;
+  if (mean <= 16) return 16;
+  if (mean <= 32) return 32;
+  if (mean <= 64) return 64;
+  return 128;
+}
+
+int capacity_rows(const moe_config* c) {
+  if (!(c->capacity_factor > 0.f)) return INT_MAX;
+  double v = std::ceil((double)c->capacity_factor * c->T * c->k / c->E);
+  return v >= (double)INT_MAX ? INT_MAX : (int)v;
+}
+
+// ----------------------------------------------------------------- the steps
+moe_status run_rmsnorm(const moe_config* c, const moe_weights* w, const void* x, void* xn,
+                       cudaStream_t st) {
+  if (c->act_dtype == MOE_BF16)
+    k_rmsnorm<__nv_bfloat16><<<c->T, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(w->rms_gamma),
+        static_cast<__nv_bfloat16*>(xn), c->d, (double)c->rms_eps);
+  else
+    k_rmsnorm<float><<<c->T, 256, 0, st>>>(static_cast<const float*>(x),
+                                           static_cast<const float*>(w->rms_gamma),
+                                           static_cast<float*>(xn), c->d, (double)c->rms_eps);
+  return check_launch();
+}
+
+moe_status run_router(const moe_config* c, const moe_weights* w, const void* xn, float* part,
+                      int ns, int32_t* err, cudaStream_t st) {
+  if (tc_router(c)) {
+    TcParams p{};
+    TcProblem& P = p.prob[0];
+    if (!map_weights(&P.tmA, w->w_router, 1, c->d, c->E)) return MOE_ERR_CUDA;
+    P.tmA2 = P.tmA;
+    if (!map_rows(&P.tmB, xn, c->T, c->d, 128)) return MOE_ERR_CUDA;
+    P.offsets = nullptr;
+    P.G = 1;
+    P.uniform_rows = c->T;
+    P.b_row_base = 0;
+    P.b_group_stride = 0;
+    P.N = c->E;
+    P.K = c->d;
+    P.out = part;
+    P.out_row_base = 0;
+    P.ld_out = c->E;
+    P.n_valid = c->E;
+    p.n_prob = 1;
+    p.err = err;
+    return launch_tc<EPI_ROUTER, 128>(p, st);
+  }
+  const int slice = router_slice(c, ns);
+  dim3 grid((c->T + kRouterTT - 1) / kRouterTT, ns);
+  const size_t smem = (size_t)kRouterTT * slice * 4;
+  int threads = c->E >= 256 ? 256 : ((c->E + 31) / 32) * 32;
+  if (c->act_dtype == MOE_BF16)
+    k_router_split<__nv_bfloat16, kRouterTT><<<grid, threads, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(xn), static_cast<const __nv_bfloat16*>(w->w_router),
+        part, c->T, c->d, c->E, slice);
+  else
+    k_router_split<float, kRouterTT><<<grid, threads, smem, st>>>(
+        static_cast<const float*>(xn), static_cast<const float*>(w->w_router), part, c->T,
+        c->d, c->E, slice);
+  return check_launch();
+}
+
+moe_status run_route(const moe_config* c, const float* part, int ns, const float* bias,
+                     int32_t* idx, float* gate, float* logits_out, cudaStream_t st) {
+  const int blocks = (c->T + 7) / 8;
+  const int mode = c->bias_mode;
+  if (mode != MOE_BIAS_NONE && !bias) return MOE_ERR_INVALID;
+#define MOE_ROUTE(EPL)                                                                     \
+  k_route<EPL><<<blocks, 256, 0, st>>>(part, ns, c->T, c->E, c->k, bias, mode,             \
+                                       c->renormalize ? 1 : 0, idx, gate, logits_out)
+  if (c->E <= 32) MOE_ROUTE(1);
+  else if (c->E <= 64) MOE_ROUTE(2);
+  else if (c->E <= 128) MOE_ROUTE(4);
+  else if (c->E <= 256) MOE_ROUTE(8);
+  else MOE_ROUTE(16);
+#undef MOE_ROUTE
+  return check_launch();
+}
+
+moe_status run_permute(const moe_config* c, const int32_t* idx, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* slot, int32_t* dropped,
+                       int32_t* err, cudaStream_t st) {
+  const size_t smem = (size_t)33 * c->E * 4;
+  if (cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  k_permute<<<1, 1024, smem, st>>>(idx, c->T * c->k, c->E, capacity_rows(c), counts, offsets,
+                                   perm, slot, dropped, err);
+  return check_launch();
+}
+
+moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
+                   const int32_t* offsets, const int32_t* perm, const float* gate, float* y,
+                   float* ys, void* ws, cudaStream_t st, Marks* mk = nullptr) {
+  Marks none;
+  if (!mk) mk = &none;
+  const Layout L = layout(c);
+  int32_t* err = at<int32_t>(ws, L.err);
+  const int T = c->T, k = c->k, S = c->n_shared;
+  if (!w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID;
+  if (S > 0 && (!w->sh_gate || !w->sh_up || !w->sh_down || !ys)) return MOE_ERR_INVALID;
+  if (!tc_experts(c)) {
+    SimtArgs a{};
+    a.xn = static_cast<const float*>(xn);
+    a.offsets = offsets;
+    a.perm_assign = perm;
+    a.gate = gate;
+    a.wg = static_cast<const float*>(w->w_gate);
+    a.wu = static_cast<const float*>(w->w_up);
+    a.wd = static_cast<const float*>(w->w_down);
+    a.swg = static_cast<const float*>(w->sh_gate);
+    a.swu = static_cast<const float*>(w->sh_up);
+    a.swd = static_cast<const float*>(w->sh_down);
+    a.h = at<float>(ws, L.h);
+    a.y = y;
+    a.ys = ys;
+    a.T = T; a.d = c->d; a.f = c->f; a.k = k; a.E = c->E; a.S = S;
+    const int grid = 2 * num_sms();
+    k_simt_ffn<false><<<grid, 128, 0, st>>>(a);
+    moe_status s = check_launch();
+    if (s != MOE_OK) return s;
+    mk->mark(st);
+    k_simt_ffn<true><<<grid, 128, 0, st>>>(a);
+    s = check_launch();
+    mk->mark(st);
+    return s;
+  }
+  // bf16 experts: gather the routed rows, then gate/up and down on the tensor cores
+  __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
+  k_gather_rows<__nv_bfloat16><<<2 * num_sms(), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
+  moe_status s = check_launch();
+  if (s != MOE_OK) return s;
+  mk->mark(st);
+  const int bn = pick_bn(c);
+  const int R = T * k;
+  {
+    TcParams p{};
+    TcProblem& P = p.prob[0];
+    if (!map_weights(&P.tmA, w->w_gate, c->E, c->d, c->f)) return MOE_ERR_CUDA;
+    if (!map_weights(&P.tmA2, w->w_up, c->E, c->d, c->f)) return MOE_ERR_CUDA;
+    if (!map_rows(&P.tmB, xp, R, c->d, bn)) return MOE_ERR_CUDA;
+    P.offsets = offsets;
+    P.G = c->E;
+    P.N = c->f;
+    P.K = c->d;
+    P.out = h;
+    P.out_row_base = 0;
+    P.ld_out = c->f;
+    P.n_valid = c->f;
+    p.n_prob = 1;
+    if (S > 0) {
+      TcProblem& Q = p.prob[1];
+      if (!map_weights(&Q.tmA, w->sh_gate, S, c->d, c->f)) return MOE_ERR_CUDA;
+      if (!map_weights(&Q.tmA2, w->sh_up, S, c->d, c->f)) return MOE_ERR_CUDA;
+      if (!map_rows(&Q.tmB, xn, T, c->d, bn)) return MOE_ERR_CUDA;
+      Q.offsets = nullptr;
+      Q.G = S;
+      Q.uniform_rows = T;
+      Q.b_row_base = 0;
+      Q.b_group_stride = 0;
+      Q.N = c->f;
+      Q.K = c->d;
+      Q.out = h;
+      Q.out_row_base = (size_t)R;
+      Q.ld_out = c->f;
+      Q.n_valid = c->f;
+      p.n_prob = 2;
+    }
+    p.err = err;
+    s = launch_tc_bn<EPI_GATEUP>(bn, p, st);
+    if (s != MOE_OK) return s;
+    mk->mark(st);
+  }
+  {
+    TcParams p{};
+    TcProblem& P = p.prob[0];
+    if (!map_weights(&P.tmA, w->w_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
+    P.tmA2 = P.tmA;
+    if (!map_rows(&P.tmB, h, R + S * T, c->f, bn)) return MOE_ERR_CUDA;
+    P.offsets = offsets;
+    P.G = c->E;
+    P.N = c->d;
+    P.K = c->f;
+    P.out = y;
+    P.out_row_base = 0;
+    P.ld_out = c->d;
+    P.perm_assign = perm;
+    P.gate = gate;
+    P.n_valid = c->d;
+    p.n_prob = 1;
+    if (S > 0) {
+      TcProblem& Q = p.prob[1];
+      if (!map_weights(&Q.tmA, w->sh_down, S, c->f, c->d)) return MOE_ERR_CUDA;
+      Q.tmA2 = Q.tmA;
+      Q.tmB = P.tmB;
+      Q.offsets = nullptr;
+      Q.G = S;
+      Q.uniform_rows = T;
+      Q.b_row_base = R;
+      Q.b_group_stride = T;
+      Q.N = c->d;
+      Q.K = c->f;
+      Q.out = ys;
+      Q.out_row_base = 0;
+      Q.ld_out = c->d;
+      Q.perm_assign = nullptr;
+      Q.gate = nullptr;
+      Q.n_valid = c->d;
+      p.n_prob = 2;
+    }
+    p.err = err;
+    s = launch_tc_bn<EPI_DOWN>(bn, p, st);
+    mk->mark(st);
+  }
+  return s;
+}
+
+moe_status run_combine(const moe_config* c, const float* y, const int32_t* slot,
+                       const float* ys, const void* res, void* out, cudaStream_t st) {
+  const size_t n = (size_t)c->T * (c->d / 4);
+  const int blocks = (int)((n + 255) / 256);
+  if (c->act_dtype == MOE_BF16 && c->out_dtype == MOE_BF16)
+    k_combine<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, st>>>(
+        y, slot, ys, c->n_shared, static_cast<const __nv_bfloat16*>(res),
+        static_cast<__nv_bfloat16*>(out), c->T, c->d, c->k);
+  else if (c->act_dtype == MOE_BF16)
+    k_combine<__nv_bfloat16, float><<<blocks, 256, 0, st>>>(
+        y, slot, ys, c->n_shared, static_cast<const __nv_bfloat16*>(res),
+        static_cast<float*>(out), c->T, c->d, c->k);
+  else
+    k_combine<float, float><<<blocks, 256, 0, st>>>(y, slot, ys, c->n_shared,
+                                                    static_cast<const float*>(res),
+                                                    static_cast<float*>(out), c->T, c->d, c->k);
+  return check_launch();
+}
+
+moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const void* x,
+                              void* out, void* ws, size_t ws_bytes, float* logits_out,
+                              int32_t* topk_idx_out, int32_t* counts_out, cudaStream_t st,
+                              Marks* mk) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!w || !x || !out || !w->rms_gamma || !w->w_router) return MOE_ERR_INVALID;
+  if (cfg->bias_mode != MOE_BIAS_NONE && !w->router_bias) return MOE_ERR_INVALID;
+  if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+  const Layout L = layout(cfg);
+  int32_t* err = at<int32_t>(ws, L.err);
+  void* xn = at<void>(ws, L.xn);
+  float* part = at<float>(ws, L.part);
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+  float* gate = at<float>(ws, L.gate);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* slot = at<int32_t>(ws, L.slot);
+  float* y = at<float>(ws, L.y);
+  float* ys = cfg->n_shared ? at<float>(ws, L.ys) : nullptr;
+  mk->mark(st);
+  if ((s = run_rmsnorm(cfg, w, x, xn, st)) != MOE_OK) return s;
+  mk->mark(st);
+  if ((s = run_router(cfg, w, xn, part, L.ns, err, st)) != MOE_OK) return s;
+  mk->mark(st);
+  if ((s = run_route(cfg, part, L.ns, static_cast<const float*>(w->router_bias), idx, gate,
+                     logits_out, st)) != MOE_OK)
+    return s;
+  mk->mark(st);
+  if ((s = run_permute(cfg, idx, counts, offsets, perm, slot, at<int32_t>(ws, L.dropped), err,
+                       st)) != MOE_OK)
+    return s;
+  mk->mark(st);
+  if ((s = run_ffn(cfg, w, xn, offsets, perm, gate, y, ys, ws, st, mk)) != MOE_OK) return s;
+  s = run_combine(cfg, y, slot, ys, x, out, st);
+  mk->mark(st);
+  return s;
+}
+
+// =================================================================== C ABI
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return layout(cfg).total;
+}
+
+moe_status moe_clear_device_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 16) return MOE_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, 16, S_(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_rmsnorm_router(const moe_config* cfg, const moe_weights* w, const void* x,
+                              void* xn_out, float* logits, void* ws, size_t ws_bytes,
+                              void* stream) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!w || !x || !logits || !w->rms_gamma || !w->w_router) return MOE_ERR_INVALID;
+  if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+  const Layout L = layout(cfg);
+  cudaStream_t st = S_(stream);
+  void* xn = xn_out ? xn_out : at<void>(ws, L.xn);
+  if ((s = run_rmsnorm(cfg, w, x, xn, st)) != MOE_OK) return s;
+  float* part = at<float>(ws, L.part);
+  if ((s = run_router(cfg, w, xn, part, L.ns, at<int32_t>(ws, L.err), st)) != MOE_OK) return s;
+  // add the K slices in order into logits (the route kernel's reduction, no selection)
+  if (L.ns == 1 && tc_router(cfg))
+    return cudaMemcpyAsync(logits, part, (size_t)cfg->T * cfg->E * 4, cudaMemcpyDeviceToDevice,
+                           st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  moe_config c1 = *cfg;
+  c1.bias_mode = MOE_BIAS_NONE;
+  return run_route(&c1, part, L.ns, nullptr, at<int32_t>(ws, L.idx), at<float>(ws, L.gate),
+                   logits, st);
+}
+
+moe_status moe_route(const moe_config* cfg, const float* logits, const float* bias,
+                     int32_t* topk_idx, float* topk_gate, void* stream) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!logits || !topk_idx || !topk_gate) return MOE_ERR_INVALID;
+  return run_route(cfg, logits, 1, bias, topk_idx, topk_gate, nullptr, S_(stream));
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
+                       int32_t* offsets, int32_t* perm_assign, int32_t* slot_of,
+                       int32_t* n_dropped, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!topk_idx || !counts || !offsets || !perm_assign || !slot_of || !n_dropped)
+    return MOE_ERR_INVALID;
+  if (!ws || ws_bytes < 16 || reinterpret_cast<uintptr_t>(ws) % kAlign) return MOE_ERR_WORKSPACE;
+  return run_permute(cfg, topk_idx, counts, offsets, perm_assign, slot_of, n_dropped,
+                     static_cast<int32_t*>(ws), S_(stream));
+}
+
+moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* xn,
+                           const int32_t* offsets, const int32_t* perm_assign,
+                           const float* topk_gate, float* y_assign, float* y_shared, void* ws,
+                           size_t ws_bytes, void* stream) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!w || !xn || !offsets || !perm_assign || !topk_gate || !y_assign) return MOE_ERR_INVALID;
+  if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+  return run_ffn(cfg, w, xn, offsets, perm_assign, topk_gate, y_assign, y_shared, ws,
+                 S_(stream));
+}
+
+moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32_t* slot_of,
+                       const float* y_shared, const void* residual, void* out, void* stream) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!y_assign || !slot_of || !out || (cfg->n_shared > 0 && !y_shared)) return MOE_ERR_INVALID;
+  return run_combine(cfg, y_assign, slot_of, y_shared, residual, out, S_(stream));
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const void* x,
+                             void* out, void* ws, size_t ws_bytes, float* logits_out,
+                             int32_t* topk_idx_out, int32_t* counts_out, void* stream) {
+  Marks none;
+  return layer_forward_impl(cfg, w, x, out, ws, ws_bytes, logits_out, topk_idx_out, counts_out,
+                            S_(stream), &none);
+}
+
+moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* w,
+                                      const void* x, void* out, void* ws, size_t ws_bytes,
+                                      void* const* events, int32_t n_events, void* stream) {
+  if (!events || n_events < moe_layer_launch_count(cfg) + 1) return MOE_ERR_INVALID;
+  Marks mk;
+  mk.ev = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
+  mk.n = n_events;
+  return layer_forward_impl(cfg, w, x, out, ws, ws_bytes, nullptr, nullptr, nullptr, S_(stream),
+                            &mk);
+}
+
+moe_status moe_get_device_status(const void* ws, int32_t* code, void* stream) {
+  if (!ws || !code) return MOE_ERR_INVALID;
+  if (cudaStreamSynchronize(S_(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  *code = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID: return "MOE_ERR_INVALID";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int32_t moe_layer_launch_count(const moe_config* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  // rmsnorm, router, route, permute, [gather], gate/up, down, combine
+  return tc_experts(cfg) ? 8 : 7;
+}
+
+}  // extern "C"

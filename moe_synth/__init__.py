@@ -33,7 +33,9 @@ scales are ``[E, d/G, f]`` (gate/up) and ``[E, f/G, d]`` (down).
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import os
 from dataclasses import dataclass, field
 from typing import Dict, Optional, Tuple
 
@@ -197,13 +199,18 @@ def make_expert_stack(shape: LayerShape, which: str, shared: bool = False,
                       experts: Optional[range] = None, device="cpu"):
     """Stacked weights (and scales, None for f32/bf16) for one matrix kind."""
     n = shape.n_shared if shared else shape.E
-    ids = range(n) if experts is None else experts
+    ids = list(range(n) if experts is None else experts)
     ws, ss = [], []
-    for e in ids:
-        q, s = _encode(shape, master_expert(shape, which, e, shared))
-        ws.append(q.to(device))
-        if s is not None:
-            ss.append(s.to(device))
+
+    def one(e):
+        return _encode(shape, master_expert(shape, which, e, shared))
+
+    # experts draw from independent streams: generate them on a few host threads
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        for q, s in ex.map(one, ids):
+            ws.append(q.to(device))
+            if s is not None:
+                ss.append(s.to(device))
     W = torch.stack(ws) if ws else None
     S = torch.stack(ss) if ss else None
     return W, S

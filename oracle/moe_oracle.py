@@ -265,21 +265,17 @@ def expert_ffn(X, wg, wu, wd) -> np.ndarray:
 # the whole layer
 # ---------------------------------------------------------------------------
 class Weights:
-    """Expert weights with lazy, cached per-expert dequantisation."""
+    """Expert weights (stacked per expert); each matrix is converted to float64
+    (dequantised for int8 / int4) when it is used."""
 
     def __init__(self, expert_dtype: str, group: int, gate, up, down,
                  s_gate=None, s_up=None, s_down=None):
         self.dt, self.group = expert_dtype, group
         self.src = dict(gate=(gate, s_gate), up=(up, s_up), down=(down, s_down))
-        self.cache = {}
 
     def get(self, which: str, e: int) -> np.ndarray:
-        key = (which, e)
-        if key not in self.cache:
-            w, s = self.src[which]
-            self.cache[key] = expert_matrix(w[e], None if s is None else s[e],
-                                            self.dt, self.group)
-        return self.cache[key]
+        w, s = self.src[which]
+        return expert_matrix(w[e], None if s is None else s[e], self.dt, self.group)
 
     def ffn(self, e: int, X) -> np.ndarray:
         return expert_ffn(X, self.get("gate", e), self.get("up", e), self.get("down", e))

@@ -1,0 +1,299 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Every test here needs a B200."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_layer_fp32_b200 as M
+import moe_synth
+from moe_synth import LayerShape
+from oracle import moe_oracle as O
+from tests.layer_check import (DELTA_GUARD, ROUTE_MARGIN, TOL, inputs_on_device, run_layer,
+                               sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+# small shapes: several tiles, ragged tails, every routing option
+SMALL = {
+    "bf16_plain": LayerShape("bf16_plain", d=256, E=16, k=4, f=256, seed=11),
+    "bf16_shared_cap": LayerShape("bf16_shared_cap", d=384, E=32, k=6, f=384, n_shared=2,
+                                  capacity_factor=1.25, bias_mode="logit", seed=12),
+    "bf16_select_tc_router": LayerShape("bf16_select", d=256, E=64, k=8, f=128, n_shared=1,
+                                        bias_mode="select", renormalize=False, seed=13),
+    "bf16_prefill_tiles": LayerShape("bf16_prefill", d=512, E=8, k=2, f=640, seed=14),
+    "f32_tiny": moe_synth.PRESETS["tiny"],
+}
+SMALL_T = {"bf16_plain": 100, "bf16_shared_cap": 77, "bf16_select_tc_router": 200,
+           "bf16_prefill_tiles": 1000, "f32_tiny": 64}
+
+
+@pytest.fixture(autouse=True)
+def _dev(cuda_device):
+    yield
+
+
+def tdev(a, dtype):
+    return torch.as_tensor(a, dtype=dtype).cuda()
+
+
+# --------------------------------------------------------------------- a1 + a2
+@pytest.mark.parametrize("name", ["bf16_plain", "bf16_select_tc_router", "f32_tiny"])
+def test_rmsnorm_bitexact_and_router(name):
+    sh, T = SMALL[name], SMALL_T[name]
+    li, x, dli, dx = inputs_on_device(sh, T)
+    cfg = M.make_config(sh, T)
+    ws = M.alloc_workspace(cfg)
+    act = torch.bfloat16 if sh.act == "bf16" else torch.float32
+    xn = torch.empty(T, sh.d, dtype=act, device="cuda")
+    logits = torch.empty(T, sh.E, dtype=torch.float32, device="cuda")
+    M.moe_rmsnorm_router(cfg, M.make_weights(dli), dx, xn, logits, ws)
+    ref_xn = O.rmsnorm(x.float().numpy(), li.gamma.numpy(), sh.rms_eps, sh.act)
+    np.testing.assert_array_equal(xn.float().cpu().numpy().astype(np.float64), ref_xn)
+    wr = li.w_router.float().numpy().astype(np.float64)
+    ref_l = O.router_logits(ref_xn, wr)
+    # FP32 accumulation of d exact products: |err| <= d 2^-24 sum|xn_i w_ie|
+    bound = sh.d * 2.0 ** -24 * (np.abs(ref_xn) @ np.abs(wr)) + 1e-30
+    assert np.all(np.abs(logits.cpu().numpy() - ref_l) <= bound)
+
+
+# --------------------------------------------------------------------- a3
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 8), (64, 6), (128, 8), (256, 8), (512, 32), (33, 1)])
+@pytest.mark.parametrize("mode", ["none", "logit", "select"])
+@pytest.mark.parametrize("renorm", [True, False])
+def test_route_bitexact_given_logits(E, k, mode, renorm):
+    r = np.random.default_rng(E * 100 + k)
+    T = 300
+    logits = r.standard_normal((T, E)).astype(np.float32)
+    logits[: T // 3] = np.round(logits[: T // 3] * 2)          # many exact ties
+    logits[5, : E // 2] = np.nan                                # NaN keys
+    bias = (r.standard_normal(E) * 0.5).astype(np.float32) if mode != "none" else None
+    sh = LayerShape("r", d=256, E=E, k=k, f=256, bias_mode=mode, renormalize=renorm,
+                    act="f32", router="f32", expert="f32")
+    cfg = M.make_config(sh, T)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    M.moe_route(cfg, tdev(logits, torch.float32), None if bias is None else tdev(bias, torch.float32),
+                idx, gate)
+    ref = O.route(logits, bias, k, mode, renorm)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref["idx"])
+    ok = np.isfinite(ref["gates"]).all(1)
+    ok[5] = False
+    # softmax over E in FP32 (expf within 2 ulp, a sum of E terms): rtol (E + k + 8) 2^-24
+    np.testing.assert_allclose(gate.cpu().numpy()[ok], ref["gates"][ok],
+                               rtol=(E + k + 8) * 2.0 ** -24, atol=1e-30)
+
+
+# --------------------------------------------------------------------- a4 + a5
+@pytest.mark.parametrize("T,k,E,C", [(1, 1, 8, 0.0), (1, 8, 64, 0.0), (37, 6, 64, 1.0),
+                                     (32, 6, 64, 1.25), (500, 8, 64, 1.5), (4096, 8, 64, 0.0),
+                                     (16384, 8, 128, 0.0), (9440, 8, 256, 1.0), (1000, 3, 512, 0.5)])
+def test_permute_bitexact(T, k, E, C):
+    r = np.random.default_rng(T + E)
+    pop = np.arange(1, E + 1, dtype=np.float64) ** -1.1
+    pop /= pop.sum()
+    idx = np.stack([r.choice(E, k, replace=False, p=pop) for _ in range(T)]).astype(np.int32)
+    sh = LayerShape("p", d=256, E=E, k=k, f=256, capacity_factor=C)
+    cfg = M.make_config(sh, T)
+    n = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    slot = torch.empty(n, dtype=torch.int32, device="cuda")
+    dropped = torch.empty(1, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    M.moe_permute(cfg, tdev(idx, torch.int32), counts, offsets, perm, slot, dropped, ws)
+    ref = O.permute(idx, E, C)
+    np.testing.assert_array_equal(counts.cpu().numpy(), ref["counts"])
+    np.testing.assert_array_equal(offsets.cpu().numpy(), ref["offsets"])
+    np.testing.assert_array_equal(slot.cpu().numpy(), ref["slot_of"])
+    kept = int(ref["offsets"][-1])
+    np.testing.assert_array_equal(perm.cpu().numpy()[:kept], ref["perm_assign"])
+    assert int(dropped.item()) == ref["dropped"]
+    assert M.moe_get_device_status(ws) == 0
+
+
+def test_permute_flags_out_of_range_expert():
+    T, k, E = 10, 2, 8
+    idx = np.tile(np.array([[0, 1]], np.int32), (T, 1))
+    idx[3, 1] = 8
+    idx[7, 0] = -1
+    cfg = M.make_config(LayerShape("p", d=256, E=E, k=k, f=256), T)
+    outs = [torch.empty(E, dtype=torch.int32, device="cuda"),
+            torch.empty(E + 1, dtype=torch.int32, device="cuda")] + \
+           [torch.empty(T * k, dtype=torch.int32, device="cuda") for _ in range(2)] + \
+           [torch.empty(1, dtype=torch.int32, device="cuda")]
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    M.moe_permute(cfg, tdev(idx, torch.int32), *outs, ws)
+    assert M.moe_get_device_status(ws) == 1
+    slot = outs[3].cpu().numpy()
+    assert slot[3 * k + 1] == -1 and slot[7 * k + 0] == -1
+    assert outs[0].cpu().numpy().sum() == T * k - 2
+
+
+# --------------------------------------------------------------------- a6 + a7
+@pytest.mark.parametrize("name", ["bf16_plain", "bf16_shared_cap", "bf16_prefill_tiles", "f32_tiny"])
+def test_grouped_ffn_matches_oracle_per_assignment(name):
+    sh, T = SMALL[name], SMALL_T[name]
+    li, x, dli, dx = inputs_on_device(sh, T)
+    own = O.layer_from_inputs(li, x, tokens=[0])
+    cfg = M.make_config(sh, T)
+    ws = M.alloc_workspace(cfg)
+    act = torch.bfloat16 if sh.act == "bf16" else torch.float32
+    xn = tdev(own["xn"], act)
+    y = torch.zeros(T * sh.k, sh.d, dtype=torch.float32, device="cuda")
+    ys = torch.zeros(max(sh.n_shared, 1), T, sh.d, dtype=torch.float32, device="cuda")
+    M.moe_grouped_ffn(cfg, M.make_weights(dli), xn, tdev(own["offsets"], torch.int32),
+                      tdev(own["perm_assign"], torch.int32),
+                      tdev(own["gates"].reshape(-1), torch.float32), y,
+                      ys if sh.n_shared else None, ws)
+    assert M.moe_get_device_status(ws) == 0
+    y = y.cpu().numpy()
+    ex = O.Weights(sh.expert, sh.group_size, *(t.float().numpy() for t in (li.w_gate, li.w_up, li.w_down)))
+    kept = np.nonzero(own["slot_of"] >= 0)[0]
+    ref = np.zeros((T * sh.k, sh.d))
+    bound = np.zeros((T * sh.k, sh.d))
+    flat_idx = own["idx"].reshape(-1)
+    gates = own["gates"].reshape(-1)
+    # The tensor-core path rounds h = silu(u) v to bf16 before the down GEMM
+    # (relative error <= 2^-9 per element); with FP32 accumulation elsewhere the
+    # error of y_n is bounded by 2^-8 g sum_i |h_i Wd[i, n]| (2^-9 doubled for the
+    # FP32 sums).  The fp32 path keeps h in FP32: bound 2^-16 g sum_i |h_i Wd[i, n]|.
+    rel = 2.0 ** -8 if sh.expert != "f32" else 2.0 ** -16
+
+    def ffn_and_bound(W, e, X):
+        u, v = X @ W.get("gate", e), X @ W.get("up", e)
+        h = O.silu(u) * v
+        return h @ W.get("down", e), np.abs(h) @ np.abs(W.get("down", e))
+
+    for e in range(sh.E):
+        a = kept[flat_idx[kept] == e]
+        if a.size:
+            yv, bv = ffn_and_bound(ex, e, own["xn"][a // sh.k])
+            ref[a] = gates[a, None] * yv
+            bound[a] = rel * gates[a, None] * bv
+    assert np.all(np.abs(y[kept] - ref[kept]) <= bound[kept] + 1e-30)
+    rms = np.sqrt(np.mean(ref[kept] ** 2))
+    print(f"{name}: max|dy|/rms(y) = {np.max(np.abs(y[kept] - ref[kept])) / rms:.3e}")
+    if sh.n_shared:
+        shw = O.Weights(sh.expert, sh.group_size, *(t.float().numpy() for t in (li.sh_gate, li.sh_up, li.sh_down)))
+        ysn = ys.cpu().numpy()
+        for s in range(sh.n_shared):
+            rs, bs = ffn_and_bound(shw, s, own["xn"])
+            assert np.all(np.abs(ysn[s] - rs) <= rel * bs + 1e-30)
+
+
+# --------------------------------------------------------------------- a8
+def test_combine_sums_in_fixed_order():
+    T, d, k, S = 33, 256, 3, 2
+    r = np.random.default_rng(5)
+    y = r.standard_normal((T * k, d)).astype(np.float32)
+    ys = r.standard_normal((S, T, d)).astype(np.float32)
+    slot = np.where(r.random(T * k) < 0.3, -1, np.arange(T * k)).astype(np.int32)
+    x = r.standard_normal((T, d)).astype(np.float32)
+    sh = LayerShape("c", d=d, E=8, k=k, f=256, n_shared=S)
+    cfg = M.make_config(sh, T, out_dtype="f32")
+    out = torch.empty(T, d, dtype=torch.float32, device="cuda")
+    M.moe_combine(cfg, tdev(y, torch.float32), tdev(slot, torch.int32), tdev(ys, torch.float32),
+                  tdev(torch.from_numpy(x).to(torch.bfloat16).float().numpy(), torch.bfloat16), out)
+    xb = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    ref = xb + ys.astype(np.float64).sum(0) + \
+        np.where((slot >= 0)[:, None], y, 0).reshape(T, k, d).astype(np.float64).sum(1)
+    terms = np.abs(xb) + np.abs(ys).sum(0) + np.abs(y).reshape(T, k, d).sum(1)
+    assert np.all(np.abs(out.cpu().numpy() - ref) <= (k + S + 1) * 2.0 ** -24 * terms + 1e-30)
+
+
+# --------------------------------------------------------------------- whole layer
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_matches_oracle(name):
+    sh, T = SMALL[name], SMALL_T[name]
+    res = run_layer(sh, T)
+    assert res.max_margin_mismatch < ROUTE_MARGIN, (res.mismatched, res.max_margin_mismatch)
+    assert res.err_ratio <= TOL[sh.expert], res.err_ratio
+    assert res.err_ratio_delta <= DELTA_GUARD[sh.expert], res.err_ratio_delta
+    print(f"{name}: err/rms(out) {res.err_ratio:.3e}  err/rms(delta) {res.err_ratio_delta:.3e}")
+
+
+def test_layer_routing_bitexact_given_gpu_logits():
+    sh, T = SMALL["bf16_shared_cap"], SMALL_T["bf16_shared_cap"]
+    res = run_layer(sh, T)
+    bias = moe_synth.make_router_bias(sh)
+    ref = O.route(res.logits, None if bias is None else bias.numpy(), sh.k, sh.bias_mode,
+                  sh.renormalize)
+    np.testing.assert_array_equal(res.idx, ref["idx"])
+
+
+def test_layer_is_deterministic_and_replayable():
+    """Two runs are bitwise identical, and the five-call chain fed the layer's own
+    routes reproduces the fused call bitwise (route replay control, picx.dev
+    summary Sub-study 2)."""
+    sh, T = SMALL["bf16_shared_cap"], SMALL_T["bf16_shared_cap"]
+    li, x, dli, dx = inputs_on_device(sh, T)
+    layer = M.MoELayer(dli, T, out_dtype="f32")
+    o1 = layer.forward(dx).clone()
+    o2 = layer.forward(dx).clone()
+    assert torch.equal(o1, o2)
+    cfg, w = layer.cfg, layer.w
+    ws = M.alloc_workspace(cfg)
+    xn = torch.empty(T, sh.d, dtype=torch.bfloat16, device="cuda")
+    logits = torch.empty(T, sh.E, dtype=torch.float32, device="cuda")
+    M.moe_rmsnorm_router(cfg, w, dx, xn, logits, ws)
+    idx = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T * sh.k, dtype=torch.float32, device="cuda")
+    M.moe_route(cfg, logits, dli.router_bias, idx, gate)
+    counts = torch.empty(sh.E, dtype=torch.int32, device="cuda")
+    offs = torch.empty(sh.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    slot = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    drop = torch.empty(1, dtype=torch.int32, device="cuda")
+    M.moe_permute(cfg, idx, counts, offs, perm, slot, drop, ws)
+    y = torch.empty(T * sh.k, sh.d, dtype=torch.float32, device="cuda")
+    ys = torch.empty(sh.n_shared, T, sh.d, dtype=torch.float32, device="cuda")
+    M.moe_grouped_ffn(cfg, w, xn, offs, perm, gate, y, ys, ws)
+    o3 = torch.empty(T, sh.d, dtype=torch.float32, device="cuda")
+    M.moe_combine(cfg, y, slot, ys, dx, o3)
+    assert M.moe_get_device_status(ws) == 0
+    assert torch.equal(o1, o3)
+
+
+def test_bf16_output_is_rounding_of_fp32_output():
+    sh, T = SMALL["bf16_plain"], SMALL_T["bf16_plain"]
+    li, x, dli, dx = inputs_on_device(sh, T)
+    o32 = M.MoELayer(dli, T, out_dtype="f32").forward(dx)
+    o16 = M.MoELayer(dli, T, out_dtype="bf16").forward(dx)
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+
+
+# --------------------------------------------------------------------- full sizes
+FULL = [("olmoe", 1), ("olmoe", 16), ("olmoe", 64), ("olmoe", 4096),
+        ("v2lite", 32), ("v2lite", 8192)]
+
+
+@pytest.mark.parametrize("preset,T", FULL)
+def test_full_size_layer_sampled(preset, T):
+    sh = moe_synth.PRESETS[preset]
+    res = run_layer(sh, T, tokens=sample_rows(T))
+    assert res.max_margin_mismatch < ROUTE_MARGIN, (res.mismatched, res.max_margin_mismatch)
+    assert res.err_ratio <= TOL[sh.expert], res.err_ratio
+    assert res.err_ratio_delta <= DELTA_GUARD[sh.expert], res.err_ratio_delta
+    print(f"{preset} T={T}: mismatched routes {res.mismatched} (max margin "
+          f"{res.max_margin_mismatch:.2e}), err/rms(out) {res.err_ratio:.3e}, "
+          f"err/rms(delta) {res.err_ratio_delta:.3e}")
+
+
+@pytest.mark.parametrize("C", [1.0, 1.5])
+def test_v2lite_capacity_factors(C):
+    sh = moe_synth.PRESETS["v2lite"].with_(capacity_factor=C)
+    res = run_layer(sh, 32)
+    assert res.max_margin_mismatch < ROUTE_MARGIN
+    assert res.err_ratio <= TOL[sh.expert], res.err_ratio
+
+
+@pytest.mark.skipif(os.environ.get("MOE_FULL") != "1", reason="22.5 GB of weights; MOE_FULL=1")
+@pytest.mark.parametrize("T", [32, 256, 9440])
+def test_v3_full_size_sampled(T):
+    sh = moe_synth.PRESETS["v3"]
+    res = run_layer(sh, T, tokens=sample_rows(T, 16))
+    assert res.max_margin_mismatch < ROUTE_MARGIN
+    assert res.err_ratio <= TOL[sh.expert], res.err_ratio
