@@ -192,7 +192,9 @@ def run_ours(args):
     layer = M.MoELayer(li, T)            # output in the activation dtype (bf16)
     cfg = layer.cfg
     L = M.moe_layer_launch_count(cfg)
+    n_steps = M.moe_layer_step_count(cfg)
     names = KERNEL_NAMES_TC if sh.expert != "f32" else KERNEL_NAMES_SIMT
+    assert len(names) == n_steps
 
     # routing statistics of this batch (touched experts, kept rows) for the roofline
     counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
@@ -213,7 +215,8 @@ def run_ours(args):
     # profiled steps: per-kernel events on up to 256 evenly spread steps
     n_prof = min(K, 256)
     prof_steps = set(np.linspace(0, K - 1, n_prof).round().astype(int).tolist())
-    evs = {s: [torch.cuda.Event(enable_timing=True) for _ in range(L + 1)] for s in prof_steps}
+    evs = {s: [torch.cuda.Event(enable_timing=True) for _ in range(n_steps + 1)]
+           for s in prof_steps}
     clocks = Clocks(local)
     clocks.start()
     time.sleep(0.3)

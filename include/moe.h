@@ -207,11 +207,13 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
                              void* out, void* ws, size_t ws_bytes, float* logits_out,
                              int32_t* topk_idx_out, int32_t* counts_out, void* stream);
 
-/* moe_layer_forward with per-kernel timing marks, for profiling: events[0] is
- * recorded on `stream` before the first kernel and events[i] right after the
- * i-th kernel (i = 1 .. moe_layer_launch_count(cfg)).  `events` holds
- * caller-created cudaEvent_t handles (as void*); n_events must be at least
- * moe_layer_launch_count(cfg) + 1.  No optional outputs. */
+/* moe_layer_forward with per-step timing marks, for profiling: events[0] is
+ * recorded on `stream` before the first kernel and events[i] right after step i
+ * (i = 1 .. moe_layer_step_count(cfg); the steps are RMSNorm, router, route,
+ * permute, [gather], gate/up GEMM, down GEMM, combine -- the gather only for
+ * tensor-core experts).  `events` holds caller-created cudaEvent_t handles (as
+ * void*); n_events must be at least moe_layer_step_count(cfg) + 1.  No
+ * optional outputs. */
 moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* w,
                                       const void* x, void* out, void* ws, size_t ws_bytes,
                                       void* const* events, int32_t n_events, void* stream);
@@ -227,6 +229,9 @@ const char* moe_status_string(moe_status s);
 /* Number of kernels moe_layer_forward launches for this configuration (for
  * launch accounting); 0 on an invalid configuration. */
 int32_t moe_layer_launch_count(const moe_config* cfg);
+
+/* Number of steps moe_layer_forward_profiled marks (see there); 0 if invalid. */
+int32_t moe_layer_step_count(const moe_config* cfg);
 
 #ifdef __cplusplus
 }

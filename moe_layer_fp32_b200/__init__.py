@@ -64,6 +64,7 @@ _SIGS = {
     "moe_get_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int32), _VP]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_layer_launch_count": (ctypes.c_int32, [_CFG]),
+    "moe_layer_step_count": (ctypes.c_int32, [_CFG]),
 }
 
 
@@ -183,7 +184,7 @@ def moe_layer_forward(cfg, w: MoeWeights, x, out, ws, logits_out=None, topk_idx_
 
 def moe_layer_forward_profiled(cfg, w: MoeWeights, x, out, ws, events, stream=None):
     """``events``: torch.cuda.Event objects (enable_timing) -- one before the first
-    kernel and one after each kernel of the layer."""
+    kernel and one after each step of the layer (moe_layer_step_count + 1)."""
     for e in events:                     # torch creates the CUDA event on first use
         if not e.cuda_event:
             e.record()
@@ -203,6 +204,10 @@ def moe_get_device_status(ws, stream=None) -> int:
 
 def moe_layer_launch_count(cfg) -> int:
     return int(lib().moe_layer_launch_count(ctypes.byref(cfg)))
+
+
+def moe_layer_step_count(cfg) -> int:
+    return int(lib().moe_layer_step_count(ctypes.byref(cfg)))
 
 
 class MoELayer:

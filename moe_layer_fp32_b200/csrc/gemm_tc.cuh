@@ -94,7 +94,10 @@ struct TcConfig {
   // barriers + bookkeeping after the tiles
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
-  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES;
+  // per-tile output row and scale of each token column, one copy per epilogue warp
+  static constexpr uint32_t EPI_BYTES = 4 * 128 * 8;
+  static constexpr uint32_t SMEM_BYTES =
+      1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES + EPI_BYTES;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
   static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
 };
@@ -166,6 +169,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
   int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
   int* prefix = reinterpret_cast<int*>(
       reinterpret_cast<uint8_t*>(smem) + STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+  int* epi_row = prefix + 2 * (kMaxGroups + 1);                  // [4 warps][128]
+  float* epi_scale = reinterpret_cast<float*>(epi_row + 4 * 128);  // [4 warps][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -285,12 +290,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    int* s_row = epi_row + q * 128;
+    float* s_scale = epi_scale + q * 128;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       TileInfo ti;
       decode_tile(p, prefix, BN, tile, ti);
       const TcProblem& P = p.prob[ti.prob];
+      // Output row and scale of every token column of this tile, staged in this
+      // warp's shared-memory slice while the MMAs run (routed DOWN rows go
+      // through the permutation and carry the gate).  Warp-private, so only
+      // __syncwarp orders it.
+      __syncwarp();
+      for (int m = lane; m < BN; m += 32) {
+        int r = -1;
+        float sc = 1.f;
+        if (m < ti.rows) {
+          if (EPI == EPI_DOWN && P.perm_assign) {
+            r = P.perm_assign[ti.slot0 + m];
+            sc = P.gate[r];
+          } else {
+            r = (int)(ti.out_seg + m);
+          }
+        }
+        s_row[m] = r;
+        s_scale[m] = sc;
+      }
+      __syncwarp();
       if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag)) break;
       tc_fence_after();
       const uint32_t t_base = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
@@ -308,30 +335,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
           __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.out);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int m = c * 16 + j;
-            if (m < ti.rows && n_ok)
-              H[(ti.out_seg + m) * (size_t)P.ld_out + n] = __float2bfloat16_rn(silu_f(v0[j]) * v1[j]);
+            const int r = s_row[c * 16 + j];
+            if (r >= 0 && n_ok)
+              H[(size_t)r * P.ld_out + n] = __float2bfloat16_rn(silu_f(v0[j]) * v1[j]);
           }
-        } else if (EPI == EPI_DOWN) {
+        } else {
           float* Y = reinterpret_cast<float*>(P.out);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int m = c * 16 + j;
-            if (m < ti.rows && n_ok) {
-              if (P.perm_assign) {
-                const int as = P.perm_assign[ti.slot0 + m];
-                Y[(size_t)as * P.ld_out + n] = v0[j] * P.gate[as];
-              } else {
-                Y[(ti.out_seg + m) * (size_t)P.ld_out + n] = v0[j];
-              }
-            }
-          }
-        } else {
-          float* L = reinterpret_cast<float*>(P.out);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = c * 16 + j;
-            if (m < ti.rows && n_ok) L[(ti.out_seg + m) * (size_t)P.ld_out + n] = v0[j];
+            const int r = s_row[c * 16 + j];
+            if (r >= 0 && n_ok) Y[(size_t)r * P.ld_out + n] = v0[j] * s_scale[c * 16 + j];
           }
         }
       }

@@ -7,6 +7,8 @@
 
 namespace moe {
 
+constexpr int kMaxExpertsScan = 512;
+
 // ---------------------------------------------------------------------------
 // block reductions
 // ---------------------------------------------------------------------------
@@ -82,6 +84,62 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const TA* __restrict__ x,
   for (int i = threadIdx.x; i < d; i += 256) {
     double v = (double)to_f32(x[row + i]);
     store_act(&xn[row + i], (v * r) * (double)gamma[i]);
+  }
+}
+
+// Vectorised RMSNorm: each thread keeps up to MAXV 16-byte vectors of the row in
+// registers between the sum of squares and the scaling pass (d up to
+// 256 * MAXV * 16 / sizeof(TA)).  Same arithmetic as k_rmsnorm.
+MOE_DEV void unpack8(const uint4& u, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { f[2 * i] = __low2float(h[i]); f[2 * i + 1] = __high2float(h[i]); }
+}
+
+template <int MAXV>
+__global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __restrict__ x,
+                                                       const float* __restrict__ gamma,
+                                                       __nv_bfloat16* __restrict__ xn, int d,
+                                                       double eps) {
+  __shared__ double red[8];
+  const int nv = d / 8;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)blockIdx.x * d);
+  uint4* outr = reinterpret_cast<uint4*>(xn + (size_t)blockIdx.x * d);
+  uint4 buf[MAXV];
+  double s = 0.0;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = threadIdx.x + i * 256;
+    if (v < nv) {
+      buf[i] = xr[v];
+      float f[8];
+      unpack8(buf[i], f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += (double)f[j] * (double)f[j];
+    }
+  }
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  double tot = 0.0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const double r = 1.0 / sqrt(tot / d + eps);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = threadIdx.x + i * 256;
+    if (v < nv) {
+      float f[8];
+      unpack8(buf[i], f);
+      const float4 g0 = reinterpret_cast<const float4*>(gamma)[2 * v];
+      const float4 g1 = reinterpret_cast<const float4*>(gamma)[2 * v + 1];
+      const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      uint4 o;
+      __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(&o);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ob[j] = bf16_from_double(((double)f[j] * r) * (double)g[j]);
+      outr[v] = o;
+    }
   }
 }
 
@@ -303,6 +361,189 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
         const int s = s_off[e] + rank;
         slot_of[a] = s;
         perm_assign[s] = a;
+      } else {
+        slot_of[a] = -1;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a4 + a5 for large batches: the same counting sort over many CTAs, in three
+// launches and still without global atomics.
+//   count: CTA b counts its chunk of kPermChunk assignments per expert and
+//          writes blk[e * nb + b];
+//   scan:  one CTA turns blk into exclusive per-expert bases over the CTAs,
+//          and kept / offsets / dropped as in the one-CTA kernel;
+//   rank:  CTA b recounts its chunk per warp and assigns
+//          rank = CTA base + earlier warps + running count + earlier lanes.
+// Each lane holds kPermPerLane assignments in registers (loads issued together).
+// ---------------------------------------------------------------------------
+constexpr int kPermPerLane = 8;
+constexpr int kPermWarps = 8;
+constexpr int kPermChunk = kPermWarps * 32 * kPermPerLane;   // 2048 assignments per CTA
+
+MOE_DEV void perm_load_chunk(const int32_t* idx, int n, int E, int base, int lane,
+                             int (&e)[kPermPerLane], int32_t* err) {
+#pragma unroll
+  for (int r = 0; r < kPermPerLane; ++r) {
+    const int a = base + r * 32 + lane;
+    e[r] = a < n ? idx[a] : -1;
+  }
+#pragma unroll
+  for (int r = 0; r < kPermPerLane; ++r) {
+    const int a = base + r * 32 + lane;
+    if (a < n && (e[r] < 0 || e[r] >= E)) {
+      if (err) set_error(err, DEV_BAD_EXPERT);
+      e[r] = -1;
+    }
+  }
+}
+
+MOE_DEV void perm_count_warp(const int (&e)[kPermPerLane], int* cnt_w, int lane) {
+#pragma unroll
+  for (int r = 0; r < kPermPerLane; ++r) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, e[r]);
+    if (e[r] >= 0 && lane == __ffs(peers) - 1) cnt_w[e[r]] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(256) k_perm_count(const int32_t* __restrict__ idx, int n, int E,
+                                                    int nb, int32_t* __restrict__ blk,
+                                                    int32_t* err) {
+  extern __shared__ int cnt[];   // [8][E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kPermWarps * E; i += 256) cnt[i] = 0;
+  __syncthreads();
+  int e[kPermPerLane];
+  perm_load_chunk(idx, n, E, blockIdx.x * kPermChunk + warp * 32 * kPermPerLane, lane, e, err);
+  perm_count_warp(e, cnt + warp * E, lane);
+  __syncthreads();
+  for (int x = tid; x < E; x += 256) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kPermWarps; ++w) s += cnt[w * E + x];
+    blk[(size_t)x * nb + blockIdx.x] = s;
+  }
+}
+
+MOE_DEV int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// exclusive scan of kept = min(tot, cap) over experts (thread e < E holds tot),
+// for a CTA of 1024 threads; writes counts, offsets, dropped and s_off
+MOE_DEV void expert_offsets_1024(int tot, int E, int cap, int32_t* counts, int32_t* offsets,
+                                 int32_t* n_dropped, int* s_off, int* wsum, int* s_drop) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kept = (tid < E) ? min(tot, cap) : 0;
+  if (tid < E) {
+    counts[tid] = tot;
+    if (tot > kept) atomicAdd(s_drop, tot - kept);
+  }
+  const int v = warp_incl_scan(kept, lane);
+  if (lane == 31) wsum[warp] = v;
+  __syncthreads();
+  if (warp == 0) wsum[lane] = warp_incl_scan(wsum[lane], lane);
+  __syncthreads();
+  if (tid < E) {
+    const int excl = v - kept + (warp > 0 ? wsum[warp - 1] : 0);
+    offsets[tid] = excl;
+    if (s_off) s_off[tid] = excl;
+    if (tid == E - 1) offsets[E] = excl + kept;
+  }
+  __syncthreads();
+  if (tid == 0) *n_dropped = *s_drop;
+}
+
+__global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ blk, int nb, int E,
+                                                    int cap, int32_t* __restrict__ counts,
+                                                    int32_t* __restrict__ offsets,
+                                                    int32_t* __restrict__ n_dropped) {
+  __shared__ int s_tot[kMaxExpertsScan];
+  __shared__ int wsum[32];
+  __shared__ int s_drop;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_drop = 0;
+  const int nch = (nb + 31) / 32;
+  const int per_w = (E + 31) / 32;
+  const int pairs = per_w * nch;
+  int carry = 0;
+  for (int p0 = 0; p0 < pairs; p0 += 8) {
+    int v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int p = p0 + u;
+      const int e = warp + 32 * (p / nch), b = (p % nch) * 32 + lane;
+      v[u] = (p < pairs && e < E && b < nb) ? blk[(size_t)e * nb + b] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int p = p0 + u;
+      if (p >= pairs) break;
+      const int e = warp + 32 * (p / nch), c = p % nch, b = c * 32 + lane;
+      if (c == 0) carry = 0;
+      const int incl = warp_incl_scan(v[u], lane);
+      if (e < E && b < nb) blk[(size_t)e * nb + b] = carry + incl - v[u];
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+      if (c == nch - 1 && lane == 0 && e < E) s_tot[e] = carry;
+    }
+  }
+  __syncthreads();
+  expert_offsets_1024(tid < E ? s_tot[tid] : 0, E, cap, counts, offsets, n_dropped, nullptr,
+                      wsum, &s_drop);
+}
+
+__global__ void __launch_bounds__(256) k_perm_rank(const int32_t* __restrict__ idx, int n, int E,
+                                                   int nb, int cap,
+                                                   const int32_t* __restrict__ blk,
+                                                   const int32_t* __restrict__ offsets,
+                                                   int32_t* __restrict__ perm_assign,
+                                                   int32_t* __restrict__ slot_of) {
+  extern __shared__ int sm[];
+  int* cnt = sm;                       // [8][E]
+  int* s_off = sm + kPermWarps * E;    // [E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kPermWarps * E; i += 256) cnt[i] = 0;
+  for (int i = tid; i < E; i += 256) s_off[i] = offsets[i];
+  __syncthreads();
+  const int base = blockIdx.x * kPermChunk + warp * 32 * kPermPerLane;
+  int e[kPermPerLane];
+  perm_load_chunk(idx, n, E, base, lane, e, nullptr);
+  perm_count_warp(e, cnt + warp * E, lane);
+  __syncthreads();
+  for (int x = tid; x < E; x += 256) {
+    int run = blk[(size_t)x * nb + blockIdx.x];
+#pragma unroll
+    for (int w = 0; w < kPermWarps; ++w) {
+      const int c = cnt[w * E + x];
+      cnt[w * E + x] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  int* cw = cnt + warp * E;
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int r = 0; r < kPermPerLane; ++r) {
+    const int a = base + r * 32 + lane;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e[r]);
+    int rank = 0;
+    if (e[r] >= 0) rank = cw[e[r]] + __popc(peers & lt);
+    __syncwarp();
+    if (e[r] >= 0 && lane == __ffs(peers) - 1) cw[e[r]] += __popc(peers);
+    __syncwarp();
+    if (a < n) {
+      if (e[r] >= 0 && rank < cap) {
+        const int sl = s_off[e[r]] + rank;
+        slot_of[a] = sl;
+        perm_assign[sl] = a;
       } else {
         slot_of[a] = -1;
       }

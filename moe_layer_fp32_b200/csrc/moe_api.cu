@@ -42,7 +42,7 @@ inline int router_slice(const moe_config* c, int ns) {
 }
 
 struct Layout {
-  size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, xp, h, y, ys, total;
+  size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, h, y, ys, total;
   int ns;
 };
 
@@ -92,6 +92,7 @@ Layout layout(const moe_config* c) {
   L.perm = o;     o = align_up(o + T * k * 4);
   L.slot = o;     o = align_up(o + T * k * 4);
   L.dropped = o;  o = align_up(o + 16);
+  L.blk = o;      o = align_up(o + (size_t)E * ((T * k + kPermChunk - 1) / kPermChunk) * 4);
   L.xp = o;       o = align_up(o + (tc_experts(c) ? T * k * d * act : 0));
   L.h = o;        o = align_up(o + (T * k + S * T) * f * hb);
   L.y = o;        o = align_up(o + T * k * d * 4);
@@ -216,6 +217,19 @@ int capacity_rows(const moe_config* c) {
 // ----------------------------------------------------------------- the steps
 moe_status run_rmsnorm(const moe_config* c, const moe_weights* w, const void* x, void* xn,
                        cudaStream_t st) {
+  if (c->act_dtype == MOE_BF16 && c->d <= 256 * 8 * 4 &&
+      reinterpret_cast<uintptr_t>(x) % 16 == 0 && reinterpret_cast<uintptr_t>(xn) % 16 == 0 &&
+      reinterpret_cast<uintptr_t>(w->rms_gamma) % 16 == 0) {
+    const int nv = c->d / 8;
+    const double eps = (double)c->rms_eps;
+    auto xb = static_cast<const __nv_bfloat16*>(x);
+    auto g = static_cast<const float*>(w->rms_gamma);
+    auto ob = static_cast<__nv_bfloat16*>(xn);
+    if (nv <= 256) k_rmsnorm_bf16v<1><<<c->T, 256, 0, st>>>(xb, g, ob, c->d, eps);
+    else if (nv <= 512) k_rmsnorm_bf16v<2><<<c->T, 256, 0, st>>>(xb, g, ob, c->d, eps);
+    else k_rmsnorm_bf16v<4><<<c->T, 256, 0, st>>>(xb, g, ob, c->d, eps);
+    return check_launch();
+  }
   if (c->act_dtype == MOE_BF16)
     k_rmsnorm<__nv_bfloat16><<<c->T, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(w->rms_gamma),
@@ -282,9 +296,29 @@ moe_status run_route(const moe_config* c, const float* part, int ns, const float
   return check_launch();
 }
 
+// assignments above which the permutation runs on many CTAs
+constexpr int kPermSingleMax = 4096;
+inline int perm_blocks(const moe_config* c) {
+  return (c->T * c->k + kPermChunk - 1) / kPermChunk;
+}
+
 moe_status run_permute(const moe_config* c, const int32_t* idx, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* slot, int32_t* dropped,
-                       int32_t* err, cudaStream_t st) {
+                       int32_t* err, int32_t* blk, cudaStream_t st) {
+  const int n = c->T * c->k;
+  if (n > kPermSingleMax && blk) {
+    const int nb = perm_blocks(c);
+    const size_t sm1 = (size_t)kPermWarps * c->E * 4;
+    const size_t sm3 = sm1 + (size_t)c->E * 4;
+    if (cudaFuncSetAttribute(k_perm_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm3) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    k_perm_count<<<nb, 256, sm1, st>>>(idx, n, c->E, nb, blk, err);
+    k_perm_scan<<<1, 1024, 0, st>>>(blk, nb, c->E, capacity_rows(c), counts, offsets, dropped);
+    k_perm_rank<<<nb, 256, sm3, st>>>(idx, n, c->E, nb, capacity_rows(c), blk, offsets, perm,
+                                      slot);
+    return check_launch();
+  }
   const size_t smem = (size_t)33 * c->E * 4;
   if (cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -472,7 +506,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
     return s;
   mk->mark(st);
   if ((s = run_permute(cfg, idx, counts, offsets, perm, slot, at<int32_t>(ws, L.dropped), err,
-                       st)) != MOE_OK)
+                       at<int32_t>(ws, L.blk), st)) != MOE_OK)
     return s;
   mk->mark(st);
   if ((s = run_ffn(cfg, w, xn, offsets, perm, gate, y, ys, ws, st, mk)) != MOE_OK) return s;
@@ -535,8 +569,10 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int32_t* 
   if (!topk_idx || !counts || !offsets || !perm_assign || !slot_of || !n_dropped)
     return MOE_ERR_INVALID;
   if (!ws || ws_bytes < 16 || reinterpret_cast<uintptr_t>(ws) % kAlign) return MOE_ERR_WORKSPACE;
+  // the multi-CTA path keeps per-CTA counts in the workspace when it is large enough
+  int32_t* blk = ws_bytes >= layout(cfg).total ? at<int32_t>(ws, layout(cfg).blk) : nullptr;
   return run_permute(cfg, topk_idx, counts, offsets, perm_assign, slot_of, n_dropped,
-                     static_cast<int32_t*>(ws), S_(stream));
+                     static_cast<int32_t*>(ws), blk, S_(stream));
 }
 
 moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* xn,
@@ -570,7 +606,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
 moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* w,
                                       const void* x, void* out, void* ws, size_t ws_bytes,
                                       void* const* events, int32_t n_events, void* stream) {
-  if (!events || n_events < moe_layer_launch_count(cfg) + 1) return MOE_ERR_INVALID;
+  if (!events || n_events < moe_layer_step_count(cfg) + 1) return MOE_ERR_INVALID;
   Marks mk;
   mk.ev = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
   mk.n = n_events;
@@ -599,10 +635,16 @@ const char* moe_status_string(moe_status s) {
   return "MOE_ERR_UNKNOWN";
 }
 
-int32_t moe_layer_launch_count(const moe_config* cfg) {
+int32_t moe_layer_step_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
   // rmsnorm, router, route, permute, [gather], gate/up, down, combine
   return tc_experts(cfg) ? 8 : 7;
+}
+
+int32_t moe_layer_launch_count(const moe_config* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  const int perm = cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
+  return moe_layer_step_count(cfg) - 1 + perm;
 }
 
 }  // extern "C"

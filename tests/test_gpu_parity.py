@@ -86,10 +86,14 @@ def test_route_bitexact_given_logits(E, k, mode, renorm):
 
 
 # --------------------------------------------------------------------- a4 + a5
+@pytest.mark.parametrize("full_ws", [False, True])
 @pytest.mark.parametrize("T,k,E,C", [(1, 1, 8, 0.0), (1, 8, 64, 0.0), (37, 6, 64, 1.0),
                                      (32, 6, 64, 1.25), (500, 8, 64, 1.5), (4096, 8, 64, 0.0),
-                                     (16384, 8, 128, 0.0), (9440, 8, 256, 1.0), (1000, 3, 512, 0.5)])
-def test_permute_bitexact(T, k, E, C):
+                                     (16384, 8, 128, 0.0), (9440, 8, 256, 1.0), (1000, 3, 512, 0.5),
+                                     (6000, 6, 512, 1.25), (513, 8, 64, 0.0)])
+def test_permute_bitexact(T, k, E, C, full_ws):
+    """full_ws: with a whole workspace, batches above 4096 assignments take the
+    three-kernel multi-CTA path; with only the error word, the one-CTA kernel."""
     r = np.random.default_rng(T + E)
     pop = np.arange(1, E + 1, dtype=np.float64) ** -1.1
     pop /= pop.sum()
@@ -102,7 +106,7 @@ def test_permute_bitexact(T, k, E, C):
     perm = torch.full((n,), -7, dtype=torch.int32, device="cuda")
     slot = torch.empty(n, dtype=torch.int32, device="cuda")
     dropped = torch.empty(1, dtype=torch.int32, device="cuda")
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = M.alloc_workspace(cfg) if full_ws else torch.zeros(256, dtype=torch.uint8, device="cuda")
     M.moe_permute(cfg, tdev(idx, torch.int32), counts, offsets, perm, slot, dropped, ws)
     ref = O.permute(idx, E, C)
     np.testing.assert_array_equal(counts.cpu().numpy(), ref["counts"])
