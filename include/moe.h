@@ -174,6 +174,28 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int32_t* 
                        int32_t* offsets, int32_t* perm_assign, int32_t* slot_of,
                        int32_t* n_dropped, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_permute without a workspace.  The pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- for example a
+ * plugin slot in another inference engine that hands an operator its input and
+ * output tensors but no allocator, or a serving process that reserves all of its
+ * device memory at start-up so that any later allocation would fail.
+ *
+ * Same outputs as moe_permute, bit for bit.  The per-CTA counts of the
+ * multi-CTA path live in a 1 MiB array built into the library (a static device
+ * array that every GPU using the library holds until the process exits), so
+ * E * ceil(T*k / 2048) must be at most 262144; larger batches return
+ * MOE_ERR_WORKSPACE and launch nothing.  Nothing is allocated or freed.
+ *
+ * The first call on each device looks up that array's device address (under a
+ * lock); make that first call before any stream capture.  Every call on a device
+ * shares the one array, so calls whose kernels overlap on the GPU (other
+ * streams, other host threads) race and give wrong results: serialise them.
+ * Expert ids outside [0, E) are dropped (slot -1) without a report, since there
+ * is no workspace to carry the device error word. */
+moe_status moe_permute_static(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
+                              int32_t* offsets, int32_t* perm_assign, int32_t* slot_of,
+                              int32_t* n_dropped, void* stream);
+
 /* Steps a6 + a7: grouped SwiGLU expert GEMMs over the permuted tokens
  * ("MoE: dynamism the compiler cannot remove", grouped GEMM section), plus the
  * shared experts on every token.

@@ -56,6 +56,7 @@ _SIGS = {
     "moe_rmsnorm_router": (ctypes.c_int, [_CFG, _WTS, _VP, _VP, _F32P, _VP, _SZ, _VP]),
     "moe_route": (ctypes.c_int, [_CFG, _F32P, _F32P, _I32P, _F32P, _VP]),
     "moe_permute": (ctypes.c_int, [_CFG, _I32P, _I32P, _I32P, _I32P, _I32P, _I32P, _VP, _SZ, _VP]),
+    "moe_permute_static": (ctypes.c_int, [_CFG, _I32P, _I32P, _I32P, _I32P, _I32P, _I32P, _VP]),
     "moe_grouped_ffn": (ctypes.c_int, [_CFG, _WTS, _VP, _I32P, _I32P, _F32P, _F32P, _F32P, _VP, _SZ, _VP]),
     "moe_combine": (ctypes.c_int, [_CFG, _F32P, _I32P, _F32P, _VP, _VP, _VP]),
     "moe_layer_forward": (ctypes.c_int, [_CFG, _WTS, _VP, _VP, _VP, _SZ, _F32P, _I32P, _I32P, _VP]),
@@ -160,6 +161,14 @@ def moe_permute(cfg, topk_idx, counts, offsets, perm_assign, slot_of, n_dropped,
     _check("moe_permute", lib().moe_permute(
         ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(offsets), _p(perm_assign), _p(slot_of),
         _p(n_dropped), _p(ws), ws.numel(), _stream(stream)))
+
+
+def moe_permute_static(cfg, topk_idx, counts, offsets, perm_assign, slot_of, n_dropped,
+                       stream=None):
+    """moe_permute for callers that cannot allocate: no workspace argument."""
+    _check("moe_permute_static", lib().moe_permute_static(
+        ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(offsets), _p(perm_assign), _p(slot_of),
+        _p(n_dropped), _stream(stream)))
 
 
 def moe_grouped_ffn(cfg, w: MoeWeights, xn, offsets, perm_assign, topk_gate, y_assign, y_shared,

@@ -7,6 +7,7 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -515,6 +516,30 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
   return s;
 }
 
+// ------------------------------------------------ allocation-free permutation
+// Scratch of moe_permute_static: the per-CTA expert counts of the multi-CTA
+// permutation live in this file-scope device array instead of a caller
+// workspace.  Every GPU that loads the library holds it until the process ends.
+constexpr size_t kStaticPermInts = size_t(1) << 18;           // 1 MiB of int32
+static __device__ __align__(256) int32_t g_perm_counts[kStaticPermInts];
+
+// Device address of g_perm_counts on the current device, looked up once per
+// device (host code may not use the symbol's name as a device pointer).
+int32_t* static_perm_counts() {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static int32_t* ptr[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_perm_counts) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<int32_t*>(p);
+  }
+  return ptr[dev];
+}
+
 // =================================================================== C ABI
 }  // namespace
 
@@ -573,6 +598,42 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int32_t* 
   int32_t* blk = ws_bytes >= layout(cfg).total ? at<int32_t>(ws, layout(cfg).blk) : nullptr;
   return run_permute(cfg, topk_idx, counts, offsets, perm_assign, slot_of, n_dropped,
                      static_cast<int32_t*>(ws), blk, S_(stream));
+}
+
+moe_status moe_permute_static(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
+                              int32_t* offsets, int32_t* perm_assign, int32_t* slot_of,
+                              int32_t* n_dropped, void* stream) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!topk_idx || !counts || !offsets || !perm_assign || !slot_of || !n_dropped)
+    return MOE_ERR_INVALID;
+  const int n = cfg->T * cfg->k;
+  const size_t need = (size_t)cfg->E * ((n + kPermChunk - 1) / kPermChunk);
+  if (need > kStaticPermInts) return MOE_ERR_WORKSPACE;
+  int32_t* blk = static_perm_counts();
+  if (!blk) return MOE_ERR_CUDA;
+  cudaStream_t st = S_(stream);
+  const int E = cfg->E, cap = capacity_rows(cfg);
+  if (n <= kPermSingleMax) {
+    const size_t smem = (size_t)33 * E * 4;
+    if (cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    k_permute<<<1, 1024, smem, st>>>(topk_idx, n, E, cap, counts, offsets, perm_assign, slot_of,
+                                     n_dropped, nullptr);
+    return check_launch();
+  }
+  // every entry of blk that the scan reads is written by the count kernel first
+  const int nb = (n + kPermChunk - 1) / kPermChunk;
+  const size_t sm1 = (size_t)kPermWarps * E * 4;
+  const size_t sm3 = sm1 + (size_t)E * 4;
+  if (cudaFuncSetAttribute(k_perm_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  k_perm_count<<<nb, 256, sm1, st>>>(topk_idx, n, E, nb, blk, nullptr);
+  k_perm_scan<<<1, 1024, 0, st>>>(blk, nb, E, cap, counts, offsets, n_dropped);
+  k_perm_rank<<<nb, 256, sm3, st>>>(topk_idx, n, E, nb, cap, blk, offsets, perm_assign, slot_of);
+  return check_launch();
 }
 
 moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* xn,
