@@ -195,14 +195,13 @@ MOE_DEV uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_byt
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A and B, FP32 accumulation,
-// A MN-major (weights, M = 128 output features), B K-major (tokens, N = n):
+// Instruction descriptor for kind::f16 with bf16 A and B and FP32 accumulation:
 //   c format F32 (1) at bit 4, a format BF16 (1) at bit 7, b format BF16 (1) at
-//   bit 10, a major MN (1) at bit 15, b major K (0) at bit 16, N >> 3 at bit 17,
-//   M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t idesc_bf16_mn_k(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
+//   bit 10, a major at bit 15 and b major at bit 16 (0 = K-major, 1 = MN-major),
+//   N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace moe

@@ -7,21 +7,26 @@
 // permutation, turned into a tile prefix inside every CTA, so the grid never
 // depends on the routing and no host synchronisation is needed.
 //
-// Orientation ("swap AB"): the weights are the MMA's M side and the tokens its
-// N side, C^T[n, m] = sum_k W[k, n] * X[m, k].
-//   A = weight tile, 128 output features x 64 k, loaded from W[G][K][N]
-//       (features contiguous, i.e. MN-major) as two 64-feature TMA boxes with
-//       the 128-byte swizzle.
-//   B = token tile, BN rows x 64 k, loaded from X[R][K] (K-major), 128-byte
+// Shared-memory tiles, per pipeline stage:
+//   weight tile: 128 output features x 64 k, loaded from W[G][K][N] (features
+//       contiguous, MN-major) as two 64-feature TMA boxes, 128-byte swizzle;
+//   token tile: BN rows x 64 k, loaded from X[R][K] (K-major), 128-byte
 //       swizzle.  Rows past the end of an expert's segment belong to the next
-//       segment or fall outside the tensor (zero fill); their columns of the
-//       accumulator are simply not stored.
-// Accumulators live in TMEM (lane = feature, column = token), double buffered
-// so that the epilogue of one tile overlaps the main loop of the next.
+//       segment or fall outside the tensor (zero fill); their accumulator
+//       entries are simply not stored.
+// Two orientations of the same tiles:
+//   swapped (decode tiles, BN = 16..64 tokens): weights on the MMA's M side and
+//       tokens on N, C^T[n, m] = sum_k W[k, n] X[m, k]; TMEM lane = feature, so
+//       a narrow token tile costs no wasted MMA rows;
+//   direct (prefill tiles, 128 tokens): tokens on M and weights on N; TMEM lane
+//       = token, so each epilogue thread owns one output row and writes it with
+//       16-byte stores, and looks up its row and gate once per tile.
+// Accumulators live in TMEM, double buffered so that the epilogue of one tile
+// overlaps the main loop of the next.
 //
-// Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 allocates TMEM and
-// its lane 0 issues tcgen05.mma; warps 2..5 drain TMEM (warp w reads lanes
-// 32*(w%4) .. +31) and run the epilogue.
+// Warp roles (320 threads): warp 0 lane 0 issues TMA; warp 1 allocates TMEM and
+// its lane 0 issues tcgen05.mma; warps 2..9 drain TMEM (warp w reads lanes
+// 32*(w%4) .. +31; warps w and w+4 split the columns) and run the epilogue.
 //
 // Epilogues:
 //   GATEUP  two accumulators (gate, up); h = silu(gate) * up -> bf16 H row.
@@ -37,7 +42,8 @@ namespace moe {
 
 enum Epi : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_ROUTER = 2 };
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;
+constexpr int kEpiWarps = 8;
 constexpr int kMaxGroups = 512;
 
 struct TcProblem {
@@ -72,16 +78,21 @@ struct TileInfo {
   int slot0;          // routed: slot of the tile's first token
 };
 
-template <int EPI>
+// Weight blocks (128 features x 64 k) per pipeline stage: gate and up for
+// GATEUP; for a direct DOWN tile, two neighbouring 128-feature blocks of W_down
+// (a 256-wide tile); otherwise one.
+template <int EPI, bool DIRECT>
 struct TcShape {
-  static constexpr int NA = (EPI == EPI_GATEUP) ? 2 : 1;
+  static constexpr int NA = (EPI == EPI_GATEUP) ? 2 : (EPI == EPI_DOWN && DIRECT) ? 2 : 1;
   static constexpr uint32_t A_BYTES = 128 * 64 * 2;
+  static constexpr int TILE_N = (EPI == EPI_DOWN && DIRECT) ? 256 : 128;   // features per tile
 };
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool DIRECT>
 struct TcConfig {
-  static constexpr int NA = TcShape<EPI>::NA;
-  static constexpr uint32_t A_BYTES = TcShape<EPI>::A_BYTES;
+  static constexpr int NA = TcShape<EPI, DIRECT>::NA;
+  static constexpr int TILE_N = TcShape<EPI, DIRECT>::TILE_N;
+  static constexpr uint32_t A_BYTES = TcShape<EPI, DIRECT>::A_BYTES;
   static constexpr uint32_t B_BYTES = BN * 64 * 2;
   static constexpr uint32_t STAGE_BYTES = NA * A_BYTES + B_BYTES;
   static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
@@ -90,37 +101,45 @@ struct TcConfig {
   static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                         : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr uint32_t IDESC = idesc_bf16_mn_k(128, BN);
+  // swapped: A = weights (MN-major), B = tokens (K-major), M = 128 features, N = BN,
+  //          one MMA per weight block;
+  // direct:  A = tokens (K-major), B = all NA weight blocks at once (MN-major, the
+  //          blocks 16 KB apart = two 64-feature boxes each at the 8 KB leading
+  //          offset), M = 128 tokens, N = 128 * NA
+  static constexpr uint32_t IDESC = DIRECT ? idesc_bf16(128, 128 * NA, false, true)
+                                           : idesc_bf16(128, BN, true, false);
   // barriers + bookkeeping after the tiles
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
-  // per-tile output row and scale of each token column, one copy per epilogue warp
-  static constexpr uint32_t EPI_BYTES = 4 * 128 * 8;
+  // swapped epilogue: per-tile output row and scale of each token, one copy per warp
+  static constexpr uint32_t EPI_BYTES = kEpiWarps * 128 * 8;
   static constexpr uint32_t SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES + EPI_BYTES;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
+  static_assert(!DIRECT || BN == 128, "direct tiles hold 128 tokens");
   static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
 };
 
 // Decode a linear tile id.  Tiles run over problems, then (group, m-tile) in the
 // tile prefix order, then the feature tiles innermost so that neighbouring CTAs
 // share a token tile.
-MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int tile, TileInfo& ti) {
+MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int TN, int tile,
+                         TileInfo& ti) {
   int pi = 0;
   for (; pi < p.n_prob; ++pi) {
     const TcProblem& P = p.prob[pi];
     const int* pre = prefix + pi * (kMaxGroups + 1);
-    const int nt = (P.N + 127) / 128;
+    const int nt = (P.N + TN - 1) / TN;
     const int cnt = pre[P.G] * nt;
     if (tile < cnt) break;
     tile -= cnt;
   }
   const TcProblem& P = p.prob[pi];
   const int* pre = prefix + pi * (kMaxGroups + 1);
-  const int nt = (P.N + 127) / 128;
+  const int nt = (P.N + TN - 1) / TN;
   const int mt = tile / nt;
   ti.prob = pi;
-  ti.n0 = (tile % nt) * 128;
+  ti.n0 = (tile % nt) * TN;
   const int g = find_group(pre, P.G, mt);
   ti.g = g;
   ti.m0 = (mt - pre[g]) * BN;
@@ -139,20 +158,20 @@ MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int tile,
   ti.out_seg = P.out_row_base + (size_t)seg_start + ti.m0;
 }
 
-MOE_DEV int total_tiles(const TcParams& p, const int* prefix) {
+MOE_DEV int total_tiles(const TcParams& p, const int* prefix, int TN) {
   int tot = 0;
   for (int pi = 0; pi < p.n_prob; ++pi) {
     const TcProblem& P = p.prob[pi];
-    tot += prefix[pi * (kMaxGroups + 1) + P.G] * ((P.N + 127) / 128);
+    tot += prefix[pi * (kMaxGroups + 1) + P.G] * ((P.N + TN - 1) / TN);
   }
   return tot;
 }
 
-MOE_DEV float silu_f(float u) { return u / (1.f + expf(-u)); }
+MOE_DEV float silu_f(float u) { return __fdividef(u, 1.f + __expf(-u)); }
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool DIRECT>
 __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant__ TcParams p) {
-  using C = TcConfig<EPI, BN>;
+  using C = TcConfig<EPI, BN, DIRECT>;
   constexpr int NA = C::NA;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -169,8 +188,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
   int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
   int* prefix = reinterpret_cast<int*>(
       reinterpret_cast<uint8_t*>(smem) + STAGES * C::STAGE_BYTES + C::BAR_BYTES);
-  int* epi_row = prefix + 2 * (kMaxGroups + 1);                  // [4 warps][128]
-  float* epi_scale = reinterpret_cast<float*>(epi_row + 4 * 128);  // [4 warps][128]
+  int* epi_row = prefix + 2 * (kMaxGroups + 1);                          // [8 warps][128]
+  float* epi_scale = reinterpret_cast<float*>(epi_row + kEpiWarps * 128);  // [8 warps][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -182,7 +201,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 4);
+      mbar_init(&tempty_bar[a], kEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -208,7 +227,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = total_tiles(p, prefix);
+  constexpr int TN = C::TILE_N;
+  const int total = total_tiles(p, prefix, TN);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -218,7 +238,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
-        decode_tile(p, prefix, BN, tile, ti);
+        decode_tile(p, prefix, BN, TN, tile, ti);
         const TcProblem& P = p.prob[ti.prob];
         const int kblocks = P.K / 64;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -229,9 +249,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
           tma_load_3d(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g);
           tma_load_3d(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g);
           if (NA == 2) {
-            tma_load_3d(st + C::A_BYTES, &P.tmA2, &full_bar[stage], ti.n0, kb * 64, ti.g);
-            tma_load_3d(st + C::A_BYTES + 8192, &P.tmA2, &full_bar[stage], ti.n0 + 64, kb * 64,
-                        ti.g);
+            // GATEUP: the up matrix at the same features; wide DOWN: features +128
+            const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
+            const int n2 = (EPI == EPI_GATEUP) ? ti.n0 : ti.n0 + 128;
+            tma_load_3d(st + C::A_BYTES, m2, &full_bar[stage], n2, kb * 64, ti.g);
+            tma_load_3d(st + C::A_BYTES + 8192, m2, &full_bar[stage], n2 + 64, kb * 64, ti.g);
           }
           tma_load_2d(st + NA * C::A_BYTES, &P.tmB, &full_bar[stage], kb * 64, ti.b_row);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -249,7 +271,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
-        decode_tile(p, prefix, BN, tile, ti);
+        decode_tile(p, prefix, BN, TN, tile, ti);
         const int kblocks = p.prob[ti.prob].K / 64;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag)) break;
         tc_fence_after();
@@ -261,15 +283,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
           const uint32_t b_addr = a_addr + NA * C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            // A: MN-major SW128, 16 k-rows of 128 B per MMA step; the two 64-feature
-            //    halves sit 8 KB apart (leading offset), 8-row groups 1 KB apart.
-            // B: K-major SW128, 16 k = 32 B per step, 8-row groups 1 KB apart.
-            const uint64_t bd = sw128_desc(b_addr + kk * 32, 16, 1024);
-            const uint64_t ad = sw128_desc(a_addr + kk * 2048, 8192, 1024);
-            tc_mma_f16(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0);
-            if (NA == 2) {
-              const uint64_t ad2 = sw128_desc(a_addr + C::A_BYTES + kk * 2048, 8192, 1024);
-              tc_mma_f16(d_tmem + BN, ad2, bd, C::IDESC, (kb | kk) != 0);
+            // weights: MN-major SW128, 16 k-rows of 128 B per MMA step; the two
+            //    64-feature halves sit 8 KB apart (leading offset), 8-row groups 1 KB
+            //    apart.  tokens: K-major SW128, 16 k = 32 B per step, 8-row groups 1 KB.
+            const uint64_t xd = sw128_desc(b_addr + kk * 32, 16, 1024);
+            const uint64_t wd = sw128_desc(a_addr + kk * 2048, 8192, 1024);
+            const uint32_t accum = (kb | kk) != 0;
+            if (DIRECT) {
+              tc_mma_f16(d_tmem, xd, wd, C::IDESC, accum);   // N = 128 * NA at once
+            } else {
+              tc_mma_f16(d_tmem, wd, xd, C::IDESC, accum);
+              if (NA == 2) {
+                const uint64_t wd2 = sw128_desc(a_addr + C::A_BYTES + kk * 2048, 8192, 1024);
+                tc_mma_f16(d_tmem + BN, wd2, xd, C::IDESC, accum);
+              }
             }
           }
           tc_commit(&empty_bar[stage]);
@@ -288,22 +315,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    int* s_row = epi_row + q * 128;
-    float* s_scale = epi_scale + q * 128;
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int half = (warp - 2) >> 2;       // which half of the columns it drains
+    int* s_row = epi_row + (warp - 2) * 128;
+    float* s_scale = epi_scale + (warp - 2) * 128;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       TileInfo ti;
-      decode_tile(p, prefix, BN, tile, ti);
+      decode_tile(p, prefix, BN, TN, tile, ti);
       const TcProblem& P = p.prob[ti.prob];
-      // Output row and scale of every token column of this tile, staged in this
-      // warp's shared-memory slice while the MMAs run (routed DOWN rows go
-      // through the permutation and carry the gate).  Warp-private, so only
-      // __syncwarp orders it.
-      __syncwarp();
-      for (int m = lane; m < BN; m += 32) {
+      const uint32_t t_base = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      if (DIRECT) {
+        // this thread's token row; its output row and gate are fetched before the
+        // accumulator wait so that the loads overlap the MMAs
+        const int m = q * 32 + lane;
         int r = -1;
         float sc = 1.f;
         if (m < ti.rows) {
@@ -314,37 +340,87 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
             r = (int)(ti.out_seg + m);
           }
         }
-        s_row[m] = r;
-        s_scale[m] = sc;
-      }
-      __syncwarp();
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t t_base = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
-      const int n = ti.n0 + row;
-      const bool n_ok = n < P.n_valid;
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag)) break;
+        tc_fence_after();
+        // GATEUP: 128 features, gate in columns [0,128), up in [128,256); each half
+        // of the warps takes 64 features.  DOWN: TILE_N features, half each.
+        constexpr int CPH = (EPI == EPI_GATEUP) ? 4 : TN / 32;   // chunks per half
 #pragma unroll 1
-      for (int c = 0; c < BN / 16; ++c) {
-        if (c * 16 >= ti.rows) break;
-        float v0[16];
-        tmem_ld16(t_base + c * 16, v0);
-        float v1[16];
-        if (NA == 2) tmem_ld16(t_base + BN + c * 16, v1);
-        tmem_wait_ld();
-        if (EPI == EPI_GATEUP) {
-          __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.out);
+        for (int c = half * CPH; c < half * CPH + CPH; ++c) {
+          const int n = ti.n0 + c * 16;
+          if (n >= P.n_valid) break;
+          float v0[16];
+          tmem_ld16(t_base + c * 16, v0);
+          float v1[16];
+          if (EPI == EPI_GATEUP) tmem_ld16(t_base + 128 + c * 16, v1);
+          tmem_wait_ld();
+          if (r >= 0 && EPI == EPI_GATEUP) {
+            uint32_t pk[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int r = s_row[c * 16 + j];
-            if (r >= 0 && n_ok)
-              H[(size_t)r * P.ld_out + n] = __float2bfloat16_rn(silu_f(v0[j]) * v1[j]);
+            for (int j = 0; j < 8; ++j) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(silu_f(v0[2 * j]) * v1[2 * j],
+                                                        silu_f(v0[2 * j + 1]) * v1[2 * j + 1]);
+              pk[j] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) +
+                                                  (size_t)r * P.ld_out + n);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          } else if (r >= 0) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) +
+                                                    (size_t)r * P.ld_out + n);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
+                                   v0[4 * j + 3] * sc);
           }
-        } else {
-          float* Y = reinterpret_cast<float*>(P.out);
+        }
+      } else {
+        // swapped: this thread owns feature n; the tile's token rows and scales are
+        // staged in this warp's shared-memory slice (warp-private: __syncwarp only)
+        __syncwarp();
+        for (int m = lane; m < BN; m += 32) {
+          int r = -1;
+          float sc = 1.f;
+          if (m < ti.rows) {
+            if (EPI == EPI_DOWN && P.perm_assign) {
+              r = P.perm_assign[ti.slot0 + m];
+              sc = P.gate[r];
+            } else {
+              r = (int)(ti.out_seg + m);
+            }
+          }
+          s_row[m] = r;
+          s_scale[m] = sc;
+        }
+        __syncwarp();
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag)) break;
+        tc_fence_after();
+        const int n = ti.n0 + q * 32 + lane;
+        const bool n_ok = n < P.n_valid;
+#pragma unroll 1
+        for (int c = half; c < BN / 16; c += 2) {
+          if (c * 16 >= ti.rows) break;
+          float v0[16];
+          tmem_ld16(t_base + c * 16, v0);
+          float v1[16];
+          if (NA == 2) tmem_ld16(t_base + BN + c * 16, v1);
+          tmem_wait_ld();
+          if (EPI == EPI_GATEUP) {
+            __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.out);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int r = s_row[c * 16 + j];
-            if (r >= 0 && n_ok) Y[(size_t)r * P.ld_out + n] = v0[j] * s_scale[c * 16 + j];
+            for (int j = 0; j < 16; ++j) {
+              const int r = s_row[c * 16 + j];
+              if (r >= 0 && n_ok)
+                H[(size_t)r * P.ld_out + n] = __float2bfloat16_rn(silu_f(v0[j]) * v1[j]);
+            }
+          } else {
+            float* Y = reinterpret_cast<float*>(P.out);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int r = s_row[c * 16 + j];
+              if (r >= 0 && n_ok) Y[(size_t)r * P.ld_out + n] = v0[j] * s_scale[c * 16 + j];
+            }
           }
         }
       }

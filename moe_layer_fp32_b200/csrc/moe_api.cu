@@ -179,10 +179,10 @@ bool map_rows(CUtensorMap* m, const void* base, int R, int K, int BN) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool DIRECT = false>
 moe_status launch_tc(const TcParams& p, cudaStream_t st) {
-  using C = TcConfig<EPI, BN>;
-  auto kern = k_tc_gemm<EPI, BN>;
+  using C = TcConfig<EPI, BN, DIRECT>;
+  auto kern = k_tc_gemm<EPI, BN, DIRECT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
@@ -196,7 +196,7 @@ moe_status launch_tc_bn(int bn, const TcParams& p, cudaStream_t st) {
     case 16: return launch_tc<EPI, 16>(p, st);
     case 32: return launch_tc<EPI, 32>(p, st);
     case 64: return launch_tc<EPI, 64>(p, st);
-    default: return launch_tc<EPI, 128>(p, st);
+    default: return launch_tc<EPI, 128, true>(p, st);   // prefill tiles: tokens on MMA-M
   }
 }
 
