@@ -47,6 +47,16 @@ MOE_DEV __nv_bfloat16 bf16_from_double(double v) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: every kernel of the layer waits for the grid
+// before it in the stream to complete (and its writes to be visible) before it
+// touches global memory, and lets the next grid launch right away, so that the
+// launch of kernel i+1 overlaps the run of kernel i.  Without the launch
+// attribute both are no-ops.
+// ---------------------------------------------------------------------------
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // shared-memory addresses, fences
 // ---------------------------------------------------------------------------
 MOE_DEV uint32_t smem_u32(const void* p) {

@@ -219,6 +219,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
       tma_prefetch_desc(&p.prob[pi].tmB);
     }
   }
+  // everything above touched only this CTA's shared memory, TMEM and the kernel
+  // parameters; from here on the previous kernel's outputs are read
+  pdl_wait();
+  pdl_trigger();
   if (warp >= 2 && warp - 2 < p.n_prob) {
     const TcProblem& P = p.prob[warp - 2];
     group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1));

@@ -67,6 +67,8 @@ template <typename TA>
 __global__ void __launch_bounds__(256) k_rmsnorm(const TA* __restrict__ x,
                                                  const float* __restrict__ gamma,
                                                  TA* __restrict__ xn, int d, double eps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double red[8];
   const size_t row = (size_t)blockIdx.x * d;
   double s = 0.0;
@@ -101,6 +103,8 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __re
                                                        const float* __restrict__ gamma,
                                                        __nv_bfloat16* __restrict__ xn, int d,
                                                        double eps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double red[8];
   const int nv = d / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)blockIdx.x * d);
@@ -153,6 +157,8 @@ __global__ void __launch_bounds__(256) k_router_split(const TA* __restrict__ xn,
                                                       const TA* __restrict__ wr,
                                                       float* __restrict__ part, int T, int d,
                                                       int E, int slice) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float xs[];   // [TT][slice]
   const int t0 = blockIdx.x * TT;
   const int k0 = blockIdx.y * slice;
@@ -179,6 +185,77 @@ __global__ void __launch_bounds__(256) k_router_split(const TA* __restrict__ xn,
   }
 }
 
+// a2 for small batches with a bf16 router: CTA (blockIdx.x, blockIdx.y) takes TT
+// tokens and `rows` consecutive rows of W_r -- one contiguous block of rows * E
+// bf16 -- streamed as 16-byte vectors, every load of a thread issued before its
+// arithmetic.  Thread t always meets the same 8-column group (256 is a multiple
+// of E/8), keeps TT x 8 partial sums in registers, and the threads of a column
+// group are summed in a fixed order through shared memory.
+template <int TT>
+__global__ void __launch_bounds__(256) k_router_vec(const __nv_bfloat16* __restrict__ xn,
+                                                    const __nv_bfloat16* __restrict__ wr,
+                                                    float* __restrict__ part, int T, int d,
+                                                    int E, int rows) {
+  extern __shared__ float sm_r[];
+  float* xs = sm_r;                      // [TT][rows]
+  float* red = sm_r + TT * rows;         // [256][8]
+  pdl_wait();
+  pdl_trigger();
+  const int t0 = blockIdx.x * TT;
+  const int k0 = blockIdx.y * rows;
+  const int kn = min(rows, d - k0);
+  for (int i = threadIdx.x; i < TT * rows; i += 256) {
+    const int tt = i / rows, kk = i % rows;
+    xs[i] = (t0 + tt < T && kk < kn) ? __bfloat162float(xn[(size_t)(t0 + tt) * d + k0 + kk]) : 0.f;
+  }
+  __syncthreads();
+  const int cgs = E / 8;
+  const int nvec = kn * cgs;
+  const uint4* wv = reinterpret_cast<const uint4*>(wr + (size_t)k0 * E);
+  float acc[TT][8];
+#pragma unroll
+  for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[tt][j] = 0.f;
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += 4 * 256) {
+    uint4 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * 256;
+      w[u] = v < nvec ? wv[v] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * 256;
+      if (v < nvec) {
+        float f[8];
+        unpack8(w[u], f);
+        const int i = v / cgs;
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+          const float x = xs[tt * rows + i];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[tt][j] = fmaf(x, f[j], acc[tt][j]);
+        }
+      }
+    }
+  }
+  const int per = 256 / cgs;   // threads per column group
+  for (int tt = 0; tt < TT; ++tt) {
+    if (t0 + tt >= T) break;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) red[threadIdx.x * 8 + j] = acc[tt][j];
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += 256) {
+      const int g = e / 8, j = e % 8;
+      float s = 0.f;
+      for (int m = 0; m < per; ++m) s += red[(g + m * cgs) * 8 + j];
+      part[((size_t)blockIdx.y * T + t0 + tt) * E + e] = s;
+    }
+    __syncthreads();
+  }
+}
+
 // ---------------------------------------------------------------------------
 // a3: softmax + top-k + bias + renormalisation, one warp per token.  Lane l
 // holds experts l, l+32, ...  Keys are FP32 (logit, plus bias in LOGIT/SELECT
@@ -195,6 +272,8 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ part, i
                                                int mode, int renorm, int32_t* __restrict__ idx,
                                                float* __restrict__ gate,
                                                float* __restrict__ logits_out) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -280,6 +359,8 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
                                                   int32_t* __restrict__ slot_of,
                                                   int32_t* __restrict__ n_dropped,
                                                   int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int sm[];
   int* cnt = sm;               // [32][E]
   int* s_off = sm + 32 * E;    // [E]
@@ -412,6 +493,8 @@ MOE_DEV void perm_count_warp(const int (&e)[kPermPerLane], int* cnt_w, int lane)
 __global__ void __launch_bounds__(256) k_perm_count(const int32_t* __restrict__ idx, int n, int E,
                                                     int nb, int32_t* __restrict__ blk,
                                                     int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int cnt[];   // [8][E]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < kPermWarps * E; i += 256) cnt[i] = 0;
@@ -466,6 +549,8 @@ __global__ void __launch_bounds__(1024) k_perm_scan(int32_t* __restrict__ blk, i
                                                     int cap, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ n_dropped) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_tot[kMaxExpertsScan];
   __shared__ int wsum[32];
   __shared__ int s_drop;
@@ -506,6 +591,8 @@ __global__ void __launch_bounds__(256) k_perm_rank(const int32_t* __restrict__ i
                                                    const int32_t* __restrict__ offsets,
                                                    int32_t* __restrict__ perm_assign,
                                                    int32_t* __restrict__ slot_of) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int sm[];
   int* cnt = sm;                       // [8][E]
   int* s_off = sm + kPermWarps * E;    // [E]
@@ -560,6 +647,8 @@ __global__ void __launch_bounds__(256) k_gather_rows(const TA* __restrict__ xn,
                                                      const int32_t* __restrict__ perm_assign,
                                                      const int32_t* __restrict__ n_rows_ptr,
                                                      int k, int d, TA* __restrict__ xp) {
+  pdl_wait();
+  pdl_trigger();
   const int n_rows = *n_rows_ptr;
   const int vec_per_row = d * (int)sizeof(TA) / 16;
   const int warps = gridDim.x * 8;
@@ -603,6 +692,8 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y,
                                                  const float* __restrict__ ys, int S,
                                                  const TA* __restrict__ res, TO* __restrict__ out,
                                                  int T, int d, int k) {
+  pdl_wait();
+  pdl_trigger();
   const int q = d / 4;
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (size_t)T * q) return;
@@ -652,6 +743,8 @@ constexpr int kSimtKC = 256;
 
 template <bool DOWN>
 __global__ void __launch_bounds__(128) k_simt_ffn(SimtArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int prefix[520];
   __shared__ float xs[kSimtRB][kSimtKC];
   __shared__ int rows_src[kSimtRB];

@@ -29,8 +29,13 @@ inline bool tc_router(const moe_config* c) {
 }
 constexpr int kRouterSlice = 128;
 constexpr int kRouterTT = 8;
+// the vectorised small-batch router needs a bf16 router and E/8 dividing 256
+inline bool vec_router(const moe_config* c) {
+  return !tc_router(c) && c->router_dtype == MOE_BF16 && c->E % 8 == 0 && 256 % (c->E / 8) == 0;
+}
 inline int router_splits(const moe_config* c) {
   if (tc_router(c)) return 1;
+  if (vec_router(c)) return (c->d + kRouterSlice - 1) / kRouterSlice;
   int ns = (c->d + kRouterSlice - 1) / kRouterSlice;
   int ttiles = (c->T + kRouterTT - 1) / kRouterTT;
   // enough CTAs to cover the SMs a couple of times, no more slices than needed
@@ -116,6 +121,29 @@ struct Marks {
   }
 };
 
+// Every kernel is launched with programmatic stream serialisation, so that its
+// launch overlaps the previous kernel of the stream (the kernels wait for their
+// predecessor with griddepcontrol.wait before touching memory).
+template <typename Kern, typename... Args>
+cudaError_t launch_k(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args... args) {
+  cudaLaunchConfig_t c = {};
+  c.gridDim = grid;
+  c.blockDim = block;
+  c.dynamicSmemBytes = smem;
+  c.stream = st;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[0].val.programmaticStreamSerializationAllowed = 1;
+  c.attrs = a;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, kern, args...);
+}
+#define MOE_LAUNCH(...)                                             \
+  do {                                                              \
+    if (launch_k(__VA_ARGS__) != cudaSuccess) return MOE_ERR_CUDA;  \
+  } while (0)
+
 moe_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -186,7 +214,7 @@ moe_status launch_tc(const TcParams& p, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  kern<<<num_sms(), kTcThreads, C::SMEM_BYTES, st>>>(p);
+  MOE_LAUNCH((kern), num_sms(), kTcThreads, C::SMEM_BYTES, st, p);
   return check_launch();
 }
 
@@ -226,17 +254,17 @@ moe_status run_rmsnorm(const moe_config* c, const moe_weights* w, const void* x,
     auto xb = static_cast<const __nv_bfloat16*>(x);
     auto g = static_cast<const float*>(w->rms_gamma);
     auto ob = static_cast<__nv_bfloat16*>(xn);
-    if (nv <= 256) k_rmsnorm_bf16v<1><<<c->T, 256, 0, st>>>(xb, g, ob, c->d, eps);
-    else if (nv <= 512) k_rmsnorm_bf16v<2><<<c->T, 256, 0, st>>>(xb, g, ob, c->d, eps);
-    else k_rmsnorm_bf16v<4><<<c->T, 256, 0, st>>>(xb, g, ob, c->d, eps);
+    if (nv <= 256) MOE_LAUNCH((k_rmsnorm_bf16v<1>), c->T, 256, 0, st, xb, g, ob, c->d, eps);
+    else if (nv <= 512) MOE_LAUNCH((k_rmsnorm_bf16v<2>), c->T, 256, 0, st, xb, g, ob, c->d, eps);
+    else MOE_LAUNCH((k_rmsnorm_bf16v<4>), c->T, 256, 0, st, xb, g, ob, c->d, eps);
     return check_launch();
   }
   if (c->act_dtype == MOE_BF16)
-    k_rmsnorm<__nv_bfloat16><<<c->T, 256, 0, st>>>(
+    MOE_LAUNCH((k_rmsnorm<__nv_bfloat16>), c->T, 256, 0, st, 
         static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(w->rms_gamma),
         static_cast<__nv_bfloat16*>(xn), c->d, (double)c->rms_eps);
   else
-    k_rmsnorm<float><<<c->T, 256, 0, st>>>(static_cast<const float*>(x),
+    MOE_LAUNCH((k_rmsnorm<float>), c->T, 256, 0, st, static_cast<const float*>(x),
                                            static_cast<const float*>(w->rms_gamma),
                                            static_cast<float*>(xn), c->d, (double)c->rms_eps);
   return check_launch();
@@ -265,16 +293,25 @@ moe_status run_router(const moe_config* c, const moe_weights* w, const void* xn,
     p.err = err;
     return launch_tc<EPI_ROUTER, 128>(p, st);
   }
+  if (vec_router(c)) {
+    dim3 grid((c->T + kRouterTT - 1) / kRouterTT, ns);
+    const size_t smem = ((size_t)kRouterTT * kRouterSlice + 256 * 8) * 4;
+    MOE_LAUNCH((k_router_vec<kRouterTT>), grid, 256, smem, st,
+               static_cast<const __nv_bfloat16*>(xn),
+               static_cast<const __nv_bfloat16*>(w->w_router), part, c->T, c->d, c->E,
+               kRouterSlice);
+    return check_launch();
+  }
   const int slice = router_slice(c, ns);
   dim3 grid((c->T + kRouterTT - 1) / kRouterTT, ns);
   const size_t smem = (size_t)kRouterTT * slice * 4;
   int threads = c->E >= 256 ? 256 : ((c->E + 31) / 32) * 32;
   if (c->act_dtype == MOE_BF16)
-    k_router_split<__nv_bfloat16, kRouterTT><<<grid, threads, smem, st>>>(
+    MOE_LAUNCH((k_router_split<__nv_bfloat16, kRouterTT>), grid, threads, smem, st, 
         static_cast<const __nv_bfloat16*>(xn), static_cast<const __nv_bfloat16*>(w->w_router),
         part, c->T, c->d, c->E, slice);
   else
-    k_router_split<float, kRouterTT><<<grid, threads, smem, st>>>(
+    MOE_LAUNCH((k_router_split<float, kRouterTT>), grid, threads, smem, st, 
         static_cast<const float*>(xn), static_cast<const float*>(w->w_router), part, c->T,
         c->d, c->E, slice);
   return check_launch();
@@ -286,7 +323,7 @@ moe_status run_route(const moe_config* c, const float* part, int ns, const float
   const int mode = c->bias_mode;
   if (mode != MOE_BIAS_NONE && !bias) return MOE_ERR_INVALID;
 #define MOE_ROUTE(EPL)                                                                     \
-  k_route<EPL><<<blocks, 256, 0, st>>>(part, ns, c->T, c->E, c->k, bias, mode,             \
+  MOE_LAUNCH((k_route<EPL>), blocks, 256, 0, st, part, ns, c->T, c->E, c->k, bias, mode,             \
                                        c->renormalize ? 1 : 0, idx, gate, logits_out)
   if (c->E <= 32) MOE_ROUTE(1);
   else if (c->E <= 64) MOE_ROUTE(2);
@@ -314,9 +351,9 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int32_t* counts,
     if (cudaFuncSetAttribute(k_perm_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm3) != cudaSuccess)
       return MOE_ERR_CUDA;
-    k_perm_count<<<nb, 256, sm1, st>>>(idx, n, c->E, nb, blk, err);
-    k_perm_scan<<<1, 1024, 0, st>>>(blk, nb, c->E, capacity_rows(c), counts, offsets, dropped);
-    k_perm_rank<<<nb, 256, sm3, st>>>(idx, n, c->E, nb, capacity_rows(c), blk, offsets, perm,
+    MOE_LAUNCH((k_perm_count), nb, 256, sm1, st, idx, n, c->E, nb, blk, err);
+    MOE_LAUNCH((k_perm_scan), 1, 1024, 0, st, blk, nb, c->E, capacity_rows(c), counts, offsets, dropped);
+    MOE_LAUNCH((k_perm_rank), nb, 256, sm3, st, idx, n, c->E, nb, capacity_rows(c), blk, offsets, perm,
                                       slot);
     return check_launch();
   }
@@ -324,7 +361,7 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int32_t* counts,
   if (cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  k_permute<<<1, 1024, smem, st>>>(idx, c->T * c->k, c->E, capacity_rows(c), counts, offsets,
+  MOE_LAUNCH((k_permute), 1, 1024, smem, st, idx, c->T * c->k, c->E, capacity_rows(c), counts, offsets,
                                    perm, slot, dropped, err);
   return check_launch();
 }
@@ -356,11 +393,11 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     a.ys = ys;
     a.T = T; a.d = c->d; a.f = c->f; a.k = k; a.E = c->E; a.S = S;
     const int grid = 2 * num_sms();
-    k_simt_ffn<false><<<grid, 128, 0, st>>>(a);
+    MOE_LAUNCH((k_simt_ffn<false>), grid, 128, 0, st, a);
     moe_status s = check_launch();
     if (s != MOE_OK) return s;
     mk->mark(st);
-    k_simt_ffn<true><<<grid, 128, 0, st>>>(a);
+    MOE_LAUNCH((k_simt_ffn<true>), grid, 128, 0, st, a);
     s = check_launch();
     mk->mark(st);
     return s;
@@ -368,7 +405,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   // bf16 experts: gather the routed rows, then gate/up and down on the tensor cores
   __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
   __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
-  k_gather_rows<__nv_bfloat16><<<2 * num_sms(), 256, 0, st>>>(
+  MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 2 * num_sms(), 256, 0, st, 
       static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
   moe_status s = check_launch();
   if (s != MOE_OK) return s;
@@ -462,15 +499,15 @@ moe_status run_combine(const moe_config* c, const float* y, const int32_t* slot,
   const size_t n = (size_t)c->T * (c->d / 4);
   const int blocks = (int)((n + 255) / 256);
   if (c->act_dtype == MOE_BF16 && c->out_dtype == MOE_BF16)
-    k_combine<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, st>>>(
+    MOE_LAUNCH((k_combine<__nv_bfloat16, __nv_bfloat16>), blocks, 256, 0, st, 
         y, slot, ys, c->n_shared, static_cast<const __nv_bfloat16*>(res),
         static_cast<__nv_bfloat16*>(out), c->T, c->d, c->k);
   else if (c->act_dtype == MOE_BF16)
-    k_combine<__nv_bfloat16, float><<<blocks, 256, 0, st>>>(
+    MOE_LAUNCH((k_combine<__nv_bfloat16, float>), blocks, 256, 0, st, 
         y, slot, ys, c->n_shared, static_cast<const __nv_bfloat16*>(res),
         static_cast<float*>(out), c->T, c->d, c->k);
   else
-    k_combine<float, float><<<blocks, 256, 0, st>>>(y, slot, ys, c->n_shared,
+    MOE_LAUNCH((k_combine<float, float>), blocks, 256, 0, st, y, slot, ys, c->n_shared,
                                                     static_cast<const float*>(res),
                                                     static_cast<float*>(out), c->T, c->d, c->k);
   return check_launch();
@@ -619,7 +656,7 @@ moe_status moe_permute_static(const moe_config* cfg, const int32_t* topk_idx, in
     if (cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
-    k_permute<<<1, 1024, smem, st>>>(topk_idx, n, E, cap, counts, offsets, perm_assign, slot_of,
+    MOE_LAUNCH((k_permute), 1, 1024, smem, st, topk_idx, n, E, cap, counts, offsets, perm_assign, slot_of,
                                      n_dropped, nullptr);
     return check_launch();
   }
@@ -630,9 +667,9 @@ moe_status moe_permute_static(const moe_config* cfg, const int32_t* topk_idx, in
   if (cudaFuncSetAttribute(k_perm_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  k_perm_count<<<nb, 256, sm1, st>>>(topk_idx, n, E, nb, blk, nullptr);
-  k_perm_scan<<<1, 1024, 0, st>>>(blk, nb, E, cap, counts, offsets, n_dropped);
-  k_perm_rank<<<nb, 256, sm3, st>>>(topk_idx, n, E, nb, cap, blk, offsets, perm_assign, slot_of);
+  MOE_LAUNCH((k_perm_count), nb, 256, sm1, st, topk_idx, n, E, nb, blk, nullptr);
+  MOE_LAUNCH((k_perm_scan), 1, 1024, 0, st, blk, nb, E, cap, counts, offsets, n_dropped);
+  MOE_LAUNCH((k_perm_rank), nb, 256, sm3, st, topk_idx, n, E, nb, cap, blk, offsets, perm_assign, slot_of);
   return check_launch();
 }
 
