@@ -101,10 +101,10 @@ typedef struct moe_config {
  *   s_gate/s_up INT8: bf16 [E, f]; INT4: bf16 [E, d/128, f]; otherwise NULL
  *   s_down      INT8: bf16 [E, d]; INT4: bf16 [E, f/128, d]; otherwise NULL
  *   sh_*        the same for the n_shared shared experts ([S, ...]); NULL if S == 0
- * int8 weights are symmetric: w = q * s per output column.  int4 weights are
+ * int8 weights are symmetric with one scale per output column; int4 weights are
  * symmetric signed 4-bit, two per byte along the contiguous dim (low nibble =
- * even column); the weight the layer uses is bf16(q * s) with one scale per 128
- * rows of K. */
+ * even column), with one scale per 128 rows of K and output column.  Either way
+ * the weight the layer uses is bf16(q * s): the exact product rounded once. */
 typedef struct moe_weights {
   const void* rms_gamma;
   const void* w_router;

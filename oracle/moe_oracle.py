@@ -40,7 +40,8 @@ Readings where the pages are silent (each is listed in the design doc):
   ``< cap``.  Kept slots keep their gate (no re-renormalisation).
 * Expert: SwiGLU, ``y = (silu(xn Wg) * (xn Wu)) Wd``.
 * Combine: ``out = x + sum_s shared_s(xn) + sum_{kept j} g_j * y_j``.
-* int4 weights dequantise to ``bf16(q * s)``; int8 weights to ``q * s`` exactly.
+* int8 and int4 weights dequantise to ``bf16(q * s)`` (the exact product rounded
+  once to bf16): the layer's tensor-core GEMMs consume bf16 weights.
 """
 from __future__ import annotations
 
@@ -224,8 +225,8 @@ def unpack_int4(packed) -> np.ndarray:
 
 
 def dequant_int8(q, s) -> np.ndarray:
-    """w[K, N] = q[K, N] * s[N] (exact in float64)."""
-    return np.asarray(q, np.float64) * np.asarray(s, np.float64)[None, :]
+    """w[K, N] = bf16(q[K, N] * s[N])."""
+    return round_bf16(np.asarray(q, np.float64) * np.asarray(s, np.float64)[None, :])
 
 
 def dequant_int4(packed, s, group: int) -> np.ndarray:

@@ -253,7 +253,9 @@ def test_quantised_weights_within_quantisation_bound():
     w = torch.from_numpy(rng(11).standard_normal((256, 64)).astype(np.float32)) * 0.05
     q8, s8 = moe_synth.quantize_int8(w)
     dq8 = O.dequant_int8(q8.numpy(), s8.float().numpy())
-    assert np.all(np.abs(dq8 - w.numpy()) <= 0.5 * s8.float().numpy()[None, :] * (1 + 1e-6))
+    bound8 = 0.5 * s8.float().numpy()[None, :] + np.abs(dq8) * 2.0 ** -8
+    assert np.all(np.abs(dq8 - w.numpy()) <= bound8 * (1 + 1e-6))
+    np.testing.assert_array_equal(dq8, O.round_bf16(dq8))
     p4, s4 = moe_synth.quantize_int4(w, 128)
     dq4 = O.dequant_int4(p4.numpy(), s4.float().numpy(), 128)
     s_full = np.repeat(s4.float().numpy(), 128, axis=0)
