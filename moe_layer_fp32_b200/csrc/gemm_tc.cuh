@@ -41,9 +41,16 @@
 namespace moe {
 
 enum Epi : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_ROUTER = 2 };
+// weight storage: bf16, or weight-only int8 / int4 dequantised to bf16(q * s) in
+// the main loop
+enum WQuant : int { WQ_BF16 = 0, WQ_INT8 = 1, WQ_INT4 = 2 };
 
-constexpr int kTcThreads = 320;
+constexpr int kTcBaseThreads = 320;   // producer, MMA, 8 epilogue warps
 constexpr int kEpiWarps = 8;
+// dequantisation warps for int8 / int4 weights (int4 is bound by shared-memory
+// bandwidth already at 8; int8's longer conversion gains from 16)
+template <int WQ>
+struct DeqWarps { static constexpr int value = WQ == 1 ? 16 : 8; };
 constexpr int kMaxGroups = 512;
 
 struct TcProblem {
@@ -63,6 +70,11 @@ struct TcProblem {
   const int32_t* perm_assign; // routed DOWN: output row = perm_assign[slot]
   const float* gate;          // routed DOWN: scale
   int n_valid;                // features actually stored (n < n_valid)
+  // int8 / int4 weights: tmA / tmA2 then map the raw bytes (uint8, no swizzle)
+  // and tmS / tmS2 their bf16 scales, [G][N] (int8) or [G][K/128][N] (int4), box
+  // 128 features
+  CUtensorMap tmS;
+  CUtensorMap tmS2;
 };
 
 struct TcParams {
@@ -88,15 +100,37 @@ struct TcShape {
   static constexpr int TILE_N = (EPI == EPI_DOWN && DIRECT) ? 256 : 128;   // features per tile
 };
 
-template <int EPI, int BN, bool DIRECT>
+template <int EPI, int BN, bool DIRECT, int WQ = WQ_BF16>
 struct TcConfig {
   static constexpr int NA = TcShape<EPI, DIRECT>::NA;
   static constexpr int TILE_N = TcShape<EPI, DIRECT>::TILE_N;
   static constexpr uint32_t A_BYTES = TcShape<EPI, DIRECT>::A_BYTES;
   static constexpr uint32_t B_BYTES = BN * 64 * 2;
-  static constexpr uint32_t STAGE_BYTES = NA * A_BYTES + B_BYTES;
-  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  // raw quantised weight block (128 features x 64 k): int8 128 B rows, int4 64 B rows
+  static constexpr uint32_t RAW_BYTES = WQ == WQ_INT8 ? 128 * 64 : WQ == WQ_INT4 ? 64 * 64 : 0;
+  static constexpr uint32_t RAW_ROW = WQ == WQ_INT8 ? 128 : 64;
+  static constexpr uint32_t SCALE_BYTES = WQ == WQ_BF16 ? 0 : 256;   // 128 bf16 scales
+  // bf16 weights: one ring of TMA stages [weights NA x 16 KB | tokens].
+  // int8 / int4 weights: a deep ring of TMA stages [tokens | raw weights | scales
+  // in a 1 KB slot] (so that enough weight bytes are in flight to cover HBM
+  // latency) and AS slots of dequantised bf16 weights that the dequantisation
+  // warps fill and the MMA drains.  Every stage and slot is 1024-byte aligned.
+  static constexpr int AS = WQ == WQ_BF16 ? 0 : 2;
+  static constexpr uint32_t A_SLOT_BYTES = NA * A_BYTES;
+  static constexpr uint32_t STAGE_BYTES =
+      WQ == WQ_BF16 ? NA * A_BYTES + B_BYTES : B_BYTES + NA * RAW_BYTES + 1024;
+  static constexpr uint32_t TOKEN_OFF = WQ == WQ_BF16 ? NA * A_BYTES : 0;
+  static constexpr uint32_t RAW_OFF = B_BYTES;
+  static constexpr uint32_t SCALE_OFF = B_BYTES + NA * RAW_BYTES;
+  // bytes the TMA delivers per stage
+  static constexpr uint32_t TX_BYTES =
+      WQ == WQ_BF16 ? STAGE_BYTES : B_BYTES + NA * (RAW_BYTES + SCALE_BYTES);
+  static constexpr int DEQ_WARPS = DeqWarps<WQ>::value;
+  static constexpr int THREADS = kTcBaseThreads + (WQ == WQ_BF16 ? 0 : 32 * DEQ_WARPS);
+  static constexpr int STAGES_RAW = (200 * 1024 - AS * A_SLOT_BYTES) / STAGE_BYTES;
+  static constexpr int STAGE_CAP = WQ == WQ_BF16 ? 8 : 16;
+  static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
+  static constexpr uint32_t A_REGION = AS * A_SLOT_BYTES;
   static constexpr uint32_t ACC_COLS = NA * BN;
   static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
@@ -109,14 +143,16 @@ struct TcConfig {
   static constexpr uint32_t IDESC = DIRECT ? idesc_bf16(128, 128 * NA, false, true)
                                            : idesc_bf16(128, BN, true, false);
   // barriers + bookkeeping after the tiles
-  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
+  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * 2) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
   // swapped epilogue: per-tile output row and scale of each token, one copy per warp
   static constexpr uint32_t EPI_BYTES = kEpiWarps * 128 * 8;
   static constexpr uint32_t SMEM_BYTES =
-      1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES + EPI_BYTES;
+      1024 + STAGES * STAGE_BYTES + A_REGION + BAR_BYTES + PREFIX_BYTES + EPI_BYTES;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
   static_assert(!DIRECT || BN == 128, "direct tiles hold 128 tokens");
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 128-byte swizzle alignment");
+  static_assert(NA * SCALE_BYTES <= 1024, "scale slot");
   static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
 };
 
@@ -169,25 +205,115 @@ MOE_DEV int total_tiles(const TcParams& p, const int* prefix, int TN) {
 
 MOE_DEV float silu_f(float u) { return __fdividef(u, 1.f + __expf(-u)); }
 
-template <int EPI, int BN, bool DIRECT>
-__global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant__ TcParams p) {
-  using C = TcConfig<EPI, BN, DIRECT>;
+// Dequantise one raw weight block (128 features x 64 k of tile (g, n, kb)) into the
+// bf16 MN-major layout with the 128-byte swizzle that a TMA load would have
+// produced: 16-byte chunk cc (8 features) of k-row k of 64-feature half h sits at
+// h * 8192 + k * 128 + ((cc ^ (k & 7)) << 4).  Value = bf16(q * s), the exact
+// product rounded once; the block's 128 scales were loaded by the TMA with it.
+// Features at or beyond N were zero-filled by the TMA (q = 0, s = 0).
+// Eight int4 values (two's complement nibbles, nibble j = feature j) to bf16 q*s,
+// packed as four bf16x2 pairs of consecutive features.  XOR 8 turns each nibble
+// into the offset value q + 8 in [0, 15]; OR-ing it into the low mantissa bits of
+// bf16 128.0 (0x4300) gives exactly 136 + q; subtracting 136.0 (0x4308) leaves q
+// exactly; byte permutes restore feature order and one bf16x2 multiply by the
+// scale pair yields the exact product q*s rounded once (round to nearest even).
+MOE_DEV void int4x8_to_bf16(uint32_t v, const uint32_t (&s2)[4], uint32_t (&o)[4]) {
+  v ^= 0x88888888u;
+  const uint32_t magic = 0x43004300u;
+  uint32_t a = (v & 0x000F000Fu) | magic;           // features (0, 4)
+  uint32_t b = ((v >> 4) & 0x000F000Fu) | magic;    // (1, 5)
+  uint32_t c = ((v >> 8) & 0x000F000Fu) | magic;    // (2, 6)
+  uint32_t d = ((v >> 12) & 0x000F000Fu) | magic;   // (3, 7)
+  const __nv_bfloat162 k136 = __halves2bfloat162(__ushort_as_bfloat16(0x4308),
+                                                 __ushort_as_bfloat16(0x4308));
+  __nv_bfloat162 qa = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), k136);
+  __nv_bfloat162 qb = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&b), k136);
+  __nv_bfloat162 qc = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&c), k136);
+  __nv_bfloat162 qd = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&d), k136);
+  const uint32_t ua = *reinterpret_cast<uint32_t*>(&qa), ub = *reinterpret_cast<uint32_t*>(&qb);
+  const uint32_t uc = *reinterpret_cast<uint32_t*>(&qc), ud = *reinterpret_cast<uint32_t*>(&qd);
+  uint32_t p[4] = {__byte_perm(ua, ub, 0x5410), __byte_perm(uc, ud, 0x5410),
+                   __byte_perm(ua, ub, 0x7632), __byte_perm(uc, ud, 0x7632)};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&p[i]),
+                               *reinterpret_cast<const __nv_bfloat162*>(&s2[i]));
+    o[i] = *reinterpret_cast<uint32_t*>(&r);
+  }
+}
+
+// Dequantise one raw weight block (128 features x 64 k of tile (g, n, kb)) into the
+// bf16 MN-major layout with the 128-byte swizzle that a TMA load would have
+// produced: 16-byte chunk cc (8 features) of k-row k of 64-feature half h sits at
+// h * 8192 + k * 128 + ((cc ^ (k & 7)) << 4).  Value = bf16(q * s), the exact
+// product rounded once; the block's 128 scales were loaded by the TMA with it.
+// Features at or beyond N were zero-filled by the TMA (q = 0, s = 0).
+template <int WQ, int NTHREADS>
+MOE_DEV void dequant_block(const uint8_t* raw, uint8_t* out, const __nv_bfloat16* ssm, int t) {
+  constexpr int RAW_ROW = WQ == WQ_INT8 ? 128 : 64;
+  constexpr int ITERS = 64 * 16 / NTHREADS;
+  static_assert(64 * 16 % NTHREADS == 0, "whole chunks per thread");
+  // the column chunk of thread t is the same in every iteration (16 | NTHREADS):
+  // load its scales once, then all raw words, then convert
+  const int c = t & 15;
+  const uint4 sv = *reinterpret_cast<const uint4*>(ssm + c * 8);
+  uint32_t w4[ITERS];
+  uint2 w8[ITERS];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int k = (t + it * NTHREADS) >> 4;
+    if (WQ == WQ_INT4) w4[it] = *reinterpret_cast<const uint32_t*>(raw + k * RAW_ROW + c * 4);
+    else w8[it] = *reinterpret_cast<const uint2*>(raw + k * RAW_ROW + c * 8);
+  }
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int k = (t + it * NTHREADS) >> 4;
+    uint32_t pk[4];
+    if (WQ == WQ_INT4) {
+      const uint32_t s2[4] = {sv.x, sv.y, sv.z, sv.w};
+      int4x8_to_bf16(w4[it], s2, pk);
+    } else {
+      const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv);
+      const uint2 v = w8[it];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t w = i < 2 ? v.x : v.y;
+        const int sh = (i & 1) * 16;
+        const float q0 = (float)(int8_t)((w >> sh) & 0xff);
+        const float q1 = (float)(int8_t)((w >> (sh + 8)) & 0xff);
+        __nv_bfloat162 h2 =
+            __floats2bfloat162_rn(q0 * __low2float(s2[i]), q1 * __high2float(s2[i]));
+        pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+    }
+    *reinterpret_cast<uint4*>(out + (c >> 3) * 8192 + k * 128 + (((c & 7) ^ (k & 7)) << 4)) =
+        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+template <int EPI, int BN, bool DIRECT, int WQ>
+__global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
+    k_tc_gemm(const __grid_constant__ TcParams p) {
+  using C = TcConfig<EPI, BN, DIRECT, WQ>;
   constexpr int NA = C::NA;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
+  uint8_t* aslots = tiles + STAGES * C::STAGE_BYTES;   // dequantised weights (int8 / int4)
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(aslots + C::A_REGION);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;       // [2]
   uint64_t* drain_bar = tempty_bar + 2;       // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* deq_bar = drain_bar + 1;          // [2] dequantised slot filled
+  uint64_t* aempty_bar = deq_bar + 2;         // [2] dequantised slot consumed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aempty_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
   int* prefix = reinterpret_cast<int*>(
-      reinterpret_cast<uint8_t*>(smem) + STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+      reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
   int* epi_row = prefix + 2 * (kMaxGroups + 1);                          // [8 warps][128]
   float* epi_scale = reinterpret_cast<float*>(epi_row + kEpiWarps * 128);  // [8 warps][128]
 
@@ -198,6 +324,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
       issued[s] = 0;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&deq_bar[a], C::DEQ_WARPS);
+      mbar_init(&aempty_bar[a], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
@@ -248,18 +378,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag)) { ok = false; break; }
           uint8_t* st = tiles + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          mbar_arrive_expect_tx(&full_bar[stage], C::TX_BYTES);
           issued[stage] = (int)phase + 1;
-          tma_load_3d(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g);
-          tma_load_3d(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g);
-          if (NA == 2) {
-            // GATEUP: the up matrix at the same features; wide DOWN: features +128
-            const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
-            const int n2 = (EPI == EPI_GATEUP) ? ti.n0 : ti.n0 + 128;
-            tma_load_3d(st + C::A_BYTES, m2, &full_bar[stage], n2, kb * 64, ti.g);
-            tma_load_3d(st + C::A_BYTES + 8192, m2, &full_bar[stage], n2 + 64, kb * 64, ti.g);
+          // GATEUP: the up matrix at the same features; wide DOWN: features +128
+          const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
+          const int n2 = (EPI == EPI_GATEUP) ? ti.n0 : ti.n0 + 128;
+          if (WQ == WQ_BF16) {
+            tma_load_3d(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g);
+            tma_load_3d(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g);
+            if (NA == 2) {
+              tma_load_3d(st + C::A_BYTES, m2, &full_bar[stage], n2, kb * 64, ti.g);
+              tma_load_3d(st + C::A_BYTES + 8192, m2, &full_bar[stage], n2 + 64, kb * 64, ti.g);
+            }
+          } else {
+            // raw bytes: x is the byte column (two int4 values per byte)
+            uint8_t* raw = st + C::RAW_OFF;
+            uint8_t* scl = st + C::SCALE_OFF;
+            const int div = WQ == WQ_INT4 ? 2 : 1;
+            const void* s2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmS2 : (const void*)&P.tmS;
+            tma_load_3d(raw, &P.tmA, &full_bar[stage], ti.n0 / div, kb * 64, ti.g);
+            // int8: scales [G][N] (second coordinate g, third 0); int4: [G][K/128][N]
+            if (WQ == WQ_INT8) tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, ti.g, 0);
+            else tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, kb / 2, ti.g);
+            if (NA == 2) {
+              tma_load_3d(raw + C::RAW_BYTES, m2, &full_bar[stage], n2 / div, kb * 64, ti.g);
+              if (WQ == WQ_INT8) tma_load_3d(scl + 256, s2, &full_bar[stage], n2, ti.g, 0);
+              else tma_load_3d(scl + 256, s2, &full_bar[stage], n2, kb / 2, ti.g);
+            }
           }
-          tma_load_2d(st + NA * C::A_BYTES, &P.tmB, &full_bar[stage], kb * 64, ti.b_row);
+          tma_load_2d(st + C::TOKEN_OFF, &P.tmB, &full_bar[stage], kb * 64, ti.b_row);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -270,6 +417,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int aslot = 0;
+      uint32_t aphase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -282,9 +431,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag)) { ok = false; break; }
+          if (WQ != WQ_BF16 &&
+              !mbar_wait(&deq_bar[aslot], aphase, p.err, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(tiles + stage * C::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + NA * C::A_BYTES;
+          const uint32_t st_addr = smem_u32(tiles + stage * C::STAGE_BYTES);
+          const uint32_t a_addr =
+              WQ == WQ_BF16 ? st_addr : smem_u32(aslots + aslot * C::A_SLOT_BYTES);
+          const uint32_t b_addr = st_addr + C::TOKEN_OFF;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             // weights: MN-major SW128, 16 k-rows of 128 B per MMA step; the two
@@ -305,6 +458,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
           }
           tc_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (WQ != WQ_BF16) {
+            tc_commit(&aempty_bar[aslot]);
+            if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+          }
         }
         if (!ok) break;
         tc_commit(&tfull_bar[acc]);
@@ -317,6 +474,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_gemm(const __grid_constant
       while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kWaitCycles) {}
     }
     __syncwarp();
+  } else if (warp >= 2 + kEpiWarps) {
+    // ------------------------------------------------------------ dequantisation
+    if (WQ != WQ_BF16) {
+      const int dt = threadIdx.x - 32 * (2 + kEpiWarps);
+      int stage = 0;
+      uint32_t phase = 0;
+      int aslot = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, TN, tile, ti);
+        const TcProblem& P = p.prob[ti.prob];
+        const int kblocks = P.K / 64;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&aempty_bar[aslot], aphase ^ 1, p.err, abort_flag)) { ok = false; break; }
+          uint8_t* st = tiles + stage * C::STAGE_BYTES;
+          uint8_t* dst = aslots + aslot * C::A_SLOT_BYTES;
+          const uint8_t* raw = st + C::RAW_OFF;
+          const __nv_bfloat16* scl = reinterpret_cast<const __nv_bfloat16*>(st + C::SCALE_OFF);
+#pragma unroll
+          for (int i = 0; i < NA; ++i)
+            dequant_block<WQ, 32 * C::DEQ_WARPS>(raw + i * C::RAW_BYTES, dst + i * C::A_BYTES,
+                                                 scl + 128 * i, dt);
+          // generic-proxy stores must be visible to the tensor core (async proxy)
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&deq_bar[aslot]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quadrant of this warp

@@ -639,6 +639,83 @@ __global__ void __launch_bounds__(256) k_perm_rank(const int32_t* __restrict__ i
 }
 
 // ---------------------------------------------------------------------------
+// Dequantise whole expert matrices to bf16 (prefill batches with int8 / int4
+// experts): w = bf16(q * s), the exact product rounded once, 8 outputs per
+// thread per step.  Experts that received no token are skipped when `offsets`
+// is given.  blockIdx.y = matrix, blockIdx.z = expert.
+// ---------------------------------------------------------------------------
+struct DeqMatrix {
+  const uint8_t* q;              // int8 [G][K][N] or packed int4 [G][K][N/2]
+  const __nv_bfloat16* s;        // [G][N] (int8) or [G][K/128][N] (int4)
+  __nv_bfloat16* out;            // [G][K][N]
+  const int32_t* offsets;        // [G+1] routed segments, or nullptr (dequantise all)
+  int G, K, N;
+};
+struct DeqArgs {
+  DeqMatrix m[6];
+  int n;
+};
+
+template <bool INT4>
+__global__ void __launch_bounds__(256) k_dequant_experts(const __grid_constant__ DeqArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  // block (x, y, z) = 8 rows of matrix y of expert z; thread (tx, ty) = row ty,
+  // 8-column chunks tx, tx + 32, ...
+  const DeqMatrix& M = a.m[blockIdx.y];
+  const int g = blockIdx.z;
+  if (g >= M.G) return;
+  if (M.offsets && M.offsets[g + 1] == M.offsets[g]) return;
+  const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (k >= M.K) return;
+  const int nch = M.N / 8;
+  const __nv_bfloat16* srow =
+      INT4 ? M.s + ((size_t)g * (M.K / 128) + k / 128) * M.N : M.s + (size_t)g * M.N;
+  const uint8_t* qrow = M.q + ((size_t)g * M.K + k) * (INT4 ? M.N / 2 : M.N);
+  __nv_bfloat16* orow = M.out + ((size_t)g * M.K + k) * M.N;
+  constexpr int U = 4;
+  for (int c0 = threadIdx.x & 31; c0 < nch; c0 += 32 * U) {
+    uint4 sv[U];
+    uint32_t v4[U];
+    uint2 v8[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nch) {
+        sv[u] = *reinterpret_cast<const uint4*>(srow + c * 8);
+        if (INT4) v4[u] = *reinterpret_cast<const uint32_t*>(qrow + c * 4);
+        else v8[u] = *reinterpret_cast<const uint2*>(qrow + c * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c >= nch) break;
+      const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv[u]);
+      float q[8];
+      if (INT4) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = (float)((int)(v4[u] << (28 - 4 * i)) >> 28);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          q[i] = (float)(int8_t)((v8[u].x >> (8 * i)) & 0xff);
+          q[4 + i] = (float)(int8_t)((v8[u].y >> (8 * i)) & 0xff);
+        }
+      }
+      uint32_t pk[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(q[2 * i] * __low2float(s2[i]),
+                                                  q[2 * i + 1] * __high2float(s2[i]));
+        pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      *reinterpret_cast<uint4*>(orow + c * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // gather: xp[s] = xn[perm_assign[s] / k] for s < offsets[E]; one warp per row,
 // 16-byte vectors (d * sizeof(TA) is a multiple of 16).
 // ---------------------------------------------------------------------------

@@ -47,8 +47,24 @@ inline int router_slice(const moe_config* c, int ns) {
   return (s + 7) / 8 * 8;
 }
 
+// token-tile width of the expert GEMMs from the mean rows per expert
+int pick_bn(const moe_config* c) {
+  const double mean = (double)c->T * c->k / c->E;
+  if (mean <= 16) return 16;
+  if (mean <= 32) return 32;
+  if (mean <= 64) return 64;
+  return 128;
+}
+// Quantised experts at prefill tile widths are dequantised once to bf16 in the
+// workspace (the in-loop dequantisation would repeat for every token tile of an
+// expert); decode tiles dequantise inside the GEMM main loop.
+inline bool dequant_once(const moe_config* c) {
+  return (c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4) && pick_bn(c) == 128;
+}
+
 struct Layout {
-  size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, h, y, ys, total;
+  size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, h, y, ys, deq,
+      total;
   int ns;
 };
 
@@ -74,7 +90,10 @@ moe_status validate(const moe_config* c) {
       break;
     case MOE_INT8:
     case MOE_INT4:
-      return MOE_ERR_UNSUPPORTED;
+      if (c->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+      if (c->d % 128 || c->f % 128 || c->E % 8) return MOE_ERR_UNSUPPORTED;
+      if (c->expert_dtype == MOE_INT4 && c->group_size != 128) return MOE_ERR_UNSUPPORTED;
+      break;
     default:
       return MOE_ERR_INVALID;
   }
@@ -103,6 +122,7 @@ Layout layout(const moe_config* c) {
   L.h = o;        o = align_up(o + (T * k + S * T) * f * hb);
   L.y = o;        o = align_up(o + T * k * d * 4);
   L.ys = o;       o = align_up(o + S * T * d * 4);
+  L.deq = o;      o = align_up(o + (dequant_once(c) ? (E + S) * 3 * d * f * 2 : 0));
   L.total = o;
   return L;
 }
@@ -194,6 +214,48 @@ bool map_weights(CUtensorMap* m, const void* base, int G, int K, int N) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// raw quantised weights [G][K][NB] bytes (NB = N for int8, N/2 for int4), no
+// swizzle; box = one 128-feature block x 64 k
+bool map_raw(CUtensorMap* m, const void* base, int G, int K, int NB, int box_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)NB, (cuuint64_t)K, (cuuint64_t)G};
+  cuuint64_t strides[2] = {(cuuint64_t)NB, (cuuint64_t)K * NB};
+  cuuint32_t box[3] = {(cuuint32_t)box_bytes, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// quantisation scales, bf16: int8 [G][N] as (N, G, 1); int4 [G][K/128][N] as
+// (N, K/128, G); box 128 features
+bool map_scales(CUtensorMap* m, const moe_config* c, const void* base, int G, int K, int N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base) return false;
+  const bool i4 = c->expert_dtype == MOE_INT4;
+  const cuuint64_t kg = i4 ? (cuuint64_t)(K / 128) : (cuuint64_t)G;
+  const cuuint64_t g3 = i4 ? (cuuint64_t)G : 1;
+  cuuint64_t dims[3] = {(cuuint64_t)N, kg, g3};
+  cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)N * 2 * kg};
+  cuuint32_t box[3] = {128, 1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// expert weight matrix [G][K][N] in the storage the GEMM reads (wq)
+bool map_expert(CUtensorMap* m, int wq, const void* base, int G, int K, int N) {
+  if (wq == WQ_INT8) return map_raw(m, base, G, K, N, 128);
+  if (wq == WQ_INT4) return map_raw(m, base, G, K, N / 2, 64);
+  return map_weights(m, base, G, K, N);
+}
+
+inline int wq_of(const moe_config* c) {
+  return c->expert_dtype == MOE_INT8 ? WQ_INT8 : c->expert_dtype == MOE_INT4 ? WQ_INT4 : WQ_BF16;
+}
+
 // activations [R][K] bf16, K contiguous; box 64 k x BN rows
 bool map_rows(CUtensorMap* m, const void* base, int R, int K, int BN) {
   EncodeTiledFn fn = encode_fn();
@@ -207,35 +269,36 @@ bool map_rows(CUtensorMap* m, const void* base, int R, int K, int BN) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, int BN, bool DIRECT = false>
+template <int EPI, int BN, bool DIRECT = false, int WQ = WQ_BF16>
 moe_status launch_tc(const TcParams& p, cudaStream_t st) {
-  using C = TcConfig<EPI, BN, DIRECT>;
-  auto kern = k_tc_gemm<EPI, BN, DIRECT>;
+  using C = TcConfig<EPI, BN, DIRECT, WQ>;
+  auto kern = k_tc_gemm<EPI, BN, DIRECT, WQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  MOE_LAUNCH((kern), num_sms(), kTcThreads, C::SMEM_BYTES, st, p);
+  MOE_LAUNCH((kern), num_sms(), C::THREADS, C::SMEM_BYTES, st, p);
   return check_launch();
 }
 
-template <int EPI>
-moe_status launch_tc_bn(int bn, const TcParams& p, cudaStream_t st) {
+template <int EPI, int WQ>
+moe_status launch_tc_bn_q(int bn, const TcParams& p, cudaStream_t st) {
   switch (bn) {
-    case 16: return launch_tc<EPI, 16>(p, st);
-    case 32: return launch_tc<EPI, 32>(p, st);
-    case 64: return launch_tc<EPI, 64>(p, st);
-    default: return launch_tc<EPI, 128, true>(p, st);   // prefill tiles: tokens on MMA-M
+    case 16: return launch_tc<EPI, 16, false, WQ>(p, st);
+    case 32: return launch_tc<EPI, 32, false, WQ>(p, st);
+    case 64: return launch_tc<EPI, 64, false, WQ>(p, st);
+    default:   // prefill tiles: tokens on MMA-M (quantised weights are dequantised first)
+      if constexpr (WQ == WQ_BF16) return launch_tc<EPI, 128, true, WQ>(p, st);
+      else return MOE_ERR_UNSUPPORTED;
   }
 }
 
-// token-tile width of the expert GEMMs from the mean rows per expert
-int pick_bn(const moe_config* c) {
-  double mean = (double)c->T * c->k / c->E;
-  if (mean <= 16) return 16;
-  if (mean <= 32) return 32;
-  if (mean <= 64) return 64;
-  return 128;
+template <int EPI>
+moe_status launch_tc_bn(int bn, int wq, const TcParams& p, cudaStream_t st) {
+  if (wq == WQ_INT8) return launch_tc_bn_q<EPI, WQ_INT8>(bn, p, st);
+  if (wq == WQ_INT4) return launch_tc_bn_q<EPI, WQ_INT4>(bn, p, st);
+  return launch_tc_bn_q<EPI, WQ_BF16>(bn, p, st);
 }
+
 
 int capacity_rows(const moe_config* c) {
   if (!(c->capacity_factor > 0.f)) return INT_MAX;
@@ -376,6 +439,10 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   const int T = c->T, k = c->k, S = c->n_shared;
   if (!w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID;
   if (S > 0 && (!w->sh_gate || !w->sh_up || !w->sh_down || !ys)) return MOE_ERR_INVALID;
+  if (c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4) {
+    if (!w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID;
+    if (S > 0 && (!w->sh_s_gate || !w->sh_s_up || !w->sh_s_down)) return MOE_ERR_INVALID;
+  }
   if (!tc_experts(c)) {
     SimtArgs a{};
     a.xn = static_cast<const float*>(xn);
@@ -402,22 +469,58 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     mk->mark(st);
     return s;
   }
-  // bf16 experts: gather the routed rows, then gate/up and down on the tensor cores
+  // tensor-core experts: [dequantise once], gather the routed rows, then gate/up and
+  // down on the tensor cores
   __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
   __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
-  MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 2 * num_sms(), 256, 0, st, 
-      static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
-  moe_status s = check_launch();
-  if (s != MOE_OK) return s;
-  mk->mark(st);
   const int bn = pick_bn(c);
   const int R = T * k;
+  int wq = wq_of(c);
+  moe_weights wl = *w;                     // the weights the GEMMs read
+  moe_status s = MOE_OK;
+  if (dequant_once(c)) {
+    const size_t per = (size_t)c->d * c->f;
+    __nv_bfloat16* base = at<__nv_bfloat16>(ws, L.deq);
+    __nv_bfloat16* dst[6];
+    for (int i = 0; i < 3; ++i) dst[i] = base + (size_t)i * c->E * per;
+    for (int i = 0; i < 3; ++i) dst[3 + i] = base + (size_t)3 * c->E * per + (size_t)i * S * per;
+    DeqArgs a{};
+    const void* srcq[6] = {w->w_gate, w->w_up, w->w_down, w->sh_gate, w->sh_up, w->sh_down};
+    const void* srcs[6] = {w->s_gate, w->s_up, w->s_down, w->sh_s_gate, w->sh_s_up, w->sh_s_down};
+    a.n = S > 0 ? 6 : 3;
+    for (int i = 0; i < a.n; ++i) {
+      DeqMatrix& m = a.m[i];
+      m.q = static_cast<const uint8_t*>(srcq[i]);
+      m.s = static_cast<const __nv_bfloat16*>(srcs[i]);
+      m.out = dst[i];
+      m.offsets = i < 3 ? offsets : nullptr;
+      m.G = i < 3 ? c->E : S;
+      m.K = (i % 3 == 2) ? c->f : c->d;
+      m.N = (i % 3 == 2) ? c->d : c->f;
+    }
+    // 8 rows of one matrix per block (K is d or f, both multiples of 128)
+    const int kmax = c->d > c->f ? c->d : c->f;
+    dim3 grid(kmax / 8, a.n, c->E > S ? c->E : S);
+    if (wq == WQ_INT4) MOE_LAUNCH((k_dequant_experts<true>), grid, 256, 0, st, a);
+    else MOE_LAUNCH((k_dequant_experts<false>), grid, 256, 0, st, a);
+    if ((s = check_launch()) != MOE_OK) return s;
+    wl.w_gate = dst[0]; wl.w_up = dst[1]; wl.w_down = dst[2];
+    wl.sh_gate = dst[3]; wl.sh_up = dst[4]; wl.sh_down = dst[5];
+    wq = WQ_BF16;
+  }
+  MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 2 * num_sms(), 256, 0, st,
+             static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
+  if ((s = check_launch()) != MOE_OK) return s;
+  mk->mark(st);
   {
     TcParams p{};
     TcProblem& P = p.prob[0];
-    if (!map_weights(&P.tmA, w->w_gate, c->E, c->d, c->f)) return MOE_ERR_CUDA;
-    if (!map_weights(&P.tmA2, w->w_up, c->E, c->d, c->f)) return MOE_ERR_CUDA;
+    if (!map_expert(&P.tmA, wq, wl.w_gate, c->E, c->d, c->f)) return MOE_ERR_CUDA;
+    if (!map_expert(&P.tmA2, wq, wl.w_up, c->E, c->d, c->f)) return MOE_ERR_CUDA;
     if (!map_rows(&P.tmB, xp, R, c->d, bn)) return MOE_ERR_CUDA;
+    if (wq != WQ_BF16 && (!map_scales(&P.tmS, c, w->s_gate, c->E, c->d, c->f) ||
+                          !map_scales(&P.tmS2, c, w->s_up, c->E, c->d, c->f)))
+      return MOE_ERR_CUDA;
     P.offsets = offsets;
     P.G = c->E;
     P.N = c->f;
@@ -429,9 +532,12 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     p.n_prob = 1;
     if (S > 0) {
       TcProblem& Q = p.prob[1];
-      if (!map_weights(&Q.tmA, w->sh_gate, S, c->d, c->f)) return MOE_ERR_CUDA;
-      if (!map_weights(&Q.tmA2, w->sh_up, S, c->d, c->f)) return MOE_ERR_CUDA;
+      if (!map_expert(&Q.tmA, wq, wl.sh_gate, S, c->d, c->f)) return MOE_ERR_CUDA;
+      if (!map_expert(&Q.tmA2, wq, wl.sh_up, S, c->d, c->f)) return MOE_ERR_CUDA;
       if (!map_rows(&Q.tmB, xn, T, c->d, bn)) return MOE_ERR_CUDA;
+      if (wq != WQ_BF16 && (!map_scales(&Q.tmS, c, w->sh_s_gate, S, c->d, c->f) ||
+                            !map_scales(&Q.tmS2, c, w->sh_s_up, S, c->d, c->f)))
+        return MOE_ERR_CUDA;
       Q.offsets = nullptr;
       Q.G = S;
       Q.uniform_rows = T;
@@ -446,15 +552,19 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
       p.n_prob = 2;
     }
     p.err = err;
-    s = launch_tc_bn<EPI_GATEUP>(bn, p, st);
+    s = launch_tc_bn<EPI_GATEUP>(bn, wq, p, st);
     if (s != MOE_OK) return s;
     mk->mark(st);
   }
   {
     TcParams p{};
     TcProblem& P = p.prob[0];
-    if (!map_weights(&P.tmA, w->w_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
+    if (!map_expert(&P.tmA, wq, wl.w_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
     P.tmA2 = P.tmA;
+    if (wq != WQ_BF16) {
+      if (!map_scales(&P.tmS, c, w->s_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
+      P.tmS2 = P.tmS;
+    }
     if (!map_rows(&P.tmB, h, R + S * T, c->f, bn)) return MOE_ERR_CUDA;
     P.offsets = offsets;
     P.G = c->E;
@@ -469,8 +579,12 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     p.n_prob = 1;
     if (S > 0) {
       TcProblem& Q = p.prob[1];
-      if (!map_weights(&Q.tmA, w->sh_down, S, c->f, c->d)) return MOE_ERR_CUDA;
+      if (!map_expert(&Q.tmA, wq, wl.sh_down, S, c->f, c->d)) return MOE_ERR_CUDA;
       Q.tmA2 = Q.tmA;
+      if (wq != WQ_BF16) {
+        if (!map_scales(&Q.tmS, c, w->sh_s_down, S, c->f, c->d)) return MOE_ERR_CUDA;
+        Q.tmS2 = Q.tmS;
+      }
       Q.tmB = P.tmB;
       Q.offsets = nullptr;
       Q.G = S;
@@ -488,7 +602,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
       p.n_prob = 2;
     }
     p.err = err;
-    s = launch_tc_bn<EPI_DOWN>(bn, p, st);
+    s = launch_tc_bn<EPI_DOWN>(bn, wq, p, st);
     mk->mark(st);
   }
   return s;
@@ -742,7 +856,7 @@ int32_t moe_layer_step_count(const moe_config* cfg) {
 int32_t moe_layer_launch_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
   const int perm = cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
-  return moe_layer_step_count(cfg) - 1 + perm;
+  return moe_layer_step_count(cfg) - 1 + perm + (dequant_once(cfg) ? 1 : 0);
 }
 
 }  // extern "C"

@@ -351,21 +351,31 @@ def moe_layer_dense(x, gamma, w_router, router_bias, experts: Weights, *, k: int
     return out
 
 
+def _npy(t):
+    if t is None:
+        return None
+    return t.float().numpy() if t.is_floating_point() else t.numpy()
+
+
+def weights_from_inputs(li, shared: bool = False) -> Optional[Weights]:
+    """Expert weights of a ``moe_synth.LayerInputs`` (host tensors); integer
+    storage stays integer."""
+    sh = li.shape
+    if shared and not sh.n_shared:
+        return None
+    pre = "sh_" if shared else ""
+    get = lambda n: _npy(getattr(li, pre + n))   # noqa: E731
+    return Weights(sh.expert, sh.group_size, get("w_gate" if not shared else "gate"),
+                   get("w_up" if not shared else "up"), get("w_down" if not shared else "down"),
+                   get("s_gate"), get("s_up"), get("s_down"))
+
+
 def layer_from_inputs(li, x, **kw) -> Dict[str, np.ndarray]:
     """Run ``moe_layer`` on a ``moe_synth.LayerInputs`` (host tensors)."""
     sh = li.shape
-
-    def npy(t):
-        if t is None:
-            return None
-        return t.float().numpy() if t.is_floating_point() else t.numpy()
-
-    experts = Weights(sh.expert, sh.group_size, npy(li.w_gate), npy(li.w_up), npy(li.w_down),
-                      npy(li.s_gate), npy(li.s_up), npy(li.s_down))
-    shared = None
-    if sh.n_shared:
-        shared = Weights(sh.expert, sh.group_size, npy(li.sh_gate), npy(li.sh_up),
-                         npy(li.sh_down), npy(li.sh_s_gate), npy(li.sh_s_up), npy(li.sh_s_down))
+    npy = _npy
+    experts = weights_from_inputs(li)
+    shared = weights_from_inputs(li, shared=True)
     args = dict(k=sh.k, act=sh.act, rms_eps=sh.rms_eps, bias_mode=sh.bias_mode,
                 renormalize=sh.renormalize, capacity_factor=sh.capacity_factor,
                 shared=shared, n_shared=sh.n_shared)

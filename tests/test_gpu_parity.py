@@ -24,9 +24,18 @@ SMALL = {
                                         bias_mode="select", renormalize=False, seed=13),
     "bf16_prefill_tiles": LayerShape("bf16_prefill", d=512, E=8, k=2, f=640, seed=14),
     "f32_tiny": moe_synth.PRESETS["tiny"],
+    "int4_decode": LayerShape("int4_decode", d=256, E=16, k=4, f=384, n_shared=1,
+                              expert="int4", seed=15),
+    "int8_decode": LayerShape("int8_decode", d=384, E=32, k=6, f=256, expert="int8",
+                              bias_mode="logit", seed=16),
+    "int4_prefill": LayerShape("int4_prefill", d=512, E=8, k=2, f=384, expert="int4",
+                               capacity_factor=1.25, seed=17),
+    "int8_prefill": LayerShape("int8_prefill", d=384, E=8, k=2, f=512, n_shared=1,
+                               expert="int8", seed=18),
 }
 SMALL_T = {"bf16_plain": 100, "bf16_shared_cap": 77, "bf16_select_tc_router": 200,
-           "bf16_prefill_tiles": 1000, "f32_tiny": 64}
+           "bf16_prefill_tiles": 1000, "f32_tiny": 64, "int4_decode": 20, "int8_decode": 50,
+           "int4_prefill": 900, "int8_prefill": 700}
 
 
 @pytest.fixture(autouse=True)
@@ -137,7 +146,8 @@ def test_permute_flags_out_of_range_expert():
 
 
 # --------------------------------------------------------------------- a6 + a7
-@pytest.mark.parametrize("name", ["bf16_plain", "bf16_shared_cap", "bf16_prefill_tiles", "f32_tiny"])
+@pytest.mark.parametrize("name", ["bf16_plain", "bf16_shared_cap", "bf16_prefill_tiles", "f32_tiny",
+                                  "int4_decode", "int8_decode", "int4_prefill", "int8_prefill"])
 def test_grouped_ffn_matches_oracle_per_assignment(name):
     sh, T = SMALL[name], SMALL_T[name]
     li, x, dli, dx = inputs_on_device(sh, T)
@@ -154,7 +164,7 @@ def test_grouped_ffn_matches_oracle_per_assignment(name):
                       ys if sh.n_shared else None, ws)
     assert M.moe_get_device_status(ws) == 0
     y = y.cpu().numpy()
-    ex = O.Weights(sh.expert, sh.group_size, *(t.float().numpy() for t in (li.w_gate, li.w_up, li.w_down)))
+    ex = O.weights_from_inputs(li)
     kept = np.nonzero(own["slot_of"] >= 0)[0]
     ref = np.zeros((T * sh.k, sh.d))
     bound = np.zeros((T * sh.k, sh.d))
@@ -181,7 +191,7 @@ def test_grouped_ffn_matches_oracle_per_assignment(name):
     rms = np.sqrt(np.mean(ref[kept] ** 2))
     print(f"{name}: max|dy|/rms(y) = {np.max(np.abs(y[kept] - ref[kept])) / rms:.3e}")
     if sh.n_shared:
-        shw = O.Weights(sh.expert, sh.group_size, *(t.float().numpy() for t in (li.sh_gate, li.sh_up, li.sh_down)))
+        shw = O.weights_from_inputs(li, shared=True)
         ysn = ys.cpu().numpy()
         for s in range(sh.n_shared):
             rs, bs = ffn_and_bound(shw, s, own["xn"])
@@ -271,7 +281,8 @@ def test_bf16_output_is_rounding_of_fp32_output():
 
 # --------------------------------------------------------------------- full sizes
 FULL = [("olmoe", 1), ("olmoe", 16), ("olmoe", 64), ("olmoe", 4096),
-        ("v2lite", 32), ("v2lite", 8192)]
+        ("v2lite", 32), ("v2lite", 8192), ("qwen3_int4", 1), ("qwen3_int4", 64),
+        ("qwen3_int4", 16384), ("qwen3_int8", 1), ("qwen3_int8", 64), ("qwen3_int8", 16384)]
 
 
 @pytest.mark.parametrize("preset,T", FULL)
