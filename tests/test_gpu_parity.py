@@ -305,10 +305,22 @@ def test_v2lite_capacity_factors(C):
     assert res.err_ratio <= TOL[sh.expert], res.err_ratio
 
 
+@pytest.fixture(scope="module")
+def v3_weights():
+    li = moe_synth.make_layer(moe_synth.PRESETS["v3"])
+    yield li, li.to("cuda")
+
+
 @pytest.mark.skipif(os.environ.get("MOE_FULL") != "1", reason="22.5 GB of weights; MOE_FULL=1")
 @pytest.mark.parametrize("T", [32, 256, 9440])
-def test_v3_full_size_sampled(T):
+def test_v3_full_size_sampled(T, v3_weights):
     sh = moe_synth.PRESETS["v3"]
-    res = run_layer(sh, T, tokens=sample_rows(T, 16))
-    assert res.max_margin_mismatch < ROUTE_MARGIN
+    li, dli = v3_weights
+    x = moe_synth.make_x(sh, T)
+    res = run_layer(sh, T, tokens=sample_rows(T, 16), data=(li, x, dli, x.cuda()))
+    assert res.max_margin_mismatch < ROUTE_MARGIN, (res.mismatched, res.max_margin_mismatch)
     assert res.err_ratio <= TOL[sh.expert], res.err_ratio
+    assert res.err_ratio_delta <= DELTA_GUARD[sh.expert], res.err_ratio_delta
+    print(f"v3 T={T}: mismatched routes {res.mismatched} (max margin "
+          f"{res.max_margin_mismatch:.2e}), err/rms(out) {res.err_ratio:.3e}, "
+          f"err/rms(delta) {res.err_ratio_delta:.3e}")
