@@ -52,6 +52,8 @@ def parse_args():
     p.add_argument("--tokens", type=int, default=4096)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--all-configs", action="store_true",
+                   help="also time every preset and token count (stream and CUDA graph)")
     return p.parse_args()
 
 
@@ -291,6 +293,10 @@ def run_ours(args):
         res["sweep"] = run_sweep(M, dev)
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(li_host, x_host, sh, T)
+    if rank == 0 and world == 1 and args.all_configs:
+        del li, layer
+        torch.cuda.empty_cache()
+        res["all_configs"] = run_all_configs(M, dev)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -378,6 +384,80 @@ def run_sweep(M, dev):
                     "hbm_roofline_us": round(nb / (peaks["hbm_gbs"] * 1e9) * 1e6, 2),
                     "hbm_frac": round(nb / (best / 1e6) / (peaks["hbm_gbs"] * 1e9), 4)})
     return out
+
+
+def time_layer(M, layer, x, n):
+    """(stream-launched us, CUDA-graph-replayed us) per layer call."""
+    o = layer.forward(x)
+    for _ in range(10):
+        layer.forward(x, o)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(n):
+        layer.forward(x, o)
+    e.record()
+    torch.cuda.synchronize()
+    us_stream = s.elapsed_time(e) / n * 1e3
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        layer.forward(x, o, stream=st)
+        st.synchronize()
+        with torch.cuda.graph(g, stream=st):
+            layer.forward(x, o, stream=st)
+    for _ in range(10):
+        g.replay()
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(n):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    us_graph = s.elapsed_time(e) / n * 1e3
+    del g
+    return us_stream, us_graph
+
+
+def run_all_configs(M, dev):
+    """Every preset at every token count: time per layer and the fraction of the
+    layer roofline (the slower of flops at the measured sustained bf16 peak and
+    touched-weight bytes at the measured HBM bandwidth)."""
+    peaks = R.measured_peaks()
+    pf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
+    bw = peaks["hbm_gbs"] * 1e9
+    rows = []
+    for name in ("tiny", "olmoe", "v2lite", "qwen3_int4", "qwen3_int8", "v3"):
+        sh = moe_synth.PRESETS[name]
+        li = moe_synth.make_layer(sh).to(dev)
+        for T in sh.tokens:
+            x = moe_synth.make_x(sh, T).to(dev)
+            layer = M.MoELayer(li, T)
+            counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
+            layer.forward(x, counts=counts)
+            torch.cuda.synchronize()
+            cnt = counts.cpu().numpy()
+            cap = None
+            if sh.capacity_factor > 0:
+                import math
+                cap = math.ceil(float(np.float32(sh.capacity_factor)) * T * sh.k / sh.E)
+            kept = int(np.minimum(cnt, cap).sum()) if cap else int(cnt.sum())
+            touched = int((cnt > 0).sum())
+            n = 50 if T >= 4096 else 300
+            us_s, us_g = time_layer(M, layer, x, n)
+            fl, nb = R.layer_flops(sh, T, kept), R.layer_bytes(sh, T, touched)
+            t_roof = R.roofline_time(fl, nb, pf, bw)
+            best = min(us_s, us_g)
+            rows.append({"workload": workload_name(sh, T), "T": T, "touched": touched,
+                         "kept": kept, "us_stream": round(us_s, 1), "us_graph": round(us_g, 1),
+                         "tokens_per_s": round(T / (best / 1e6), 1),
+                         "roofline_us": round(t_roof * 1e6, 1),
+                         "bound": "tensor" if fl / pf > nb / bw else "hbm",
+                         "frac": round(t_roof * 1e6 / best, 4)})
+            del layer
+        del li
+        torch.cuda.empty_cache()
+    return rows
 
 
 def cpu_baseline(li_host, x_host, sh, T, n_tokens=512):
