@@ -145,10 +145,14 @@ struct TcConfig {
   // barriers + bookkeeping after the tiles
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * 2) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
-  // swapped epilogue: per-tile output row and scale of each token, one copy per warp
-  static constexpr uint32_t EPI_BYTES = kEpiWarps * 128 * 8;
+  // swapped epilogue: per-tile output row and scale of each token, one copy per warp;
+  // direct DOWN epilogue: a 32-row x 16-column FP32 staging tile per warp (rows
+  // padded to 20 floats) through which rows are stored transposed
+  static constexpr uint32_t EPI_BYTES =
+      (EPI == EPI_DOWN && DIRECT) ? kEpiWarps * 32 * 20 * 4 : kEpiWarps * 128 * 8;
   static constexpr uint32_t SMEM_BYTES =
-      1024 + STAGES * STAGE_BYTES + A_REGION + BAR_BYTES + PREFIX_BYTES + EPI_BYTES;
+      1024 + STAGES * STAGE_BYTES + A_REGION + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
   static_assert(!DIRECT || BN == 128, "direct tiles hold 128 tokens");
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 128-byte swizzle alignment");
@@ -314,7 +318,9 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
   int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
   int* prefix = reinterpret_cast<int*>(
       reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
-  int* epi_row = prefix + 2 * (kMaxGroups + 1);                          // [8 warps][128]
+  // epilogue scratch, 16-byte aligned (float4 staging in the direct DOWN epilogue)
+  int* epi_row = reinterpret_cast<int*>(
+      (reinterpret_cast<uintptr_t>(prefix + 2 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
   float* epi_scale = reinterpret_cast<float*>(epi_row + kEpiWarps * 128);  // [8 warps][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -561,13 +567,28 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
                                                   (size_t)r * P.ld_out + n);
             dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          } else if (r >= 0) {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) +
-                                                    (size_t)r * P.ld_out + n);
+          } else if (EPI != EPI_GATEUP) {
+            // Through a per-warp staging tile: each lane writes its row's 16 scaled values,
+            // then 4 lanes store one row's 64 contiguous bytes, 8 rows per instruction,
+            // so every store fills whole 32-byte sectors.
+            float* stg = reinterpret_cast<float*>(epi_row) + (warp - 2) * (32 * 20);
+            float4* srow = reinterpret_cast<float4*>(stg + lane * 20);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              dst[j] = make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
-                                   v0[4 * j + 3] * sc);
+              srow[j] = make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
+                                    v0[4 * j + 3] * sc);
+            __syncwarp();
+            const int qq = (lane & 3) * 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rr = (lane >> 2) + 8 * i;
+              const int rout = __shfl_sync(0xffffffffu, r, rr);
+              const float4 v = *reinterpret_cast<const float4*>(stg + rr * 20 + qq);
+              if (rout >= 0)
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) +
+                                           (size_t)rout * P.ld_out + n + qq) = v;
+            }
+            __syncwarp();
           }
         }
       } else {
