@@ -174,10 +174,16 @@ __global__ void __launch_bounds__(256) k_router_split(const TA* __restrict__ xn,
     float acc[TT];
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt) acc[tt] = 0.f;
-    for (int kk = 0; kk < kn; ++kk) {
-      float w = to_f32(wr[(size_t)(k0 + kk) * E + e]);
+    for (int kb = 0; kb < kn; kb += 16) {
+      float w[16];
 #pragma unroll
-      for (int tt = 0; tt < TT; ++tt) acc[tt] = fmaf(xs[tt * slice + kk], w, acc[tt]);
+      for (int u = 0; u < 16; ++u) w[u] = kb + u < kn ? to_f32(wr[(size_t)(k0 + kb + u) * E + e]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (kb + u >= kn) break;
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) acc[tt] = fmaf(xs[tt * slice + kb + u], w[u], acc[tt]);
+      }
     }
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt)
@@ -879,18 +885,27 @@ __global__ void __launch_bounds__(128) k_simt_ffn(SimtArgs a) {
       }
       __syncthreads();
       if (n < N) {
-        for (int kk = 0; kk < kn; ++kk) {
-          if (DOWN) {
-            const float w = W[(size_t)(k0 + kk) * N + n];
+        // 16 k-steps of weights are loaded before they are used, so that the
+        // loads overlap instead of each waiting on the memory system in turn
+        for (int kb = 0; kb < kn; kb += 16) {
+          float wa[16], wb[16];
 #pragma unroll
-            for (int r = 0; r < kSimtRB; ++r) acc0[r] = fmaf(xs[r][kk], w, acc0[r]);
-          } else {
-            const float wg = Wg[(size_t)(k0 + kk) * N + n];
-            const float wu = Wu[(size_t)(k0 + kk) * N + n];
+          for (int u = 0; u < 16; ++u) {
+            const bool in = kb + u < kn;
+            if (DOWN) {
+              wa[u] = in ? W[(size_t)(k0 + kb + u) * N + n] : 0.f;
+            } else {
+              wa[u] = in ? Wg[(size_t)(k0 + kb + u) * N + n] : 0.f;
+              wb[u] = in ? Wu[(size_t)(k0 + kb + u) * N + n] : 0.f;
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            if (kb + u >= kn) break;
 #pragma unroll
             for (int r = 0; r < kSimtRB; ++r) {
-              acc0[r] = fmaf(xs[r][kk], wg, acc0[r]);
-              acc1[r] = fmaf(xs[r][kk], wu, acc1[r]);
+              acc0[r] = fmaf(xs[r][kb + u], wa[u], acc0[r]);
+              if (!DOWN) acc1[r] = fmaf(xs[r][kb + u], wb[u], acc1[r]);
             }
           }
         }

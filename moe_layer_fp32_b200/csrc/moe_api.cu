@@ -340,7 +340,6 @@ moe_status run_router(const moe_config* c, const moe_weights* w, const void* xn,
     TcProblem& P = p.prob[0];
     if (!map_weights(&P.tmA, w->w_router, 1, c->d, c->E)) return MOE_ERR_CUDA;
     P.tmA2 = P.tmA;
-    if (!map_rows(&P.tmB, xn, c->T, c->d, 128)) return MOE_ERR_CUDA;
     P.offsets = nullptr;
     P.G = 1;
     P.uniform_rows = c->T;
@@ -354,7 +353,14 @@ moe_status run_router(const moe_config* c, const moe_weights* w, const void* xn,
     P.n_valid = c->E;
     p.n_prob = 1;
     p.err = err;
-    return launch_tc<EPI_ROUTER, 128>(p, st);
+    // narrower token tiles when 128-token tiles would leave most SMs idle
+    const int ftiles = (c->E + 127) / 128;
+    if ((c->T + 127) / 128 * ftiles >= num_sms()) {
+      if (!map_rows(&P.tmB, xn, c->T, c->d, 128)) return MOE_ERR_CUDA;
+      return launch_tc<EPI_ROUTER, 128>(p, st);
+    }
+    if (!map_rows(&P.tmB, xn, c->T, c->d, 32)) return MOE_ERR_CUDA;
+    return launch_tc<EPI_ROUTER, 32>(p, st);
   }
   if (vec_router(c)) {
     dim3 grid((c->T + kRouterTT - 1) / kRouterTT, ns);
