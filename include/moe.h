@@ -232,8 +232,10 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
 /* moe_layer_forward with per-step timing marks, for profiling: events[0] is
  * recorded on `stream` before the first kernel and events[i] right after step i
  * (i = 1 .. moe_layer_step_count(cfg); the steps are RMSNorm, router, route,
- * permute, [gather], gate/up GEMM, down GEMM, combine -- the gather only for
- * tensor-core experts).  `events` holds caller-created cudaEvent_t handles (as
+ * permute, [dequantise + gather], gate/up GEMM, down GEMM, combine -- that step
+ * exists for tensor-core experts; at prefill batch sizes it gathers the routed
+ * token rows (and dequantises int8/int4 experts), at decode sizes the gate/up
+ * GEMM gathers them itself and the step is empty).  `events` holds caller-created cudaEvent_t handles (as
  * void*); n_events must be at least moe_layer_step_count(cfg) + 1.  No
  * optional outputs. */
 moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* w,

@@ -124,6 +124,19 @@ MOE_DEV void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int c0, int
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
+// Rows r0..r3 of a 2-D tensor, columns [c0, c0 + box width), into four consecutive
+// box-sized rows at dst (tile::gather4; the tensor map's box is one row high).
+// With the 128-byte swizzle the rows land exactly as rows (dst - tile) / 128 of a
+// tiled load of the same width would, given a 1024-byte aligned tile.
+MOE_DEV void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int c0, int r0, int r1,
+                         int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
 MOE_DEV void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"

@@ -56,7 +56,8 @@ constexpr int kMaxGroups = 512;
 struct TcProblem {
   CUtensorMap tmA;            // weights [G][K][N] bf16 (dims n, k, g), box (64, 64, 1)
   CUtensorMap tmA2;           // second weight matrix (up) for GATEUP
-  CUtensorMap tmB;            // activations [R][K] bf16 (dims k, r), box (64, BN)
+  CUtensorMap tmB;            // activations [R][K] bf16 (dims k, r), box (64, BN); with
+                              // gather_rows: box (64, 1), rows fetched four at a time
   const int32_t* offsets;     // [G+1] segments (B rows and output rows), or nullptr
   int G;                      // groups
   int uniform_rows;           // rows per group when offsets == nullptr
@@ -67,6 +68,8 @@ struct TcProblem {
   void* out;                  // H (bf16) / Y / Ys / logits (fp32)
   size_t out_row_base;        // GATEUP / shared DOWN / ROUTER: row = base + seg + m
   int ld_out;                 // elements per output row
+  const int32_t* gather_rows; // routed GATEUP: B row of slot s = gather_rows[s] / gather_k
+  int gather_k;               //   (the token of the slot's assignment), or nullptr
   const int32_t* perm_assign; // routed DOWN: output row = perm_assign[slot]
   const float* gate;          // routed DOWN: scale
   int n_valid;                // features actually stored (n < n_valid)
@@ -81,13 +84,25 @@ struct TcParams {
   TcProblem prob[2];
   int n_prob;
   int32_t* err;
+  // Split-K for swapped tiles (nullptr: off).  When the output tiles fill at most
+  // half of the grid, each is split along K into S <= kMaxSplit parts.  Each part
+  // stores its FP32 accumulators to split_part, and the last part of an output tile
+  // to finish adds all S parts in split order and runs the epilogue.
+  // split_part: gridDim.x * NA * BN * 128 floats.  split_cnt: gridDim.x * 8 zeroed
+  // ints, left zeroed again.
+  float* split_part;
+  int32_t* split_cnt;
 };
+
+constexpr int kMaxSplit = 4;
 
 struct TileInfo {
   int prob, g, m0, rows, n0;
   int b_row;          // B row of the tile's first token
   size_t out_seg;     // output row of the tile's first token (non-routed-DOWN cases)
   int slot0;          // routed: slot of the tile's first token
+  int bt, ks;         // split-K: output tile and this work item's part of K
+  int kb0, kb1;       // k-blocks [kb0, kb1) of this work item
 };
 
 // Weight blocks (128 features x 64 k) per pipeline stage: gate and up for
@@ -198,6 +213,16 @@ MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int TN, i
   ti.out_seg = P.out_row_base + (size_t)seg_start + ti.m0;
 }
 
+// Work item t of an S-way split: output tile t / S, k-blocks of part t % S.
+MOE_DEV void decode_work(const TcParams& p, const int* prefix, int BN, int TN, int S, int t,
+                         TileInfo& ti) {
+  ti.bt = t / S;
+  ti.ks = t % S;
+  decode_tile(p, prefix, BN, TN, ti.bt, ti);
+  const int kbl = p.prob[ti.prob].K / 64;
+  ti.kb0 = ti.ks * kbl / S;
+  ti.kb1 = (ti.ks + 1) * kbl / S;
+}
 MOE_DEV int total_tiles(const TcParams& p, const int* prefix, int TN) {
   int tot = 0;
   for (int pi = 0; pi < p.n_prob; ++pi) {
@@ -368,51 +393,103 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   constexpr int TN = C::TILE_N;
-  const int total = total_tiles(p, prefix, TN);
+  const int out_tiles = total_tiles(p, prefix, TN);
+  // split-K is compiled into the narrow swapped expert tiles only
+  constexpr bool kCanSplit = !DIRECT && EPI != EPI_ROUTER && BN <= 32;
+  int S = 1;
+  if (kCanSplit && p.split_part != nullptr && out_tiles > 0) {
+    int kbmin = p.prob[0].K / 64;
+    if (p.n_prob > 1 && p.prob[1].K / 64 < kbmin) kbmin = p.prob[1].K / 64;
+    S = (int)gridDim.x / out_tiles;
+    if (S > kMaxSplit) S = kMaxSplit;
+    if (S > kbmin / 2) S = kbmin / 2;
+    if (S < 1) S = 1;
+  }
+  const int total = out_tiles * S;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
+    // Lane 0 waits for free stages, arms them and loads the weights.  Token rows: a
+    // tiled load by lane 0, or (gathered problems) one tile::gather4 of four rows
+    // per lane, lanes 0 .. BN/4-1, after lane 0 has armed the stage.  Without any
+    // gathered problem lane 0 runs alone.
+    const bool any_gather = p.prob[0].gather_rows != nullptr ||
+                            (p.n_prob > 1 && p.prob[1].gather_rows != nullptr);
+    // arm stage `stage` of tile ti, k-block kb, and request everything but gathered rows
+    auto issue_stage = [&](uint8_t* st, int stage, uint32_t phase, const TileInfo& ti,
+                           const TcProblem& P, int kb, bool gather) {
+      mbar_arrive_expect_tx(&full_bar[stage], C::TX_BYTES);
+      issued[stage] = (int)phase + 1;
+      // GATEUP: the up matrix at the same features; wide DOWN: features +128
+      const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
+      const int n2 = (EPI == EPI_GATEUP) ? ti.n0 : ti.n0 + 128;
+      if (WQ == WQ_BF16) {
+        tma_load_3d(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g);
+        tma_load_3d(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g);
+        if (NA == 2) {
+          tma_load_3d(st + C::A_BYTES, m2, &full_bar[stage], n2, kb * 64, ti.g);
+          tma_load_3d(st + C::A_BYTES + 8192, m2, &full_bar[stage], n2 + 64, kb * 64, ti.g);
+        }
+      } else {
+        // raw bytes: x is the byte column (two int4 values per byte)
+        uint8_t* raw = st + C::RAW_OFF;
+        uint8_t* scl = st + C::SCALE_OFF;
+        const int div = WQ == WQ_INT4 ? 2 : 1;
+        const void* s2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmS2 : (const void*)&P.tmS;
+        tma_load_3d(raw, &P.tmA, &full_bar[stage], ti.n0 / div, kb * 64, ti.g);
+        // int8: scales [G][N] (second coordinate g, third 0); int4: [G][K/128][N]
+        if (WQ == WQ_INT8) tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, ti.g, 0);
+        else tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, kb / 2, ti.g);
+        if (NA == 2) {
+          tma_load_3d(raw + C::RAW_BYTES, m2, &full_bar[stage], n2 / div, kb * 64, ti.g);
+          if (WQ == WQ_INT8) tma_load_3d(scl + 256, s2, &full_bar[stage], n2, ti.g, 0);
+          else tma_load_3d(scl + 256, s2, &full_bar[stage], n2, kb / 2, ti.g);
+        }
+      }
+      if (!gather) tma_load_2d(st + C::TOKEN_OFF, &P.tmB, &full_bar[stage], kb * 64, ti.b_row);
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    if (!any_gather) {
+      if (lane == 0) {
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+          TileInfo ti;
+          decode_work(p, prefix, BN, TN, S, tile, ti);
+          const TcProblem& P = p.prob[ti.prob];
+          for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag)) { ok = false; break; }
+            issue_stage(tiles + stage * C::STAGE_BYTES, stage, phase, ti, P, kb, false);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+    } else {
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
-        decode_tile(p, prefix, BN, TN, tile, ti);
+        decode_work(p, prefix, BN, TN, S, tile, ti);
         const TcProblem& P = p.prob[ti.prob];
-        const int kblocks = P.K / 64;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag)) { ok = false; break; }
-          uint8_t* st = tiles + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], C::TX_BYTES);
-          issued[stage] = (int)phase + 1;
-          // GATEUP: the up matrix at the same features; wide DOWN: features +128
-          const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
-          const int n2 = (EPI == EPI_GATEUP) ? ti.n0 : ti.n0 + 128;
-          if (WQ == WQ_BF16) {
-            tma_load_3d(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g);
-            tma_load_3d(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g);
-            if (NA == 2) {
-              tma_load_3d(st + C::A_BYTES, m2, &full_bar[stage], n2, kb * 64, ti.g);
-              tma_load_3d(st + C::A_BYTES + 8192, m2, &full_bar[stage], n2 + 64, kb * 64, ti.g);
-            }
-          } else {
-            // raw bytes: x is the byte column (two int4 values per byte)
-            uint8_t* raw = st + C::RAW_OFF;
-            uint8_t* scl = st + C::SCALE_OFF;
-            const int div = WQ == WQ_INT4 ? 2 : 1;
-            const void* s2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmS2 : (const void*)&P.tmS;
-            tma_load_3d(raw, &P.tmA, &full_bar[stage], ti.n0 / div, kb * 64, ti.g);
-            // int8: scales [G][N] (second coordinate g, third 0); int4: [G][K/128][N]
-            if (WQ == WQ_INT8) tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, ti.g, 0);
-            else tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, kb / 2, ti.g);
-            if (NA == 2) {
-              tma_load_3d(raw + C::RAW_BYTES, m2, &full_bar[stage], n2 / div, kb * 64, ti.g);
-              if (WQ == WQ_INT8) tma_load_3d(scl + 256, s2, &full_bar[stage], n2, ti.g, 0);
-              else tma_load_3d(scl + 256, s2, &full_bar[stage], n2, kb / 2, ti.g);
-            }
+        const bool gather = P.gather_rows != nullptr;
+        // this lane's four rows; rows past the segment repeat the tile's first row
+        // (their accumulators are never stored)
+        int rr[4] = {0, 0, 0, 0};
+        if (gather && lane < BN / 4) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int m = 4 * lane + j;
+            rr[j] = P.gather_rows[ti.slot0 + (m < ti.rows ? m : 0)] / P.gather_k;
           }
-          tma_load_2d(st + C::TOKEN_OFF, &P.tmB, &full_bar[stage], kb * 64, ti.b_row);
+        }
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          int okw = 1;
+          if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
+          uint8_t* st = tiles + stage * C::STAGE_BYTES;
+          if (lane == 0) issue_stage(st, stage, phase, ti, P, kb, gather);
+          __syncwarp();   // the stage is armed before any gathered row can land
+          if (gather && lane < BN / 4)
+            tma_gather4(st + C::TOKEN_OFF + lane * 512, &P.tmB, &full_bar[stage], kb * 64,
+                        rr[0], rr[1], rr[2], rr[3]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -430,12 +507,11 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
-        decode_tile(p, prefix, BN, TN, tile, ti);
-        const int kblocks = p.prob[ti.prob].K / 64;
+        decode_work(p, prefix, BN, TN, S, tile, ti);
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag)) { ok = false; break; }
           if (WQ != WQ_BF16 &&
               !mbar_wait(&deq_bar[aslot], aphase, p.err, abort_flag)) { ok = false; break; }
@@ -451,7 +527,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
             //    apart.  tokens: K-major SW128, 16 k = 32 B per step, 8-row groups 1 KB.
             const uint64_t xd = sw128_desc(b_addr + kk * 32, 16, 1024);
             const uint64_t wd = sw128_desc(a_addr + kk * 2048, 8192, 1024);
-            const uint32_t accum = (kb | kk) != 0;
+            const uint32_t accum = (kb != ti.kb0 || kk != 0);
             if (DIRECT) {
               tc_mma_f16(d_tmem, xd, wd, C::IDESC, accum);   // N = 128 * NA at once
             } else {
@@ -491,10 +567,8 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
-        decode_tile(p, prefix, BN, TN, tile, ti);
-        const TcProblem& P = p.prob[ti.prob];
-        const int kblocks = P.K / 64;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        decode_work(p, prefix, BN, TN, S, tile, ti);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag)) { ok = false; break; }
           if (!mbar_wait(&aempty_bar[aslot], aphase ^ 1, p.err, abort_flag)) { ok = false; break; }
           uint8_t* st = tiles + stage * C::STAGE_BYTES;
@@ -524,7 +598,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       TileInfo ti;
-      decode_tile(p, prefix, BN, TN, tile, ti);
+      decode_work(p, prefix, BN, TN, S, tile, ti);
       const TcProblem& P = p.prob[ti.prob];
       const uint32_t t_base = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
       if (DIRECT) {
@@ -614,14 +688,63 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
         tc_fence_after();
         const int n = ti.n0 + q * 32 + lane;
         const bool n_ok = n < P.n_valid;
+        // split-K: this work item's partial sums, feature-contiguous per column
+        // (column c*16+j of the gate block, BN + c*16+j of the up block)
+        constexpr size_t PART = (size_t)NA * BN * 128;
+        const int fo = q * 32 + lane;
+        bool finish = true;   // this work item stores the tile's outputs
+        if (kCanSplit && S > 1) {
+          float* part = p.split_part + (size_t)tile * PART;
 #pragma unroll 1
-        for (int c = half; c < BN / 16; c += 2) {
+          for (int c = half; c < BN / 16; c += 2) {
+            if (c * 16 >= ti.rows) break;
+            float v0[16];
+            tmem_ld16(t_base + c * 16, v0);
+            float v1[16];
+            if (NA == 2) tmem_ld16(t_base + BN + c * 16, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              part[(size_t)(c * 16 + j) * 128 + fo] = v0[j];
+              if (NA == 2) part[(size_t)(BN + c * 16 + j) * 128 + fo] = v1[j];
+            }
+          }
+          // Count this part of the warp's slice once its stores are visible; the
+          // last of the S parts adds them all in split order (the same sums
+          // whichever part finishes last) and stores the outputs.  Nothing waits.
+          __threadfence();
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) {
+            int32_t* cnt = p.split_cnt + ti.bt * kEpiWarps + (warp - 2);
+            last = atomicAdd(cnt, 1) == S - 1;
+            if (last) atomicExch(cnt, 0);   // zero again for the next launch
+          }
+          finish = __shfl_sync(0xffffffffu, last, 0) != 0;
+          if (finish) __threadfence();
+        }
+        const float* p0 = S > 1 ? p.split_part + (size_t)ti.bt * S * PART : nullptr;
+#pragma unroll 1
+        for (int c = half; c < BN / 16 && finish; c += 2) {
           if (c * 16 >= ti.rows) break;
-          float v0[16];
-          tmem_ld16(t_base + c * 16, v0);
-          float v1[16];
-          if (NA == 2) tmem_ld16(t_base + BN + c * 16, v1);
-          tmem_wait_ld();
+          float v0[16], v1[16];
+          if (!kCanSplit || S == 1) {
+            tmem_ld16(t_base + c * 16, v0);
+            if (NA == 2) tmem_ld16(t_base + BN + c * 16, v1);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              float a0 = 0.f, a1 = 0.f;
+              for (int ss = 0; ss < S; ++ss) {
+                const float* ps = p0 + (size_t)ss * PART;
+                a0 += __ldcg(ps + (size_t)(c * 16 + j) * 128 + fo);
+                if (NA == 2) a1 += __ldcg(ps + (size_t)(BN + c * 16 + j) * 128 + fo);
+              }
+              v0[j] = a0;
+              v1[j] = a1;
+            }
+          }
           if (EPI == EPI_GATEUP) {
             __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.out);
 #pragma unroll

@@ -1,8 +1,10 @@
 // CUDA-core kernels of the layer: RMSNorm (a1), the split-K router for small
 // batches (a2), softmax/top-k routing (a3), histogram + scan + permutation
-// (a4/a5), the row gather that feeds the grouped GEMM, the combine (a8), and the
-// FP32 grouped SwiGLU FFN used when the expert weights are fp32.
+// (a4/a5), the one-pass dequantisation of int8/int4 experts, the row gather for
+// prefill tiles, the combine (a8), and the FP32 grouped SwiGLU FFN used when the
+// expert weights are fp32.
 #pragma once
+#include <type_traits>
 #include "common.cuh"
 
 namespace moe {
@@ -63,12 +65,17 @@ MOE_DEV int find_group(const int* prefix, int G, int mt) {
 MOE_DEV void store_act(__nv_bfloat16* p, double v) { *p = bf16_from_double(v); }
 MOE_DEV void store_act(float* p, double v) { *p = (float)v; }
 
+// Both RMSNorm kernels also zero `nzero` ints at `zero` (CTA 0): the split-K
+// counters of the expert GEMMs that follow later in the same layer.
 template <typename TA>
 __global__ void __launch_bounds__(256) k_rmsnorm(const TA* __restrict__ x,
                                                  const float* __restrict__ gamma,
-                                                 TA* __restrict__ xn, int d, double eps) {
+                                                 TA* __restrict__ xn, int d, double eps,
+                                                 int32_t* __restrict__ zero, int nzero) {
   pdl_wait();
   pdl_trigger();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
   __shared__ double red[8];
   const size_t row = (size_t)blockIdx.x * d;
   double s = 0.0;
@@ -102,9 +109,12 @@ template <int MAXV>
 __global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __restrict__ x,
                                                        const float* __restrict__ gamma,
                                                        __nv_bfloat16* __restrict__ xn, int d,
-                                                       double eps) {
+                                                       double eps, int32_t* __restrict__ zero,
+                                                       int nzero) {
   pdl_wait();
   pdl_trigger();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
   __shared__ double red[8];
   const int nv = d / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)blockIdx.x * d);
@@ -272,17 +282,34 @@ MOE_DEV bool key_better(float ka, int ea, float kb, int eb) {
   return ka > kb || (ka == kb && ea < eb);
 }
 
+// Routes token t with the calling warp.  The router partials of the ns K-slices
+// are added in slice order; their loads are issued 8 at a time so that they
+// overlap instead of each waiting for the previous add.
 template <int EPL>
-__global__ void __launch_bounds__(256) k_route(const float* __restrict__ part, int ns, int T,
-                                               int E, int k, const float* __restrict__ bias,
-                                               int mode, int renorm, int32_t* __restrict__ idx,
-                                               float* __restrict__ gate,
-                                               float* __restrict__ logits_out) {
-  pdl_wait();
-  pdl_trigger();
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
+MOE_DEV void route_token(const float* part, int ns, int T, int E, int k, const float* bias,
+                         int mode, int renorm, int32_t* idx, float* gate, float* logits_out,
+                         int t, int lane) {
+  // logits: the ns slice partials of this lane's experts, loaded SU slices at a time
+  // for all of them together, each added in slice order
+  constexpr int SU = EPL <= 4 ? 4 : EPL <= 8 ? 2 : 1;
+  float lg[EPL];
+  const size_t sstride = (size_t)T * E;
+  const float* pt = part + (size_t)t * E + lane;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) lg[i] = 0.f;
+  for (int s0 = 0; s0 < ns; s0 += SU) {
+    float v[EPL][SU];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+#pragma unroll
+      for (int u = 0; u < SU; ++u)
+        v[i][u] = (lane + 32 * i < E && s0 + u < ns) ? pt[(size_t)(s0 + u) * sstride + 32 * i] : 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+#pragma unroll
+      for (int u = 0; u < SU; ++u)
+        if (s0 + u < ns) lg[i] += v[i][u];
+  }
   float key[EPL], pin[EPL];
   float mx = -INFINITY;
 #pragma unroll
@@ -291,8 +318,7 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ part, i
     key[i] = -INFINITY;
     pin[i] = -INFINITY;
     if (e < E) {
-      float l = 0.f;
-      for (int s = 0; s < ns; ++s) l += part[((size_t)s * T + t) * E + e];
+      const float l = lg[i];
       if (logits_out) logits_out[(size_t)t * E + e] = l;
       float b = (mode != 0 && bias) ? bias[e] : 0.f;
       float sk = (mode != 0) ? l + b : l;
@@ -350,6 +376,20 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ part, i
   }
 }
 
+template <int EPL>
+__global__ void __launch_bounds__(256) k_route(const float* __restrict__ part, int ns, int T,
+                                               int E, int k, const float* __restrict__ bias,
+                                               int mode, int renorm, int32_t* __restrict__ idx,
+                                               float* __restrict__ gate,
+                                               float* __restrict__ logits_out) {
+  pdl_wait();
+  pdl_trigger();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  route_token<EPL>(part, ns, T, E, k, bias, mode, renorm, idx, gate, logits_out, t,
+                   threadIdx.x & 31);
+}
+
 // ---------------------------------------------------------------------------
 // a4 + a5: histogram, scan, capacity and stable permutation in one CTA of
 // 1024 threads.  Warp w owns a contiguous chunk of the flat assignments; no
@@ -358,15 +398,11 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ part, i
 // experts of kept = min(count, cap) gives the offsets; pass 2 assigns
 // rank = base + running count + lanes before it with the same expert.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ idx, int n, int E,
-                                                  int cap, int32_t* __restrict__ counts,
-                                                  int32_t* __restrict__ offsets,
-                                                  int32_t* __restrict__ perm_assign,
-                                                  int32_t* __restrict__ slot_of,
-                                                  int32_t* __restrict__ n_dropped,
-                                                  int32_t* err) {
-  pdl_wait();
-  pdl_trigger();
+// idx may have been written earlier in the same kernel (by other warps of this
+// CTA, before a __syncthreads), so it is read through the coherent path.
+MOE_DEV void permute_cta(const int32_t* idx, int n, int E, int cap, int32_t* counts,
+                         int32_t* offsets, int32_t* perm_assign, int32_t* slot_of,
+                         int32_t* n_dropped, int32_t* err) {
   extern __shared__ int sm[];
   int* cnt = sm;               // [32][E]
   int* s_off = sm + 32 * E;    // [E]
@@ -453,6 +489,36 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
       }
     }
   }
+}
+
+__global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ idx, int n, int E,
+                                                  int cap, int32_t* __restrict__ counts,
+                                                  int32_t* __restrict__ offsets,
+                                                  int32_t* __restrict__ perm_assign,
+                                                  int32_t* __restrict__ slot_of,
+                                                  int32_t* __restrict__ n_dropped,
+                                                  int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
+  permute_cta(idx, n, E, cap, counts, offsets, perm_assign, slot_of, n_dropped, err);
+}
+
+// a3 + a4 + a5 in one CTA for small batches: the 32 warps route the tokens, then
+// the same CTA builds the permutation from the routes it just wrote.
+template <int EPL>
+__global__ void __launch_bounds__(1024) k_route_permute(
+    const float* __restrict__ part, int ns, int T, int E, int k, const float* __restrict__ bias,
+    int mode, int renorm, int32_t* idx, float* __restrict__ gate, float* __restrict__ logits_out,
+    int cap, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_assign, int32_t* __restrict__ slot_of,
+    int32_t* __restrict__ n_dropped, int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < T; t += 32)
+    route_token<EPL>(part, ns, T, E, k, bias, mode, renorm, idx, gate, logits_out, t, lane);
+  __syncthreads();
+  permute_cta(idx, T * k, E, cap, counts, offsets, perm_assign, slot_of, n_dropped, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -722,8 +788,9 @@ __global__ void __launch_bounds__(256) k_dequant_experts(const __grid_constant__
 }
 
 // ---------------------------------------------------------------------------
-// gather: xp[s] = xn[perm_assign[s] / k] for s < offsets[E]; one warp per row,
-// 16-byte vectors (d * sizeof(TA) is a multiple of 16).
+// gather for wide (prefill) token tiles: xp[s] = xn[perm_assign[s] / k] for
+// s < offsets[E]; one warp per row, 16-byte vectors (d * sizeof(TA) is a multiple
+// of 16).  Narrow tiles gather inside the GEMM instead.
 // ---------------------------------------------------------------------------
 template <typename TA>
 __global__ void __launch_bounds__(256) k_gather_rows(const TA* __restrict__ xn,
@@ -821,19 +888,37 @@ struct SimtArgs {
   int T, d, f, k, E, S;
 };
 
-constexpr int kSimtRB = 8;
-constexpr int kSimtKC = 256;
+constexpr int kSimtRB = 8;     // rows (token slots) per tile
+constexpr int kSimtKC = 256;   // k-rows of x staged in shared memory at a time
+constexpr int kSimtWarps = 8;  // warps per CTA, each taking every 8th k-row
+constexpr int kSimtBatch = 8;  // k-rows of weights loaded before they are used
+static_assert(kSimtRB == kSimtWarps, "warp w finishes row w of the tile");
 
-template <bool DOWN>
-__global__ void __launch_bounds__(128) k_simt_ffn(SimtArgs a) {
+MOE_DEV float silu_f32(float u) { return u / (1.f + expf(-u)); }
+
+// Tile of kSimtRB rows x (32 * VEC) columns.  Each warp accumulates the rows'
+// products over its share of K (k-rows w, w + 8, ...), a lane holding VEC
+// adjacent columns loaded as one vector; the 8 warps' partial sums are then added
+// in warp order in shared memory, so the result does not depend on timing.
+// Dynamic shared memory: kSimtWarps * kSimtRB * 32 * VEC * (DOWN ? 1 : 2) floats
+// (this also holds the staged x rows, kSimtRB * kSimtKC floats).
+template <bool DOWN, int VEC>
+__global__ void __launch_bounds__(256) k_simt_ffn(SimtArgs a) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int prefix[520];
-  __shared__ float xs[kSimtRB][kSimtKC];
+  constexpr int TW = 32 * VEC;
+  using VT = typename std::conditional<VEC == 4, float4, float>::type;
+  extern __shared__ float sm_f[];
+  float* xs = sm_f;     // [kSimtRB][kSimtKC] during the K loop
+  float* red = sm_f;    // [NM][kSimtWarps][kSimtRB][TW] afterwards
+  __shared__ int prefix[520];   // at most 512 groups + 1
   __shared__ int rows_src[kSimtRB];
+  __shared__ int rows_out[kSimtRB];
+  __shared__ float rows_scale[kSimtRB];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = DOWN ? a.d : a.f;
   const int K = DOWN ? a.f : a.d;
-  const int n_tiles = (N + 127) / 128;
+  const int n_tiles = (N + TW - 1) / TW;
   if (threadIdx.x < 32) group_tile_prefix(a.offsets, a.E, 0, kSimtRB, prefix);
   __syncthreads();
   const int routed_mt = prefix[a.E];
@@ -853,80 +938,116 @@ __global__ void __launch_bounds__(128) k_simt_ffn(SimtArgs a) {
       r0 = (m2 % shared_mt_per) * kSimtRB;
       rows = min(kSimtRB, a.T - r0);
     }
-    __syncthreads();
+    __syncthreads();   // the previous tile is done with rows_* and the buffer
     if (threadIdx.x < kSimtRB) {
-      int r = threadIdx.x, src = -1;
+      const int r = threadIdx.x;
+      int src = -1, dst = -1;
+      float sc = 1.f;
       if (r < rows) {
-        if (DOWN) src = shared ? a.T * a.k + g * a.T + r0 + r : r0 + r;     // row of h
-        else src = shared ? r0 + r : a.perm_assign[r0 + r] / a.k;          // row of xn
+        if (DOWN) {
+          src = shared ? a.T * a.k + g * a.T + r0 + r : r0 + r;        // row of h
+          if (shared) {
+            dst = g * a.T + r0 + r;                                     // row of ys
+          } else {
+            dst = a.perm_assign[r0 + r];                                // row of y
+            sc = a.gate[dst];
+          }
+        } else {
+          src = shared ? r0 + r : a.perm_assign[r0 + r] / a.k;          // row of xn
+          dst = shared ? a.T * a.k + g * a.T + r0 + r : r0 + r;         // row of h
+        }
       }
       rows_src[r] = src;
+      rows_out[r] = dst;
+      rows_scale[r] = sc;
     }
-    const float* W;
-    if (DOWN) W = shared ? a.swd + (size_t)g * a.f * a.d : a.wd + (size_t)g * a.f * a.d;
-    else W = nullptr;
-    const float* Wg = shared ? a.swg + (size_t)g * a.d * a.f : a.wg + (size_t)g * a.d * a.f;
-    const float* Wu = shared ? a.swu + (size_t)g * a.d * a.f : a.wu + (size_t)g * a.d * a.f;
-    const int n = nt * 128 + threadIdx.x;
-    float acc0[kSimtRB], acc1[kSimtRB];
+    const float* W0;
+    const float* W1 = nullptr;
+    if (DOWN) {
+      W0 = (shared ? a.swd : a.wd) + (size_t)g * a.f * a.d;
+    } else {
+      W0 = (shared ? a.swg : a.wg) + (size_t)g * a.d * a.f;
+      W1 = (shared ? a.swu : a.wu) + (size_t)g * a.d * a.f;
+    }
+    const int n = nt * TW + lane * VEC;
+    const bool n_ok = n < N;   // N % VEC == 0, so the whole vector is in range
+    float acc0[kSimtRB][VEC], acc1[kSimtRB][VEC];
 #pragma unroll
-    for (int r = 0; r < kSimtRB; ++r) { acc0[r] = 0.f; acc1[r] = 0.f; }
+    for (int r = 0; r < kSimtRB; ++r)
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) { acc0[r][v] = 0.f; acc1[r][v] = 0.f; }
     for (int k0 = 0; k0 < K; k0 += kSimtKC) {
       const int kn = min(kSimtKC, K - k0);
       __syncthreads();
-      for (int i = threadIdx.x; i < kSimtRB * kSimtKC; i += 128) {
+#pragma unroll
+      for (int i0 = 0; i0 < kSimtRB * kSimtKC; i0 += 256) {
+        const int i = i0 + threadIdx.x;
         const int r = i / kSimtKC, kk = i % kSimtKC;
         float v = 0.f;
         if (rows_src[r] >= 0 && kk < kn) {
           const float* src = DOWN ? a.h + (size_t)rows_src[r] * a.f : a.xn + (size_t)rows_src[r] * a.d;
           v = src[k0 + kk];
         }
-        xs[r][kk] = v;
+        xs[i] = v;
       }
       __syncthreads();
-      if (n < N) {
-        // 16 k-steps of weights are loaded before they are used, so that the
-        // loads overlap instead of each waiting on the memory system in turn
-        for (int kb = 0; kb < kn; kb += 16) {
-          float wa[16], wb[16];
+      if (n_ok) {
+        for (int kb = warp; kb < kn; kb += kSimtWarps * kSimtBatch) {
+          VT wa[kSimtBatch], wb[kSimtBatch];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const bool in = kb + u < kn;
-            if (DOWN) {
-              wa[u] = in ? W[(size_t)(k0 + kb + u) * N + n] : 0.f;
-            } else {
-              wa[u] = in ? Wg[(size_t)(k0 + kb + u) * N + n] : 0.f;
-              wb[u] = in ? Wu[(size_t)(k0 + kb + u) * N + n] : 0.f;
+          for (int u = 0; u < kSimtBatch; ++u) {
+            const int kk = kb + u * kSimtWarps;
+            const size_t off = (size_t)(k0 + kk) * N + n;
+            if (kk < kn) {
+              wa[u] = *reinterpret_cast<const VT*>(W0 + off);
+              if (!DOWN) wb[u] = *reinterpret_cast<const VT*>(W1 + off);
             }
           }
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            if (kb + u >= kn) break;
+          for (int u = 0; u < kSimtBatch; ++u) {
+            const int kk = kb + u * kSimtWarps;
+            if (kk >= kn) break;
+            const float* fa = reinterpret_cast<const float*>(&wa[u]);
+            const float* fb = reinterpret_cast<const float*>(&wb[u]);
 #pragma unroll
             for (int r = 0; r < kSimtRB; ++r) {
-              acc0[r] = fmaf(xs[r][kb + u], wa[u], acc0[r]);
-              if (!DOWN) acc1[r] = fmaf(xs[r][kb + u], wb[u], acc1[r]);
+              const float x = xs[r * kSimtKC + kk];
+#pragma unroll
+              for (int v = 0; v < VEC; ++v) {
+                acc0[r][v] = fmaf(x, fa[v], acc0[r][v]);
+                if (!DOWN) acc1[r][v] = fmaf(x, fb[v], acc1[r][v]);
+              }
             }
           }
         }
       }
     }
-    if (n < N) {
-      for (int r = 0; r < rows; ++r) {
-        if (DOWN) {
-          if (shared) {
-            a.ys[((size_t)g * a.T + r0 + r) * a.d + n] = acc0[r];
-          } else {
-            const int as = a.perm_assign[r0 + r];
-            a.y[(size_t)as * a.d + n] = a.gate[as] * acc0[r];
-          }
-        } else {
-          const float u = acc0[r];
-          const float hv = (u / (1.f + expf(-u))) * acc1[r];
-          const size_t hrow = shared ? (size_t)a.T * a.k + (size_t)g * a.T + r0 + r : (size_t)(r0 + r);
-          a.h[hrow * a.f + n] = hv;
-        }
+    __syncthreads();   // the staged rows are no longer read: reuse the buffer
+#pragma unroll
+    for (int r = 0; r < kSimtRB; ++r)
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) {
+        red[((0 * kSimtWarps + warp) * kSimtRB + r) * TW + lane * VEC + v] = acc0[r][v];
+        if (!DOWN) red[((1 * kSimtWarps + warp) * kSimtRB + r) * TW + lane * VEC + v] = acc1[r][v];
       }
+    __syncthreads();
+    // thread (warp w, lane l) finishes row w, columns l*VEC .. l*VEC+VEC-1
+    const int r = warp;
+    if (r < rows && n_ok) {
+      float o[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSimtWarps; ++w) {
+          s0 += red[((0 * kSimtWarps + w) * kSimtRB + r) * TW + lane * VEC + v];
+          if (!DOWN) s1 += red[((1 * kSimtWarps + w) * kSimtRB + r) * TW + lane * VEC + v];
+        }
+        o[v] = DOWN ? s0 * rows_scale[r] : silu_f32(s0) * s1;
+      }
+      float* dst = DOWN ? (shared ? a.ys : a.y) + (size_t)rows_out[r] * a.d + n
+                        : a.h + (size_t)rows_out[r] * a.f + n;
+      *reinterpret_cast<VT*>(dst) = *reinterpret_cast<const VT*>(o);
     }
   }
 }

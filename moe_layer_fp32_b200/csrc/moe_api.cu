@@ -36,7 +36,9 @@ inline bool vec_router(const moe_config* c) {
 inline int router_splits(const moe_config* c) {
   if (tc_router(c)) return 1;
   if (vec_router(c)) return (c->d + kRouterSlice - 1) / kRouterSlice;
-  int ns = (c->d + kRouterSlice - 1) / kRouterSlice;
+  // K-slices of at least 16 rows: small batches get enough CTAs in flight that the
+  // weight loads of the many short slices overlap
+  int ns = (c->d + 15) / 16;
   int ttiles = (c->T + kRouterTT - 1) / kRouterTT;
   // enough CTAs to cover the SMs a couple of times, no more slices than needed
   int want = (296 + ttiles - 1) / ttiles;
@@ -58,12 +60,31 @@ int pick_bn(const moe_config* c) {
 // Quantised experts at prefill tile widths are dequantised once to bf16 in the
 // workspace (the in-loop dequantisation would repeat for every token tile of an
 // expert); decode tiles dequantise inside the GEMM main loop.
+// Token tiles up to this width gather their rows inside the gate/up GEMM
+// (tile::gather4, four rows per copy: a few copies per stage, hidden behind the
+// weight stream); wider tiles would be bound by the copy rate, so their rows are
+// gathered once by a kernel into xp and loaded as whole tiles.
+constexpr int kGather4MaxBN = 32;
+constexpr bool kGather4Int = false;   // int8 / int4 stages hold 4x fewer weight bytes
+inline bool gather_in_gemm(const moe_config* c) {
+  return pick_bn(c) <= kGather4MaxBN && (kGather4Int || c->expert_dtype == MOE_BF16);
+}
+int num_sms();
+// Split-K of narrow (decode) tiles when the expert tiles fill at most half the SMs;
+// the GEMM decides per launch from the actual tile count.
+constexpr bool kSplitBf16 = false;   // int experts only: bf16 tiles stream faster whole
+inline bool split_k(const moe_config* c) {
+  return tc_experts(c) && pick_bn(c) <= kGather4MaxBN &&
+         (kSplitBf16 || c->expert_dtype != MOE_BF16);
+}
+inline int split_counters() { return num_sms() * 8; }
 inline bool dequant_once(const moe_config* c) {
   return (c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4) && pick_bn(c) == 128;
 }
 
 struct Layout {
-  size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, h, y, ys, deq,
+  size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, split,
+      splitcnt, h, y, ys, deq,
       total;
   int ns;
 };
@@ -118,7 +139,9 @@ Layout layout(const moe_config* c) {
   L.slot = o;     o = align_up(o + T * k * 4);
   L.dropped = o;  o = align_up(o + 16);
   L.blk = o;      o = align_up(o + (size_t)E * ((T * k + kPermChunk - 1) / kPermChunk) * 4);
-  L.xp = o;       o = align_up(o + (tc_experts(c) ? T * k * d * act : 0));
+  L.xp = o;       o = align_up(o + (tc_experts(c) && !gather_in_gemm(c) ? T * k * d * act : 0));
+  L.split = o;    o = align_up(o + (split_k(c) ? (size_t)num_sms() * 2 * pick_bn(c) * 128 * 4 : 0));
+  L.splitcnt = o; o = align_up(o + (split_k(c) ? (size_t)split_counters() * 4 : 0));
   L.h = o;        o = align_up(o + (T * k + S * T) * f * hb);
   L.y = o;        o = align_up(o + T * k * d * 4);
   L.ys = o;       o = align_up(o + S * T * d * 4);
@@ -308,7 +331,7 @@ int capacity_rows(const moe_config* c) {
 
 // ----------------------------------------------------------------- the steps
 moe_status run_rmsnorm(const moe_config* c, const moe_weights* w, const void* x, void* xn,
-                       cudaStream_t st) {
+                       cudaStream_t st, int32_t* zero = nullptr, int nzero = 0) {
   if (c->act_dtype == MOE_BF16 && c->d <= 256 * 8 * 4 &&
       reinterpret_cast<uintptr_t>(x) % 16 == 0 && reinterpret_cast<uintptr_t>(xn) % 16 == 0 &&
       reinterpret_cast<uintptr_t>(w->rms_gamma) % 16 == 0) {
@@ -317,19 +340,23 @@ moe_status run_rmsnorm(const moe_config* c, const moe_weights* w, const void* x,
     auto xb = static_cast<const __nv_bfloat16*>(x);
     auto g = static_cast<const float*>(w->rms_gamma);
     auto ob = static_cast<__nv_bfloat16*>(xn);
-    if (nv <= 256) MOE_LAUNCH((k_rmsnorm_bf16v<1>), c->T, 256, 0, st, xb, g, ob, c->d, eps);
-    else if (nv <= 512) MOE_LAUNCH((k_rmsnorm_bf16v<2>), c->T, 256, 0, st, xb, g, ob, c->d, eps);
-    else MOE_LAUNCH((k_rmsnorm_bf16v<4>), c->T, 256, 0, st, xb, g, ob, c->d, eps);
+    if (nv <= 256)
+      MOE_LAUNCH((k_rmsnorm_bf16v<1>), c->T, 256, 0, st, xb, g, ob, c->d, eps, zero, nzero);
+    else if (nv <= 512)
+      MOE_LAUNCH((k_rmsnorm_bf16v<2>), c->T, 256, 0, st, xb, g, ob, c->d, eps, zero, nzero);
+    else
+      MOE_LAUNCH((k_rmsnorm_bf16v<4>), c->T, 256, 0, st, xb, g, ob, c->d, eps, zero, nzero);
     return check_launch();
   }
   if (c->act_dtype == MOE_BF16)
     MOE_LAUNCH((k_rmsnorm<__nv_bfloat16>), c->T, 256, 0, st, 
         static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(w->rms_gamma),
-        static_cast<__nv_bfloat16*>(xn), c->d, (double)c->rms_eps);
+        static_cast<__nv_bfloat16*>(xn), c->d, (double)c->rms_eps, zero, nzero);
   else
     MOE_LAUNCH((k_rmsnorm<float>), c->T, 256, 0, st, static_cast<const float*>(x),
                                            static_cast<const float*>(w->rms_gamma),
-                                           static_cast<float*>(xn), c->d, (double)c->rms_eps);
+                                           static_cast<float*>(xn), c->d, (double)c->rms_eps,
+                                           zero, nzero);
   return check_launch();
 }
 
@@ -409,6 +436,39 @@ inline int perm_blocks(const moe_config* c) {
   return (c->T * c->k + kPermChunk - 1) / kPermChunk;
 }
 
+// routing and the one-CTA permutation share a launch up to this many tokens (one
+// token per warp of the 1024-thread CTA; beyond that the warps would route in turn)
+constexpr int kFusedRouteMaxT = 32;
+inline bool fused_route_permute(const moe_config* c) {
+  return c->T <= kFusedRouteMaxT && c->T * c->k <= kPermSingleMax;
+}
+
+moe_status run_route_permute(const moe_config* c, const float* part, int ns, const float* bias,
+                             int32_t* idx, float* gate, float* logits_out, int32_t* counts,
+                             int32_t* offsets, int32_t* perm, int32_t* slot, int32_t* dropped,
+                             int32_t* err, cudaStream_t st) {
+  const int mode = c->bias_mode;
+  if (mode != MOE_BIAS_NONE && !bias) return MOE_ERR_INVALID;
+  const size_t smem = (size_t)33 * c->E * 4;
+#define MOE_ROUTE_PERMUTE(EPL)                                                              \
+  do {                                                                                      \
+    if (cudaFuncSetAttribute(k_route_permute<EPL>,                                          \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=     \
+        cudaSuccess)                                                                        \
+      return MOE_ERR_CUDA;                                                                  \
+    MOE_LAUNCH((k_route_permute<EPL>), 1, 1024, smem, st, part, ns, c->T, c->E, c->k, bias, \
+               mode, c->renormalize ? 1 : 0, idx, gate, logits_out, capacity_rows(c),       \
+               counts, offsets, perm, slot, dropped, err);                                  \
+  } while (0)
+  if (c->E <= 32) MOE_ROUTE_PERMUTE(1);
+  else if (c->E <= 64) MOE_ROUTE_PERMUTE(2);
+  else if (c->E <= 128) MOE_ROUTE_PERMUTE(4);
+  else if (c->E <= 256) MOE_ROUTE_PERMUTE(8);
+  else MOE_ROUTE_PERMUTE(16);
+#undef MOE_ROUTE_PERMUTE
+  return check_launch();
+}
+
 moe_status run_permute(const moe_config* c, const int32_t* idx, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* slot, int32_t* dropped,
                        int32_t* err, int32_t* blk, cudaStream_t st) {
@@ -435,9 +495,22 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int32_t* counts,
   return check_launch();
 }
 
+template <bool DOWN, int VEC>
+moe_status launch_simt(const SimtArgs& a, int grid, cudaStream_t st) {
+  const size_t red = (size_t)(DOWN ? 1 : 2) * kSimtWarps * kSimtRB * 32 * VEC * 4;
+  const size_t stage = (size_t)kSimtRB * kSimtKC * 4;
+  const size_t smem = red > stage ? red : stage;
+  if (cudaFuncSetAttribute(k_simt_ffn<DOWN, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  MOE_LAUNCH((k_simt_ffn<DOWN, VEC>), grid, 256, smem, st, a);
+  return check_launch();
+}
+
 moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
                    const int32_t* offsets, const int32_t* perm, const float* gate, float* y,
-                   float* ys, void* ws, cudaStream_t st, Marks* mk = nullptr) {
+                   float* ys, void* ws, cudaStream_t st, Marks* mk = nullptr,
+                   bool counters_zeroed = false) {
   Marks none;
   if (!mk) mk = &none;
   const Layout L = layout(c);
@@ -465,19 +538,21 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     a.y = y;
     a.ys = ys;
     a.T = T; a.d = c->d; a.f = c->f; a.k = k; a.E = c->E; a.S = S;
+    // float4 columns where the rows and every matrix base allow 16-byte vectors
+    auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    const bool v4_gu = c->f % 4 == 0 && a16(a.wg) && a16(a.wu) && a16(a.h) &&
+                       (S == 0 || (a16(a.swg) && a16(a.swu)));
+    const bool v4_dn = c->d % 4 == 0 && a16(a.wd) && a16(a.y) && (S == 0 || (a16(a.swd) && a16(a.ys)));
     const int grid = 2 * num_sms();
-    MOE_LAUNCH((k_simt_ffn<false>), grid, 128, 0, st, a);
-    moe_status s = check_launch();
+    moe_status s = v4_gu ? launch_simt<false, 4>(a, grid, st) : launch_simt<false, 1>(a, grid, st);
     if (s != MOE_OK) return s;
     mk->mark(st);
-    MOE_LAUNCH((k_simt_ffn<true>), grid, 128, 0, st, a);
-    s = check_launch();
+    s = v4_dn ? launch_simt<true, 4>(a, grid, st) : launch_simt<true, 1>(a, grid, st);
     mk->mark(st);
     return s;
   }
-  // tensor-core experts: [dequantise once], gather the routed rows, then gate/up and
-  // down on the tensor cores
-  __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  // tensor-core experts: [dequantise once], [gather the routed rows into xp], then
+  // gate/up and down on the tensor cores
   __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
   const int bn = pick_bn(c);
   const int R = T * k;
@@ -514,16 +589,32 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     wl.sh_gate = dst[3]; wl.sh_up = dst[4]; wl.sh_down = dst[5];
     wq = WQ_BF16;
   }
-  MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 2 * num_sms(), 256, 0, st,
-             static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
-  if ((s = check_launch()) != MOE_OK) return s;
-  mk->mark(st);
+  const bool g4 = gather_in_gemm(c);
+  float* split_part = split_k(c) ? at<float>(ws, L.split) : nullptr;
+  int32_t* split_cnt = split_k(c) ? at<int32_t>(ws, L.splitcnt) : nullptr;
+  if (split_cnt && !counters_zeroed &&
+      cudaMemsetAsync(split_cnt, 0, (size_t)split_counters() * 4, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
+  if (!g4) {
+    MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 2 * num_sms(), 256, 0, st,
+               static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
+    if ((s = check_launch()) != MOE_OK) return s;
+  }
+  mk->mark(st);   // end of the (optional) dequantisation and gather step
   {
     TcParams p{};
     TcProblem& P = p.prob[0];
     if (!map_expert(&P.tmA, wq, wl.w_gate, c->E, c->d, c->f)) return MOE_ERR_CUDA;
     if (!map_expert(&P.tmA2, wq, wl.w_up, c->E, c->d, c->f)) return MOE_ERR_CUDA;
-    if (!map_rows(&P.tmB, xp, R, c->d, bn)) return MOE_ERR_CUDA;
+    if (g4) {
+      // routed rows: slot s reads token perm[s] / k of xn, four rows per copy
+      if (!map_rows(&P.tmB, xn, T, c->d, 1)) return MOE_ERR_CUDA;
+      P.gather_rows = perm;
+      P.gather_k = k;
+    } else if (!map_rows(&P.tmB, xp, R, c->d, bn)) {
+      return MOE_ERR_CUDA;
+    }
     if (wq != WQ_BF16 && (!map_scales(&P.tmS, c, w->s_gate, c->E, c->d, c->f) ||
                           !map_scales(&P.tmS2, c, w->s_up, c->E, c->d, c->f)))
       return MOE_ERR_CUDA;
@@ -558,6 +649,8 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
       p.n_prob = 2;
     }
     p.err = err;
+    p.split_part = split_part;
+    p.split_cnt = split_cnt;
     s = launch_tc_bn<EPI_GATEUP>(bn, wq, p, st);
     if (s != MOE_OK) return s;
     mk->mark(st);
@@ -608,6 +701,8 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
       p.n_prob = 2;
     }
     p.err = err;
+    p.split_part = split_part;
+    p.split_cnt = split_cnt;
     s = launch_tc_bn<EPI_DOWN>(bn, wq, p, st);
     mk->mark(st);
   }
@@ -655,19 +750,32 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
   float* y = at<float>(ws, L.y);
   float* ys = cfg->n_shared ? at<float>(ws, L.ys) : nullptr;
   mk->mark(st);
-  if ((s = run_rmsnorm(cfg, w, x, xn, st)) != MOE_OK) return s;
+  int32_t* split_cnt = split_k(cfg) ? at<int32_t>(ws, L.splitcnt) : nullptr;
+  if ((s = run_rmsnorm(cfg, w, x, xn, st, split_cnt, split_cnt ? split_counters() : 0)) !=
+      MOE_OK)
+    return s;
   mk->mark(st);
   if ((s = run_router(cfg, w, xn, part, L.ns, err, st)) != MOE_OK) return s;
   mk->mark(st);
-  if ((s = run_route(cfg, part, L.ns, static_cast<const float*>(w->router_bias), idx, gate,
-                     logits_out, st)) != MOE_OK)
-    return s;
+  if (fused_route_permute(cfg)) {
+    // one launch; the permutation step has no time of its own in the profile
+    if ((s = run_route_permute(cfg, part, L.ns, static_cast<const float*>(w->router_bias), idx,
+                               gate, logits_out, counts, offsets, perm, slot,
+                               at<int32_t>(ws, L.dropped), err, st)) != MOE_OK)
+      return s;
+    mk->mark(st);
+  } else {
+    if ((s = run_route(cfg, part, L.ns, static_cast<const float*>(w->router_bias), idx, gate,
+                       logits_out, st)) != MOE_OK)
+      return s;
+    mk->mark(st);
+    if ((s = run_permute(cfg, idx, counts, offsets, perm, slot, at<int32_t>(ws, L.dropped), err,
+                         at<int32_t>(ws, L.blk), st)) != MOE_OK)
+      return s;
+  }
   mk->mark(st);
-  if ((s = run_permute(cfg, idx, counts, offsets, perm, slot, at<int32_t>(ws, L.dropped), err,
-                       at<int32_t>(ws, L.blk), st)) != MOE_OK)
+  if ((s = run_ffn(cfg, w, xn, offsets, perm, gate, y, ys, ws, st, mk, true)) != MOE_OK)
     return s;
-  mk->mark(st);
-  if ((s = run_ffn(cfg, w, xn, offsets, perm, gate, y, ys, ws, st, mk)) != MOE_OK) return s;
   s = run_combine(cfg, y, slot, ys, x, out, st);
   mk->mark(st);
   return s;
@@ -855,14 +963,19 @@ const char* moe_status_string(moe_status s) {
 
 int32_t moe_layer_step_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
-  // rmsnorm, router, route, permute, [gather], gate/up, down, combine
+  // rmsnorm, router, route, permute, [dequantise + gather], gate/up, down, combine
   return tc_experts(cfg) ? 8 : 7;
 }
 
 int32_t moe_layer_launch_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
-  const int perm = cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
-  return moe_layer_step_count(cfg) - 1 + perm + (dequant_once(cfg) ? 1 : 0);
+  // rmsnorm, router, route, gate/up, down and combine, plus the permutation (its
+  // own launch, three for large batches, or none when it shares the routing
+  // launch), and for tensor-core experts at wide tiles the row gather and (int8 /
+  // int4) the one-pass dequantisation
+  const int perm = fused_route_permute(cfg) ? 0 : cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
+  const int gather = tc_experts(cfg) && !gather_in_gemm(cfg) ? 1 : 0;
+  return 6 + perm + gather + (dequant_once(cfg) ? 1 : 0);
 }
 
 }  // extern "C"
