@@ -29,6 +29,10 @@
  *   - Every tensor pointer is DEVICE memory owned by the caller; shapes are
  *     row-major with the last index contiguous.  The library allocates nothing
  *     and keeps no global state.
+ *   - Alignment: tensors need only the alignment of their element type, except
+ *     that with tensor-core experts (bf16 / int8 / int4) xn, the expert weights
+ *     and their scales must be 16-byte aligned (TMA operands; MOE_ERR_INVALID
+ *     otherwise).  16-byte aligned tensors take vectorised kernels elsewhere.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls are asynchronous on that stream and never synchronise the host,
  *     except moe_get_device_status.

@@ -65,7 +65,8 @@ struct TcProblem {
   int b_group_stride;         //   b_row_base + g * b_group_stride
   int N;                      // output features
   int K;                      // reduction length (multiple of 64)
-  void* out;                  // H (bf16) / Y / Ys / logits (fp32)
+  void* out;                  // H (bf16) / Y / Ys / logits (fp32; Y bf16 with out_bf16)
+  int out_bf16;               // DOWN: store the gated rows in bf16
   size_t out_row_base;        // GATEUP / shared DOWN / ROUTER: row = base + seg + m
   int ld_out;                 // elements per output row
   const int32_t* gather_rows; // routed GATEUP: B row of slot s = gather_rows[s] / gather_k
@@ -643,8 +644,9 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           } else if (EPI != EPI_GATEUP) {
             // Through a per-warp staging tile: each lane writes its row's 16 scaled values,
-            // then 4 lanes store one row's 64 contiguous bytes, 8 rows per instruction,
-            // so every store fills whole 32-byte sectors.
+            // then several lanes store one row's contiguous bytes (FP32: 4 lanes x 16 B,
+            // 8 rows per instruction; bf16: 2 lanes x 16 B, 16 rows per instruction), so
+            // every store fills whole 32-byte sectors.
             float* stg = reinterpret_cast<float*>(epi_row) + (warp - 2) * (32 * 20);
             float4* srow = reinterpret_cast<float4*>(stg + lane * 20);
 #pragma unroll
@@ -652,15 +654,37 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
               srow[j] = make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
                                     v0[4 * j + 3] * sc);
             __syncwarp();
-            const int qq = (lane & 3) * 4;
+            if (P.out_bf16) {
+              const int hh = (lane & 1) * 8;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int rr = (lane >> 2) + 8 * i;
-              const int rout = __shfl_sync(0xffffffffu, r, rr);
-              const float4 v = *reinterpret_cast<const float4*>(stg + rr * 20 + qq);
-              if (rout >= 0)
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) +
-                                           (size_t)rout * P.ld_out + n + qq) = v;
+              for (int i = 0; i < 2; ++i) {
+                const int rr = (lane >> 1) + 16 * i;
+                const int rout = __shfl_sync(0xffffffffu, r, rr);
+                const float4 a = *reinterpret_cast<const float4*>(stg + rr * 20 + hh);
+                const float4 b = *reinterpret_cast<const float4*>(stg + rr * 20 + hh + 4);
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(a.z, a.w);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y);
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(b.z, b.w);
+                if (rout >= 0)
+                  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) +
+                                            (size_t)rout * P.ld_out + n + hh) =
+                      make_uint4(*reinterpret_cast<uint32_t*>(&h0),
+                                 *reinterpret_cast<uint32_t*>(&h1),
+                                 *reinterpret_cast<uint32_t*>(&h2),
+                                 *reinterpret_cast<uint32_t*>(&h3));
+              }
+            } else {
+              const int qq = (lane & 3) * 4;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int rr = (lane >> 2) + 8 * i;
+                const int rout = __shfl_sync(0xffffffffu, r, rr);
+                const float4 v = *reinterpret_cast<const float4*>(stg + rr * 20 + qq);
+                if (rout >= 0)
+                  *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) +
+                                             (size_t)rout * P.ld_out + n + qq) = v;
+              }
             }
             __syncwarp();
           }
@@ -752,6 +776,14 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
               const int r = s_row[c * 16 + j];
               if (r >= 0 && n_ok)
                 H[(size_t)r * P.ld_out + n] = __float2bfloat16_rn(silu_f(v0[j]) * v1[j]);
+            }
+          } else if (EPI == EPI_DOWN && P.out_bf16) {
+            __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(P.out);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int r = s_row[c * 16 + j];
+              if (r >= 0 && n_ok)
+                Y[(size_t)r * P.ld_out + n] = __float2bfloat16_rn(v0[j] * s_scale[c * 16 + j]);
             }
           } else {
             float* Y = reinterpret_cast<float*>(P.out);

@@ -811,62 +811,100 @@ __global__ void __launch_bounds__(256) k_gather_rows(const TA* __restrict__ xn,
 }
 
 // ---------------------------------------------------------------------------
-// a8: combine, 4 consecutive elements per thread.  out = residual + shared
-// experts (s ascending) + kept assignments (j ascending), FP32.
+// a8: combine, VEC consecutive elements per thread.  out = residual + shared
+// experts (s ascending) + kept assignments (j ascending), summed in FP32.  The
+// routed rows are FP32, or bf16 inside the layer forward (tensor-core experts),
+// widened before the sum.  VEC = 4 needs every tensor 16-byte aligned (d % 8 == 0
+// always holds); VEC = 1 takes any alignment.
 // ---------------------------------------------------------------------------
-MOE_DEV void load4(const float* p, float (&v)[4]) {
-  float4 q = *reinterpret_cast<const float4*>(p);
-  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+template <int VEC>
+MOE_DEV void loadv(const float* p, float (&v)[VEC]) {
+  if constexpr (VEC == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else {
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) v[u] = p[u];
+  }
 }
-MOE_DEV void load4(const __nv_bfloat16* p, float (&v)[4]) {
-  uint2 q = *reinterpret_cast<const uint2*>(p);
-  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&q.x);
-  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&q.y);
-  v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
+template <int VEC>
+MOE_DEV void loadv(const __nv_bfloat16* p, float (&v)[VEC]) {
+  if constexpr (VEC == 4) {
+    const uint2 q = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&q.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&q.y);
+    v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
+  } else {
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) v[u] = __bfloat162float(p[u]);
+  }
 }
-MOE_DEV void store4(float* p, const float (&v)[4]) {
-  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+template <int VEC>
+MOE_DEV void storev(float* p, const float (&v)[VEC]) {
+  if constexpr (VEC == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) p[u] = v[u];
+  }
 }
-MOE_DEV void store4(__nv_bfloat16* p, const float (&v)[4]) {
-  __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
-  __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
-  uint2 q;
-  q.x = *reinterpret_cast<uint32_t*>(&a);
-  q.y = *reinterpret_cast<uint32_t*>(&b);
-  *reinterpret_cast<uint2*>(p) = q;
+template <int VEC>
+MOE_DEV void storev(__nv_bfloat16* p, const float (&v)[VEC]) {
+  if constexpr (VEC == 4) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+  } else {
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) p[u] = __float2bfloat16_rn(v[u]);
+  }
 }
 
-template <typename TA, typename TO>
-__global__ void __launch_bounds__(256) k_combine(const float* __restrict__ y,
+template <typename TA, typename TO, typename TY, int VEC>
+__global__ void __launch_bounds__(256) k_combine(const TY* __restrict__ y,
                                                  const int32_t* __restrict__ slot_of,
                                                  const float* __restrict__ ys, int S,
                                                  const TA* __restrict__ res, TO* __restrict__ out,
                                                  int T, int d, int k) {
   pdl_wait();
   pdl_trigger();
-  const int q = d / 4;
+  // The rows of JB assignments are loaded together, unconditionally (a dropped
+  // slot's row is read but not added; past k the token's first row is re-read), so
+  // that their memory latencies overlap; the adds then follow in j order.
+  constexpr int JB = 8;
+  const int q = d / VEC;
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (size_t)T * q) return;
   const int t = (int)(i / q);
-  const int c = (int)(i % q) * 4;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (res) load4(res + (size_t)t * d + c, acc);
+  const int c = (int)(i % q) * VEC;
+  float acc[VEC];
+#pragma unroll
+  for (int u = 0; u < VEC; ++u) acc[u] = 0.f;
+  if (res) loadv<VEC>(res + (size_t)t * d + c, acc);
   for (int s = 0; s < S; ++s) {
-    float v[4];
-    load4(ys + ((size_t)s * T + t) * d + c, v);
+    float v[VEC];
+    loadv<VEC>(ys + ((size_t)s * T + t) * d + c, v);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] += v[u];
+    for (int u = 0; u < VEC; ++u) acc[u] += v[u];
   }
-  for (int j = 0; j < k; ++j) {
-    const size_t a = (size_t)t * k + j;
-    if (slot_of[a] >= 0) {
-      float v[4];
-      load4(y + a * d + c, v);
+  const size_t a0 = (size_t)t * k;
+  for (int j0 = 0; j0 < k; j0 += JB) {
+    int sl[JB];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] += v[u];
-    }
+    for (int jj = 0; jj < JB; ++jj) sl[jj] = j0 + jj < k ? slot_of[a0 + j0 + jj] : -1;
+    float v[JB][VEC];
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj)
+      loadv<VEC>(y + (a0 + (j0 + jj < k ? j0 + jj : 0)) * d + c, v[jj]);
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj)
+      if (sl[jj] >= 0) {
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) acc[u] += v[jj][u];
+      }
   }
-  store4(out + (size_t)t * d + c, acc);
+  storev<VEC>(out + (size_t)t * d + c, acc);
 }
 
 // ---------------------------------------------------------------------------

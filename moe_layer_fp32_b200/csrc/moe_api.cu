@@ -78,6 +78,10 @@ inline bool split_k(const moe_config* c) {
          (kSplitBf16 || c->expert_dtype != MOE_BF16);
 }
 inline int split_counters() { return num_sms() * 8; }
+// Inside the layer forward the gated routed rows of tensor-core experts are kept
+// in bf16 (half the bytes the down GEMM writes and the combine reads); the
+// grouped-FFN and combine entry points exchange them in FP32.
+inline bool y_bf16(const moe_config* c) { return tc_experts(c); }
 inline bool dequant_once(const moe_config* c) {
   return (c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4) && pick_bn(c) == 128;
 }
@@ -143,7 +147,7 @@ Layout layout(const moe_config* c) {
   L.split = o;    o = align_up(o + (split_k(c) ? (size_t)num_sms() * 2 * pick_bn(c) * 128 * 4 : 0));
   L.splitcnt = o; o = align_up(o + (split_k(c) ? (size_t)split_counters() * 4 : 0));
   L.h = o;        o = align_up(o + (T * k + S * T) * f * hb);
-  L.y = o;        o = align_up(o + T * k * d * 4);
+  L.y = o;        o = align_up(o + T * k * d * (y_bf16(c) ? 2 : 4));
   L.ys = o;       o = align_up(o + S * T * d * 4);
   L.deq = o;      o = align_up(o + (dequant_once(c) ? (E + S) * 3 * d * f * 2 : 0));
   L.total = o;
@@ -389,7 +393,9 @@ moe_status run_router(const moe_config* c, const moe_weights* w, const void* xn,
     if (!map_rows(&P.tmB, xn, c->T, c->d, 32)) return MOE_ERR_CUDA;
     return launch_tc<EPI_ROUTER, 32>(p, st);
   }
-  if (vec_router(c)) {
+  // the vectorised router loads 16-byte weight vectors; other alignments take the
+  // split kernel below with the same slices
+  if (vec_router(c) && (reinterpret_cast<uintptr_t>(w->w_router) & 15) == 0) {
     dim3 grid((c->T + kRouterTT - 1) / kRouterTT, ns);
     const size_t smem = ((size_t)kRouterTT * kRouterSlice + 256 * 8) * 4;
     MOE_LAUNCH((k_router_vec<kRouterTT>), grid, 256, smem, st,
@@ -508,9 +514,9 @@ moe_status launch_simt(const SimtArgs& a, int grid, cudaStream_t st) {
 }
 
 moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
-                   const int32_t* offsets, const int32_t* perm, const float* gate, float* y,
+                   const int32_t* offsets, const int32_t* perm, const float* gate, void* y,
                    float* ys, void* ws, cudaStream_t st, Marks* mk = nullptr,
-                   bool counters_zeroed = false) {
+                   bool counters_zeroed = false, bool rows_bf16 = false) {
   Marks none;
   if (!mk) mk = &none;
   const Layout L = layout(c);
@@ -535,7 +541,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     a.swu = static_cast<const float*>(w->sh_up);
     a.swd = static_cast<const float*>(w->sh_down);
     a.h = at<float>(ws, L.h);
-    a.y = y;
+    a.y = static_cast<float*>(y);
     a.ys = ys;
     a.T = T; a.d = c->d; a.f = c->f; a.k = k; a.E = c->E; a.S = S;
     // float4 columns where the rows and every matrix base allow 16-byte vectors
@@ -552,7 +558,16 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     return s;
   }
   // tensor-core experts: [dequantise once], [gather the routed rows into xp], then
-  // gate/up and down on the tensor cores
+  // gate/up and down on the tensor cores.  The TMA (and the vector loads of the
+  // gather and dequantisation kernels) need 16-byte aligned operands.
+  {
+    auto a16 = [](const void* q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    const void* ops[] = {xn, w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up, w->s_down,
+                         w->sh_gate, w->sh_up, w->sh_down, w->sh_s_gate, w->sh_s_up,
+                         w->sh_s_down};
+    for (const void* o : ops)
+      if (!a16(o)) return MOE_ERR_INVALID;
+  }
   __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
   const int bn = pick_bn(c);
   const int R = T * k;
@@ -670,6 +685,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     P.N = c->d;
     P.K = c->f;
     P.out = y;
+    P.out_bf16 = rows_bf16 ? 1 : 0;
     P.out_row_base = 0;
     P.ld_out = c->d;
     P.perm_assign = perm;
@@ -709,23 +725,45 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   return s;
 }
 
-moe_status run_combine(const moe_config* c, const float* y, const int32_t* slot,
-                       const float* ys, const void* res, void* out, cudaStream_t st) {
-  const size_t n = (size_t)c->T * (c->d / 4);
+template <int VEC>
+moe_status launch_combine(const moe_config* c, const void* y, bool rows_bf16,
+                          const int32_t* slot, const float* ys, const void* res, void* out,
+                          cudaStream_t st) {
+  const size_t n = (size_t)c->T * (c->d / VEC);
   const int blocks = (int)((n + 255) / 256);
-  if (c->act_dtype == MOE_BF16 && c->out_dtype == MOE_BF16)
-    MOE_LAUNCH((k_combine<__nv_bfloat16, __nv_bfloat16>), blocks, 256, 0, st, 
-        y, slot, ys, c->n_shared, static_cast<const __nv_bfloat16*>(res),
-        static_cast<__nv_bfloat16*>(out), c->T, c->d, c->k);
-  else if (c->act_dtype == MOE_BF16)
-    MOE_LAUNCH((k_combine<__nv_bfloat16, float>), blocks, 256, 0, st, 
-        y, slot, ys, c->n_shared, static_cast<const __nv_bfloat16*>(res),
-        static_cast<float*>(out), c->T, c->d, c->k);
-  else
-    MOE_LAUNCH((k_combine<float, float>), blocks, 256, 0, st, y, slot, ys, c->n_shared,
-                                                    static_cast<const float*>(res),
-                                                    static_cast<float*>(out), c->T, c->d, c->k);
+  using bf = __nv_bfloat16;
+  auto yf = static_cast<const float*>(y);
+  auto yb = static_cast<const bf*>(y);
+  auto rb = static_cast<const bf*>(res);
+  auto rf = static_cast<const float*>(res);
+  if (c->act_dtype == MOE_BF16 && c->out_dtype == MOE_BF16) {
+    if (rows_bf16)
+      MOE_LAUNCH((k_combine<bf, bf, bf, VEC>), blocks, 256, 0, st, yb, slot, ys, c->n_shared, rb,
+                 static_cast<bf*>(out), c->T, c->d, c->k);
+    else
+      MOE_LAUNCH((k_combine<bf, bf, float, VEC>), blocks, 256, 0, st, yf, slot, ys, c->n_shared,
+                 rb, static_cast<bf*>(out), c->T, c->d, c->k);
+  } else if (c->act_dtype == MOE_BF16) {
+    if (rows_bf16)
+      MOE_LAUNCH((k_combine<bf, float, bf, VEC>), blocks, 256, 0, st, yb, slot, ys, c->n_shared,
+                 rb, static_cast<float*>(out), c->T, c->d, c->k);
+    else
+      MOE_LAUNCH((k_combine<bf, float, float, VEC>), blocks, 256, 0, st, yf, slot, ys,
+                 c->n_shared, rb, static_cast<float*>(out), c->T, c->d, c->k);
+  } else {
+    if (rows_bf16) return MOE_ERR_UNSUPPORTED;
+    MOE_LAUNCH((k_combine<float, float, float, VEC>), blocks, 256, 0, st, yf, slot, ys,
+               c->n_shared, rf, static_cast<float*>(out), c->T, c->d, c->k);
+  }
   return check_launch();
+}
+
+moe_status run_combine(const moe_config* c, const void* y, bool rows_bf16, const int32_t* slot,
+                       const float* ys, const void* res, void* out, cudaStream_t st) {
+  auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  if (a16(y) && a16(ys) && a16(res) && a16(out))
+    return launch_combine<4>(c, y, rows_bf16, slot, ys, res, out, st);
+  return launch_combine<1>(c, y, rows_bf16, slot, ys, res, out, st);
 }
 
 moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const void* x,
@@ -747,7 +785,7 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm = at<int32_t>(ws, L.perm);
   int32_t* slot = at<int32_t>(ws, L.slot);
-  float* y = at<float>(ws, L.y);
+  void* y = at<void>(ws, L.y);
   float* ys = cfg->n_shared ? at<float>(ws, L.ys) : nullptr;
   mk->mark(st);
   int32_t* split_cnt = split_k(cfg) ? at<int32_t>(ws, L.splitcnt) : nullptr;
@@ -774,9 +812,10 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
       return s;
   }
   mk->mark(st);
-  if ((s = run_ffn(cfg, w, xn, offsets, perm, gate, y, ys, ws, st, mk, true)) != MOE_OK)
+  if ((s = run_ffn(cfg, w, xn, offsets, perm, gate, y, ys, ws, st, mk, true, y_bf16(cfg))) !=
+      MOE_OK)
     return s;
-  s = run_combine(cfg, y, slot, ys, x, out, st);
+  s = run_combine(cfg, y, y_bf16(cfg), slot, ys, x, out, st);
   mk->mark(st);
   return s;
 }
@@ -918,7 +957,7 @@ moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32
   moe_status s = validate(cfg);
   if (s != MOE_OK) return s;
   if (!y_assign || !slot_of || !out || (cfg->n_shared > 0 && !y_shared)) return MOE_ERR_INVALID;
-  return run_combine(cfg, y_assign, slot_of, y_shared, residual, out, S_(stream));
+  return run_combine(cfg, y_assign, false, slot_of, y_shared, residual, out, S_(stream));
 }
 
 moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const void* x,

@@ -1,5 +1,6 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
 same seeded inputs.  Every test here needs a B200."""
+import dataclasses
 import os
 
 import numpy as np
@@ -32,10 +33,14 @@ SMALL = {
                                capacity_factor=1.25, seed=17),
     "int8_prefill": LayerShape("int8_prefill", d=384, E=8, k=2, f=512, n_shared=1,
                                expert="int8", seed=18),
+    # FP32 experts with f not a multiple of 4 (scalar weight columns in gate/up)
+    "f32_odd_f": LayerShape("f32_odd_f", d=136, E=6, k=2, f=130, n_shared=1, act="f32",
+                            router="f32", expert="f32", capacity_factor=1.5,
+                            bias_mode="logit", seed=19),
 }
 SMALL_T = {"bf16_plain": 100, "bf16_shared_cap": 77, "bf16_select_tc_router": 200,
            "bf16_prefill_tiles": 1000, "f32_tiny": 64, "int4_decode": 20, "int8_decode": 50,
-           "int4_prefill": 900, "int8_prefill": 700}
+           "int4_prefill": 900, "int8_prefill": 700, "f32_odd_f": 37}
 
 
 @pytest.fixture(autouse=True)
@@ -240,7 +245,8 @@ def test_layer_routing_bitexact_given_gpu_logits():
 
 def test_layer_is_deterministic_and_replayable():
     """Two runs are bitwise identical, and the five-call chain fed the layer's own
-    routes reproduces the fused call bitwise (route replay control, picx.dev
+    routes (its routed rows rounded to bf16 as the fused call stores them)
+    reproduces the fused call bitwise (route replay control, picx.dev
     summary Sub-study 2)."""
     sh, T = SMALL["bf16_shared_cap"], SMALL_T["bf16_shared_cap"]
     li, x, dli, dx = inputs_on_device(sh, T)
@@ -266,7 +272,10 @@ def test_layer_is_deterministic_and_replayable():
     ys = torch.empty(sh.n_shared, T, sh.d, dtype=torch.float32, device="cuda")
     M.moe_grouped_ffn(cfg, w, xn, offs, perm, gate, y, ys, ws)
     o3 = torch.empty(T, sh.d, dtype=torch.float32, device="cuda")
-    M.moe_combine(cfg, y, slot, ys, dx, o3)
+    # inside the layer the gated routed rows of tensor-core experts are stored in
+    # bf16: the round-to-nearest-even of the same FP32 rows this entry point returns
+    y_layer = y.to(torch.bfloat16).to(torch.float32) if sh.expert != "f32" else y
+    M.moe_combine(cfg, y_layer, slot, ys, dx, o3)
     assert M.moe_get_device_status(ws) == 0
     assert torch.equal(o1, o3)
 
@@ -324,3 +333,48 @@ def test_v3_full_size_sampled(T, v3_weights):
     print(f"v3 T={T}: mismatched routes {res.mismatched} (max margin "
           f"{res.max_margin_mismatch:.2e}), err/rms(out) {res.err_ratio:.3e}, "
           f"err/rms(delta) {res.err_ratio_delta:.3e}")
+
+
+# --------------------------------------------------------------------- alignment
+def _offset_copy(t):
+    """A copy of ``t`` whose data starts one element past a 16-byte boundary."""
+    buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    v = buf[1:].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+def test_misaligned_tensors():
+    """Tensors aligned only to their element type take the scalar kernels and give
+    the same results; tensor-core operands must be 16-byte aligned."""
+    sh, T = SMALL["bf16_shared_cap"], SMALL_T["bf16_shared_cap"]
+    li, x, dli, dx = inputs_on_device(sh, T)
+    layer = M.MoELayer(dli, T, out_dtype="f32")
+    lg = torch.empty(T, sh.E, dtype=torch.float32, device="cuda")
+    ref = layer.forward(dx, logits=lg).clone()
+    # input and output off a 16-byte boundary: scalar RMSNorm and combine, same bits
+    xm = _offset_copy(dx)
+    om = _offset_copy(torch.empty_like(ref))
+    layer.forward(xm, om)
+    assert torch.equal(om, ref)
+    assert M.moe_get_device_status(layer.ws) == 0
+    # router weights off a boundary: the CUDA-core split router, same logits up to
+    # the order of the FP32 additions
+    dli2 = dataclasses.replace(dli, w_router=_offset_copy(dli.w_router))
+    layer2 = M.MoELayer(dli2, T, out_dtype="f32")
+    lg2 = torch.empty_like(lg)
+    layer2.forward(dx, logits=lg2)
+    assert M.moe_get_device_status(layer2.ws) == 0
+    torch.testing.assert_close(lg2, lg, rtol=1e-5, atol=1e-5)
+    # a misaligned TMA operand is an argument error, found before any launch
+    cfg, w = layer.cfg, layer.w
+    ws = M.alloc_workspace(cfg)
+    xn = _offset_copy(torch.zeros(T, sh.d, dtype=torch.bfloat16, device="cuda"))
+    offs = torch.zeros(sh.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.zeros(T * sh.k, dtype=torch.int32, device="cuda")
+    gate = torch.zeros(T * sh.k, dtype=torch.float32, device="cuda")
+    y = torch.empty(T * sh.k, sh.d, dtype=torch.float32, device="cuda")
+    ys = torch.empty(sh.n_shared, T, sh.d, dtype=torch.float32, device="cuda")
+    with pytest.raises(M.MoeError) as e:
+        M.moe_grouped_ffn(cfg, w, xn, offs, perm, gate, y, ys, ws)
+    assert e.value.status == M.MOE_ERR_INVALID
