@@ -93,6 +93,10 @@ struct TcParams {
   // ints, left zeroed again.
   float* split_part;
   int32_t* split_cnt;
+  // ROUTER: K is split into k_splits parts (>= 1); part s writes its partial logits
+  // at out + s * split_out_stride (the routing kernel adds the parts in order)
+  int k_splits;
+  size_t split_out_stride;
 };
 
 constexpr int kMaxSplit = 4;
@@ -398,6 +402,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
   // split-K is compiled into the narrow swapped expert tiles only
   constexpr bool kCanSplit = !DIRECT && EPI != EPI_ROUTER && BN <= 32;
   int S = 1;
+  if (EPI == EPI_ROUTER && p.k_splits > 1) S = p.k_splits;
   if (kCanSplit && p.split_part != nullptr && out_tiles > 0) {
     int kbmin = p.prob[0].K / 64;
     if (p.n_prob > 1 && p.prob[1].K / 64 < kbmin) kbmin = p.prob[1].K / 64;
@@ -786,7 +791,8 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
                 Y[(size_t)r * P.ld_out + n] = __float2bfloat16_rn(v0[j] * s_scale[c * 16 + j]);
             }
           } else {
-            float* Y = reinterpret_cast<float*>(P.out);
+            float* Y = reinterpret_cast<float*>(P.out) +
+                       (EPI == EPI_ROUTER ? ti.ks * p.split_out_stride : 0);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int r = s_row[c * 16 + j];

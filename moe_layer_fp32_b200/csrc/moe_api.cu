@@ -33,8 +33,20 @@ constexpr int kRouterTT = 8;
 inline bool vec_router(const moe_config* c) {
   return !tc_router(c) && c->router_dtype == MOE_BF16 && c->E % 8 == 0 && 256 % (c->E / 8) == 0;
 }
+int num_sms();
+// Tensor-core router: 128-token tiles, K split into parts (partial logits, added
+// in order by the routing kernel) until the SMs are filled; at most 8 parts of at
+// least 4 k-blocks each.
+inline int tc_router_splits(const moe_config* c) {
+  const int tiles = (c->T + 127) / 128 * ((c->E + 127) / 128);
+  int s = num_sms() / tiles;
+  const int kmax = c->d / 64 / 4;
+  if (s > kmax) s = kmax;
+  if (s > 8) s = 8;
+  return s < 1 ? 1 : s;
+}
 inline int router_splits(const moe_config* c) {
-  if (tc_router(c)) return 1;
+  if (tc_router(c)) return tc_router_splits(c);
   if (vec_router(c)) return (c->d + kRouterSlice - 1) / kRouterSlice;
   // K-slices of at least 16 rows: small batches get enough CTAs in flight that the
   // weight loads of the many short slices overlap
@@ -69,7 +81,6 @@ constexpr bool kGather4Int = false;   // int8 / int4 stages hold 4x fewer weight
 inline bool gather_in_gemm(const moe_config* c) {
   return pick_bn(c) <= kGather4MaxBN && (kGather4Int || c->expert_dtype == MOE_BF16);
 }
-int num_sms();
 // Split-K of narrow (decode) tiles when the expert tiles fill at most half the SMs;
 // the GEMM decides per launch from the actual tile count.
 constexpr bool kSplitBf16 = false;   // int experts only: bf16 tiles stream faster whole
@@ -384,14 +395,10 @@ moe_status run_router(const moe_config* c, const moe_weights* w, const void* xn,
     P.n_valid = c->E;
     p.n_prob = 1;
     p.err = err;
-    // narrower token tiles when 128-token tiles would leave most SMs idle
-    const int ftiles = (c->E + 127) / 128;
-    if ((c->T + 127) / 128 * ftiles >= num_sms()) {
-      if (!map_rows(&P.tmB, xn, c->T, c->d, 128)) return MOE_ERR_CUDA;
-      return launch_tc<EPI_ROUTER, 128>(p, st);
-    }
-    if (!map_rows(&P.tmB, xn, c->T, c->d, 32)) return MOE_ERR_CUDA;
-    return launch_tc<EPI_ROUTER, 32>(p, st);
+    p.k_splits = ns;
+    p.split_out_stride = (size_t)c->T * c->E;
+    if (!map_rows(&P.tmB, xn, c->T, c->d, 128)) return MOE_ERR_CUDA;
+    return launch_tc<EPI_ROUTER, 128>(p, st);
   }
   // the vectorised router loads 16-byte weight vectors; other alignments take the
   // split kernel below with the same slices

@@ -33,6 +33,8 @@ SMALL = {
                                capacity_factor=1.25, seed=17),
     "int8_prefill": LayerShape("int8_prefill", d=384, E=8, k=2, f=512, n_shared=1,
                                expert="int8", seed=18),
+    # tensor-core router with K split into 4 parts (partial logits added by the route)
+    "bf16_tc_router_split": LayerShape("bf16_router_split", d=1024, E=64, k=4, f=256, seed=20),
     # FP32 experts with f not a multiple of 4 (scalar weight columns in gate/up)
     "f32_odd_f": LayerShape("f32_odd_f", d=136, E=6, k=2, f=130, n_shared=1, act="f32",
                             router="f32", expert="f32", capacity_factor=1.5,
@@ -40,7 +42,8 @@ SMALL = {
 }
 SMALL_T = {"bf16_plain": 100, "bf16_shared_cap": 77, "bf16_select_tc_router": 200,
            "bf16_prefill_tiles": 1000, "f32_tiny": 64, "int4_decode": 20, "int8_decode": 50,
-           "int4_prefill": 900, "int8_prefill": 700, "f32_odd_f": 37}
+           "int4_prefill": 900, "int8_prefill": 700, "f32_odd_f": 37,
+           "bf16_tc_router_split": 300}
 
 
 @pytest.fixture(autouse=True)
@@ -53,7 +56,8 @@ def tdev(a, dtype):
 
 
 # --------------------------------------------------------------------- a1 + a2
-@pytest.mark.parametrize("name", ["bf16_plain", "bf16_select_tc_router", "f32_tiny"])
+@pytest.mark.parametrize("name", ["bf16_plain", "bf16_select_tc_router", "bf16_tc_router_split",
+                                  "f32_tiny", "f32_odd_f"])
 def test_rmsnorm_bitexact_and_router(name):
     sh, T = SMALL[name], SMALL_T[name]
     li, x, dli, dx = inputs_on_device(sh, T)
