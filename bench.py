@@ -148,16 +148,25 @@ def max_over_ranks(v: float, world: int) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_throughput(units_per_rank: float, ms_local: float, world: int):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's
+    time (ms).  Returns (units/s, slowest ms)."""
+    ms_max = max_over_ranks(ms_local, world)
+    return units_per_rank * world / (ms_max / 1e3), ms_max
 
 
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def cpu_threads():
@@ -235,11 +244,9 @@ def run_ours(args):
     clk = clocks.stop()
     ms = start.elapsed_time(end)
     assert M.moe_get_device_status(layer.ws) == 0, "device error word set"
-    ms_max = max_over_ranks(ms, world)
+    value, ms_max = aggregate_throughput(T * K, ms, world)
     per_kernel = {n: float(np.mean([evs[s][i].elapsed_time(evs[s][i + 1]) for s in prof_steps]))
                   for i, n in enumerate(names)}
-    tokens_total = T * K * world
-    value = tokens_total / (ms_max / 1e3)
 
     # roofline of the dominant kernel
     peaks = R.measured_peaks()
@@ -323,8 +330,8 @@ def run_e2e(M, layer, x_host, sh, T, K, world):
         outp.copy_(od, non_blocking=True)
     e.record()
     torch.cuda.synchronize()
-    ms = max_over_ranks(s.elapsed_time(e), world)
-    return {"value": round(T * K * world / (ms / 1e3), 1), "unit": "tokens/s",
+    value, _ = aggregate_throughput(T * K, s.elapsed_time(e), world)
+    return {"value": round(value, 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(xp.numel() * xp.element_size()),
             "d2h_bytes_per_step": int(outp.numel() * outp.element_size()), "steps": K}
 
