@@ -228,20 +228,27 @@ moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32
 
 /* The whole layer: a1..a8 chained on one stream, no host synchronisation.
  *   x [T, d] act dtype, out [T, d] out dtype.  Optional outputs (NULL to skip):
- *   logits_out [T, E] float32, topk_idx_out [T, k] int32, counts_out [E] int32. */
+ *   logits_out [T, E] float32, topk_idx_out [T, k] int32, counts_out [E] int32.
+ * Between the down GEMM and the combine the gated routed rows of tensor-core
+ * experts are kept in bf16 (the round-to-nearest-even of the FP32 rows that
+ * moe_grouped_ffn returns), so the result equals moe_combine applied to those
+ * rounded rows, bit for bit. */
 moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const void* x,
                              void* out, void* ws, size_t ws_bytes, float* logits_out,
                              int32_t* topk_idx_out, int32_t* counts_out, void* stream);
 
 /* moe_layer_forward with per-step timing marks, for profiling: events[0] is
  * recorded on `stream` before the first kernel and events[i] right after step i
- * (i = 1 .. moe_layer_step_count(cfg); the steps are RMSNorm, router, route,
- * permute, [dequantise + gather], gate/up GEMM, down GEMM, combine -- that step
- * exists for tensor-core experts; at prefill batch sizes it gathers the routed
- * token rows (and dequantises int8/int4 experts), at decode sizes the gate/up
- * GEMM gathers them itself and the step is empty).  `events` holds caller-created cudaEvent_t handles (as
- * void*); n_events must be at least moe_layer_step_count(cfg) + 1.  No
- * optional outputs. */
+ * (i = 1 .. moe_layer_step_count(cfg)).  The steps are RMSNorm, router, route,
+ * permute, [dequantise + gather], gate/up GEMM, down GEMM, combine:
+ *   - up to 32 tokens the route launch also builds the permutation, and the
+ *     permute step is empty;
+ *   - the bracketed step exists for tensor-core experts: it gathers the routed
+ *     token rows (and, at prefill batch sizes, dequantises int8/int4 experts),
+ *     except on bf16 decode tiles, where the gate/up GEMM gathers them itself
+ *     and the step is empty.
+ * `events` holds caller-created cudaEvent_t handles (as void*); n_events must be
+ * at least moe_layer_step_count(cfg) + 1.  No optional outputs. */
 moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* w,
                                       const void* x, void* out, void* ws, size_t ws_bytes,
                                       void* const* events, int32_t n_events, void* stream);
