@@ -802,11 +802,21 @@ __global__ void __launch_bounds__(256) k_gather_rows(const TA* __restrict__ xn,
   const int n_rows = *n_rows_ptr;
   const int vec_per_row = d * (int)sizeof(TA) / 16;
   const int warps = gridDim.x * 8;
+  const int lane = threadIdx.x & 31;
+  constexpr int U = 8;   // vectors per lane loaded before they are stored
   for (int s = blockIdx.x * 8 + (threadIdx.x >> 5); s < n_rows; s += warps) {
     const int t = perm_assign[s] / k;
     const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)s * d);
-    for (int i = threadIdx.x & 31; i < vec_per_row; i += 32) dst[i] = src[i];
+    for (int i0 = lane; i0 < vec_per_row; i0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + 32 * u < vec_per_row) v[u] = src[i0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + 32 * u < vec_per_row) dst[i0 + 32 * u] = v[u];
+    }
   }
 }
 

@@ -619,7 +619,8 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     return MOE_ERR_CUDA;
   __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
   if (!g4) {
-    MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 2 * num_sms(), 256, 0, st,
+    // 64 warps per SM, so that many rows are in flight at once
+    MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 8 * num_sms(), 256, 0, st,
                static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
     if ((s = check_launch()) != MOE_OK) return s;
   }
