@@ -129,3 +129,24 @@ def test_make_weights_maps_every_layer_tensor():
     w = M.make_weights(li)
     assert w.rms_gamma == 4096 and w.w_router == 8192 and w.sh_down == 4096 * 9
     assert w.s_gate is None and w.sh_s_gate is None
+
+
+# (preset, T) -> kernel launches per layer call.  Six always run (RMSNorm, router,
+# route, gate/up, down, combine); the permutation adds 0 (it shares the routing
+# launch up to 32 tokens), 1 (one CTA, T*k <= 4096) or 3 (count / scan / rank);
+# tensor-core experts add the row gather unless bf16 decode tiles (<= 32 rows per
+# expert on average) gather inside the GEMM; int8/int4 experts at 128-token tiles
+# add the one-pass dequantisation.
+LAUNCHES = [("tiny", 64, 7), ("olmoe", 1, 6), ("olmoe", 16, 6), ("olmoe", 64, 7),
+            ("olmoe", 4096, 10), ("v2lite", 32, 6), ("v2lite", 8192, 10),
+            ("qwen3_int4", 1, 7), ("qwen3_int4", 64, 8), ("qwen3_int4", 16384, 11),
+            ("qwen3_int8", 16384, 11), ("v3", 32, 6), ("v3", 256, 7), ("v3", 9440, 10)]
+
+
+@pytest.mark.parametrize("preset,T,n", LAUNCHES)
+def test_launch_and_step_counts(lib, preset, T, n):
+    sh = moe_synth.PRESETS[preset]
+    cfg = M.make_config(sh, T)
+    assert M.moe_layer_launch_count(cfg) == n
+    # profiled steps: 7 for FP32 experts, 8 with the [dequantise + gather] step
+    assert M.moe_layer_step_count(cfg) == (7 if sh.expert == "f32" else 8)
