@@ -26,7 +26,7 @@ Sources (page title, then section):
 * "MoE at the inference level ...", Workarounds: gather -> grouped GEMM ->
   scatter; int4 expert weights.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * RMSNorm: ``xn = x * (mean(x^2) + eps)^-1/2 * gamma``, computed in float64 and
   rounded once to the activation dtype (bf16 or fp32) -- the experts and the

@@ -1,7 +1,7 @@
 """Helpers for the GPU parity tests: run the CUDA path through the C ABI and the
 CPU oracle on the same seeded inputs, and compare them.
 
-Tolerances (derivations in the design doc):
+Tolerances (each derived from the arithmetic of the path):
 * routing indices, counts, offsets, permutation: bit-exact given the same FP32
   logits; end to end, a token may differ from the oracle's selection only where
   the oracle's k-th/(k+1)-th key margin is below 1e-4;
