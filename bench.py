@@ -517,8 +517,8 @@ def run_reference(args):
     x = moe_synth.make_x(sh, T)
     # size each step's sample so the whole run takes a few minutes
     probe = time_oracle(li, x, 1)
-    budget = 150.0
-    per_step = budget / (K + W)
+    target_s = 150.0   # seconds for the whole reference run
+    per_step = target_s / (K + W)
     n_tok = 1
     if per_step > 2 * probe:
         n_tok = int(min(T, max(1, (per_step / probe))))

@@ -88,7 +88,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def measured_peaks(path: Optional[str] = None) -> dict:
-    """The machine's measured peaks (generated file), else the fallback."""
+    """Peaks measured on this kind of GPU (MEASURED_PEAKS.json at the repository
+    root: a copy-kernel HBM bandwidth and cuBLAS bf16 throughput), else the
+    fallback figures above."""
     path = path or os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                                 "MEASURED_PEAKS.json")
     try:
