@@ -2,15 +2,17 @@
 """Benchmark of the top-k MoE FFN layer forward on B200.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
-                    [--preset olmoe --tokens 4096] [--no-sweep] [--no-cpu]
+                    [--preset v3 --tokens 9440] [--no-sweep] [--no-cpu] [--no-parity]
 
 One step = one whole layer forward (RMSNorm, router, top-k, permutation,
 grouped gate/up and down GEMMs, combine) over one batch of T synthetic tokens,
-through the C ABI (moe_layer_forward).  Default workload: the OLMoE-1B-7B-shaped
-layer (d 2048, 64 experts, top-8, expert hidden 1024, bf16) at T = 4096 prefill
-tokens.  With N > 1 (torchrun) every rank runs its own batch on its own GPU with
-replicated weights -- token data parallelism, no collective on the data path
-(weak scaling); the step time is the max over ranks.
+through the C ABI (moe_layer_forward).  Default workload: the largest
+single-GPU configuration, the DeepSeek-V3-shaped layer (d 7168, 256 routed
+experts with a Zipf(1.1)-skewed select-mode bias, top-8, expert hidden 2048, one
+shared expert, bf16) at T = 9440 tokens, the batch where this layer crosses from
+memory- to compute-bound.  With N > 1 (torchrun) every rank runs its own batch
+on its own GPU with replicated weights -- token data parallelism, no collective
+on the data path (weak scaling); the step time is the max over ranks.
 
 Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle (the
 only reference this layer has) on the host cores instead.
@@ -45,15 +47,15 @@ KERNEL_NAMES_SIMT = ["rmsnorm", "router", "route_topk", "permute", "gateup_simt"
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
-    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--preset", default="olmoe")
-    p.add_argument("--tokens", type=int, default=4096)
-    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--preset", default="v3")
+    p.add_argument("--tokens", type=int, default=9440)
+    p.add_argument("--no-sweep", action="store_true",
+                   help="skip the other configurations (decode and prefill batches)")
     p.add_argument("--no-cpu", action="store_true")
-    p.add_argument("--all-configs", action="store_true",
-                   help="also time every preset and token count (stream and CUDA graph)")
+    p.add_argument("--no-parity", action="store_true")
     return p.parse_args()
 
 
@@ -72,8 +74,8 @@ def config_dict(sh, T, world):
             "expert_dtype": sh.expert, "router_dtype": sh.router, "bias_mode": sh.bias_mode,
             "capacity_factor": sh.capacity_factor, "renormalize": sh.renormalize,
             "parallelism": f"replicas x{world} (token data parallel, no collective)",
-            "l2": "inputs larger than L2 (126 MB): every step streams all touched expert "
-                  "weights (%.0f MB at this batch)" % (
+            "l2": "not flushed; inputs larger than L2 (126 MB): the routed experts' weights "
+                  "total %.0f MB and every step streams the touched ones from HBM" % (
                       R.expert_bytes(sh.expert, sh.d, sh.f, sh.group_size) * sh.E / 1e6)}
 
 
@@ -189,6 +191,17 @@ def time_oracle(li, x, n_tokens, reps=1):
     return (time.perf_counter() - t0) / reps
 
 
+def routing_stats(sh, T, counts):
+    """(kept rows, touched experts) of one batch from its per-expert counts."""
+    cnt = counts.cpu().numpy()
+    cap = None
+    if sh.capacity_factor > 0:
+        import math
+        cap = math.ceil(float(np.float32(sh.capacity_factor)) * T * sh.k / sh.E)
+    kept = int(np.minimum(cnt, cap).sum()) if cap else int(cnt.sum())
+    return kept, int((cnt > 0).sum())
+
+
 # --------------------------------------------------------------------- our arm
 def run_ours(args):
     import moe_layer_fp32_b200 as M
@@ -211,13 +224,7 @@ def run_ours(args):
     counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
     out = layer.forward(x, counts=counts)
     torch.cuda.synchronize()
-    cnt = counts.cpu().numpy()
-    cap = None
-    if sh.capacity_factor > 0:
-        import math
-        cap = math.ceil(float(np.float32(sh.capacity_factor)) * T * sh.k / sh.E)
-    kept = int(np.minimum(cnt, cap).sum()) if cap else int(cnt.sum())
-    touched = int((cnt > 0).sum())
+    kept, touched = routing_stats(sh, T, counts)
 
     for _ in range(W):
         layer.forward(x, out)
@@ -248,8 +255,9 @@ def run_ours(args):
     per_kernel = {n: float(np.mean([evs[s][i].elapsed_time(evs[s][i + 1]) for s in prof_steps]))
                   for i, n in enumerate(names)}
 
-    # roofline of the dominant kernel
+    # the peak that applies to a kernel timed inside this loop (burst or sustained)
     peaks = R.measured_peaks()
+    tc_peak, peak_label = R.tensor_peak(peaks, ms_max / 1e3, clk.get("sm_mhz"))
     dom = max(per_kernel, key=per_kernel.get)
     dom_ms = per_kernel[dom]
     if dom in ("gateup_gemm", "down_gemm", "router"):
@@ -259,12 +267,10 @@ def run_ours(args):
             fl = 2.0 * sh.d * sh.f * (kept + sh.n_shared * T)
         else:
             fl = 2.0 * T * sh.d * sh.E
-        tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         ach = fl / (dom_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 2),
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(ach / tc_peak, 4),
-                "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a "
-                               "seconds-long loop)",
+                "peak_source": peak_label,
                 "algorithmic_per_launch": fl, "avg_launch_us": round(dom_ms * 1e3, 2),
                 "traffic": read_traffic(dom, sh, T)}
     else:
@@ -272,38 +278,36 @@ def run_ours(args):
         ach = nb / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peaks['source']} hbm_gbs (copy kernel)",
                 "avg_launch_us": round(dom_ms * 1e3, 2), "traffic": None}
     # whole-layer roofline (slower of flops at the tensor peak and bytes over HBM)
     fl_layer = R.layer_flops(sh, T, kept)
     by_layer = R.layer_bytes(sh, T, touched)
-    t_roof = R.roofline_time(fl_layer, by_layer,
-                             peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12,
-                             peaks["hbm_gbs"] * 1e9)
+    t_roof = R.roofline_time(fl_layer, by_layer, tc_peak * 1e12, peaks["hbm_gbs"] * 1e9)
     layer_roof = {"t_roof_us": round(t_roof * 1e6, 2), "t_step_us": round(ms_max / K * 1e3, 2),
                   "frac": round(t_roof / (ms_max / K / 1e3), 4),
-                  "bound": "tensor" if fl_layer / (peaks.get("bf16_tflops_sustained", 1) * 1e12)
+                  "bound": "tensor" if fl_layer / (tc_peak * 1e12)
                   > by_layer / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                  "peak_tflops": tc_peak, "peak_gbs": peaks["hbm_gbs"],
                   "flops": fl_layer, "bytes": by_layer, "touched_experts": touched,
                   "kept_rows": kept}
 
     # end to end through the C ABI with host buffers
-    e2e = run_e2e(M, layer, x_host, sh, T, min(K, 200), world)
+    e2e = run_e2e(M, layer, x_host, sh, T, min(K, 100), world)
 
     res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
            "steps": K, "warmup": W, "ms_per_step": round(ms_max / K, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic (seeded N(0,1) tokens, fan-in-scaled random expert weights)",
            "config": config_dict(sh, T, world), "roofline": roof, "layer_roofline": layer_roof,
-           "e2e": e2e, "gpu_launches": L * K, "clocks": clk,
+           "e2e": e2e, "gpu_launches": L * K, "launches_per_step": L, "clocks": clk,
            "kernels_avg_us": {k: round(v * 1e3, 2) for k, v in per_kernel.items()}}
+    if rank == 0 and world == 1 and not args.no_parity:
+        res["parity"] = parity_sample(M, layer, li_host, x_host, x, sh, T)
     if rank == 0 and world == 1 and not args.no_sweep:
-        res["sweep"] = run_sweep(M, dev)
+        res["sweep"] = run_sweep(M, dev, sh, T, li)
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(li_host, x_host, sh, T)
-    if rank == 0 and world == 1 and args.all_configs:
-        del li, layer
-        torch.cuda.empty_cache()
-        res["all_configs"] = run_all_configs(M, dev)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -336,61 +340,33 @@ def run_e2e(M, layer, x_host, sh, T, K, world):
             "d2h_bytes_per_step": int(outp.numel() * outp.element_size()), "steps": K}
 
 
-def run_sweep(M, dev):
-    """Decode batches of the same layer: whole-layer time, stream-launched and
-    replayed from a CUDA graph, and the fraction of the HBM roofline."""
-    sh = moe_synth.PRESETS["olmoe"]
-    li = moe_synth.make_layer(sh).to(dev)
-    peaks = R.measured_peaks()
-    out = []
-    for T in (1, 16, 64):
-        x = moe_synth.make_x(sh, T).to(dev)
-        layer = M.MoELayer(li, T)
-        counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
-        o = layer.forward(x, counts=counts)
-        torch.cuda.synchronize()
-        touched = int((counts.cpu().numpy() > 0).sum())
-        for _ in range(20):
-            layer.forward(x, o)
-        n = 500
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        s.record()
-        for _ in range(n):
-            layer.forward(x, o)
-        e.record()
-        torch.cuda.synchronize()
-        us_stream = s.elapsed_time(e) / n * 1e3
-        us_graph = None
-        try:
-            g = torch.cuda.CUDAGraph()
-            st = torch.cuda.Stream()
-            with torch.cuda.stream(st):
-                layer.forward(x, o)
-                st.synchronize()
-                with torch.cuda.graph(g, stream=st):
-                    layer.forward(x, o, stream=st)
-            for _ in range(20):
-                g.replay()
-            torch.cuda.synchronize()
-            s.record()
-            for _ in range(n):
-                g.replay()
-            e.record()
-            torch.cuda.synchronize()
-            us_graph = s.elapsed_time(e) / n * 1e3
-            del g
-        except Exception as ex:  # capture problems are reported, not hidden
-            us_graph = f"capture failed: {ex}"
-        nb = R.layer_bytes(sh, T, touched)
-        best = min(us_stream, us_graph) if isinstance(us_graph, float) else us_stream
-        out.append({"workload": workload_name(sh, T), "T": T, "touched_experts": touched,
-                    "us_per_layer_stream": round(us_stream, 2),
-                    "us_per_layer_graph": round(us_graph, 2) if isinstance(us_graph, float) else us_graph,
-                    "tokens_per_s": round(T / (best / 1e6), 1),
-                    "hbm_roofline_us": round(nb / (peaks["hbm_gbs"] * 1e9) * 1e6, 2),
-                    "hbm_frac": round(nb / (best / 1e6) / (peaks["hbm_gbs"] * 1e9), 4)})
-    return out
+def parity_sample(M, layer, li_host, x_host, x, sh, T, n_rows=8):
+    """This batch's output (FP32, the layer the bench times) against the oracle on
+    sampled rows: the oracle routes the whole batch itself (route mismatches and
+    drift) and is then re-run with the GPU's routes on the sampled rows (output
+    error over RMS(out) and over RMS(out - x))."""
+    from moe_layer_fp32_b200.drift import route_drift
+    from oracle import moe_oracle as O
+    t0 = time.perf_counter()
+    l32 = M.MoELayer(layer.inputs, T, out_dtype="f32")
+    idx = torch.empty(T, sh.k, dtype=torch.int32, device=x.device)
+    out = l32.forward(x, topk_idx=idx).float().cpu().numpy()
+    gi = idx.cpu().numpy()
+    del l32
+    r = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, T - 1], r.choice(T, min(T, n_rows) - 2 if T > 2 else 0,
+                                                           replace=False)]))
+    own = O.layer_from_inputs(li_host, x_host, tokens=[0])
+    rep = O.layer_from_inputs(li_host, x_host, forced_idx=gi, tokens=rows)
+    diff = (np.sort(gi, 1) != np.sort(own["idx"], 1)).any(1)
+    x64 = x_host.float().numpy().astype(np.float64)[rows]
+    err = float(np.max(np.abs(out[rows] - rep["out"])))
+    return {"rows": int(rows.size), "route_mismatches": int(diff.sum()),
+            "max_margin_of_mismatch": float(own["margin"][diff].max()) if diff.any() else 0.0,
+            "drift": route_drift(gi, own["idx"]),
+            "err_over_rms_out": err / float(np.sqrt(np.mean(rep["out"] ** 2))),
+            "err_over_rms_delta": err / float(np.sqrt(np.mean((rep["out"] - x64) ** 2))),
+            "oracle_s": round(time.perf_counter() - t0, 1)}
 
 
 def time_layer(M, layer, x, n):
@@ -406,75 +382,99 @@ def time_layer(M, layer, x, n):
     e.record()
     torch.cuda.synchronize()
     us_stream = s.elapsed_time(e) / n * 1e3
-    g = torch.cuda.CUDAGraph()
-    st = torch.cuda.Stream()
-    with torch.cuda.stream(st):
-        layer.forward(x, o, stream=st)
-        st.synchronize()
-        with torch.cuda.graph(g, stream=st):
+    us_graph = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
             layer.forward(x, o, stream=st)
-    for _ in range(10):
-        g.replay()
-    torch.cuda.synchronize()
-    s.record()
-    for _ in range(n):
-        g.replay()
-    e.record()
-    torch.cuda.synchronize()
-    us_graph = s.elapsed_time(e) / n * 1e3
-    del g
+            st.synchronize()
+            with torch.cuda.graph(g, stream=st):
+                layer.forward(x, o, stream=st)
+        for _ in range(10):
+            g.replay()
+        torch.cuda.synchronize()
+        s.record()
+        for _ in range(n):
+            g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        us_graph = s.elapsed_time(e) / n * 1e3
+        del g
+    except Exception as ex:  # capture problems are reported, not hidden
+        us_graph = f"capture failed: {ex}"
     return us_stream, us_graph
 
 
-def run_all_configs(M, dev):
-    """Every preset at every token count: time per layer and the fraction of the
-    layer roofline (the slower of flops at the measured sustained bf16 peak and
-    touched-weight bytes at the measured HBM bandwidth)."""
+SWEEP = [("olmoe", 1), ("olmoe", 16), ("olmoe", 64), ("olmoe", 4096), ("v2lite", 32),
+         ("v2lite", 8192), ("qwen3_int4", 1), ("qwen3_int4", 64), ("qwen3_int4", 16384),
+         ("qwen3_int8", 1), ("qwen3_int8", 64), ("qwen3_int8", 16384), ("v3", 32), ("v3", 256),
+         ("v3", 9440), ("tiny", 64)]
+
+
+def run_sweep(M, dev, head_sh, head_T, head_li):
+    """Every other configuration: whole-layer time, stream-launched and replayed
+    from a CUDA graph, and the fraction of the layer roofline (the slower of the
+    flops at the bf16 peak that applies to the loop and the touched-weight bytes
+    at the measured HBM bandwidth)."""
     peaks = R.measured_peaks()
-    pf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
     bw = peaks["hbm_gbs"] * 1e9
     rows = []
-    for name in ("tiny", "olmoe", "v2lite", "qwen3_int4", "qwen3_int8", "v3"):
+    cache = {head_sh.name: head_li}
+    for name in dict.fromkeys(n for n, _ in SWEEP):
         sh = moe_synth.PRESETS[name]
-        li = moe_synth.make_layer(sh).to(dev)
-        for T in sh.tokens:
+        li = cache.get(name)
+        if li is None:
+            li = moe_synth.make_layer(sh).to(dev)
+        for pname, T in SWEEP:
+            if pname != name or (name == head_sh.name and T == head_T):
+                continue
             x = moe_synth.make_x(sh, T).to(dev)
             layer = M.MoELayer(li, T)
             counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
             layer.forward(x, counts=counts)
             torch.cuda.synchronize()
-            cnt = counts.cpu().numpy()
-            cap = None
-            if sh.capacity_factor > 0:
-                import math
-                cap = math.ceil(float(np.float32(sh.capacity_factor)) * T * sh.k / sh.E)
-            kept = int(np.minimum(cnt, cap).sum()) if cap else int(cnt.sum())
-            touched = int((cnt > 0).sum())
-            n = 50 if T >= 4096 else 300
+            kept, touched = routing_stats(sh, T, counts)
+            n = 40 if T >= 4096 else 400
             us_s, us_g = time_layer(M, layer, x, n)
+            best = min(us_s, us_g) if isinstance(us_g, float) else us_s
+            pf, _ = R.tensor_peak(peaks, best * n / 1e6)
             fl, nb = R.layer_flops(sh, T, kept), R.layer_bytes(sh, T, touched)
-            t_roof = R.roofline_time(fl, nb, pf, bw)
-            best = min(us_s, us_g)
+            t_roof = R.roofline_time(fl, nb, pf * 1e12, bw)
             rows.append({"workload": workload_name(sh, T), "T": T, "touched": touched,
-                         "kept": kept, "us_stream": round(us_s, 1), "us_graph": round(us_g, 1),
+                         "kept": kept, "launches": M.moe_layer_launch_count(layer.cfg),
+                         "us_stream": round(us_s, 1),
+                         "us_graph": round(us_g, 1) if isinstance(us_g, float) else us_g,
                          "tokens_per_s": round(T / (best / 1e6), 1),
                          "roofline_us": round(t_roof * 1e6, 1),
-                         "bound": "tensor" if fl / pf > nb / bw else "hbm",
+                         "bound": "tensor" if fl / (pf * 1e12) > nb / bw else "hbm",
                          "frac": round(t_roof * 1e6 / best, 4)})
             del layer
-        del li
+        if name != head_sh.name:
+            del li
         torch.cuda.empty_cache()
     return rows
 
 
-def cpu_baseline(li_host, x_host, sh, T, n_tokens=512):
-    """The oracle, as it stands, on the host cores: the first n_tokens rows of
-    the same batch (routing over that sub-batch, every expert they touch)."""
-    n = min(n_tokens, T)
+def cpu_baseline(li_host, x_host, sh, T):
+    """The oracle, as it stands, on the host cores: the first tokens of the same
+    batch (routing over that sub-batch, every expert they touch), once on all
+    the threads numpy's BLAS uses and once on a single thread."""
+    n = min(T, 32 if sh.d >= 4096 else 512)
     sec = time_oracle(li_host, x_host, n)
-    return {"value": round(n / sec, 2), "unit": "tokens/s", "cores": cpu_threads(),
-            "kind": "oracle", "sample": f"first {n} of the {T} tokens of the timed batch, one "
-                                        f"call ({sec:.1f} s), numpy float64"}
+    res = {"value": round(n / sec, 2), "unit": "tokens/s", "cores": cpu_threads(),
+           "kind": "oracle", "sample": f"first {n} of the {T} tokens of the timed batch, one "
+                                       f"call ({sec:.1f} s), numpy float64"}
+    try:
+        import threadpoolctl
+        n1 = max(1, n // 4)
+        with threadpoolctl.threadpool_limits(limits=1):
+            sec1 = time_oracle(li_host, x_host, n1)
+        res["single_thread"] = {"value": round(n1 / sec1, 2), "unit": "tokens/s", "cores": 1,
+                                "sample": f"first {n1} tokens, one call ({sec1:.1f} s)"}
+    except Exception as ex:  # reported, not hidden
+        res["single_thread"] = f"unavailable: {ex}"
+    return res
 
 
 # --------------------------------------------------------------------- traffic

@@ -27,8 +27,11 @@
  *
  * Conventions common to every entry point:
  *   - Every tensor pointer is DEVICE memory owned by the caller; shapes are
- *     row-major with the last index contiguous.  The library allocates nothing
- *     and keeps no global state.
+ *     row-major with the last index contiguous.  The library allocates no device
+ *     memory.  Its only state shared between calls is the built-in scratch
+ *     array of moe_permute_static (1 MiB per device, see there for the rule on
+ *     overlapping calls); every other entry point works in the caller's
+ *     workspace only.
  *   - Alignment: tensors need only the alignment of their element type, except
  *     that with tensor-core experts (bf16 / int8 / int4) xn, the expert weights
  *     and their scales must be 16-byte aligned (TMA operands; MOE_ERR_INVALID
@@ -94,6 +97,10 @@ typedef struct moe_config {
   int32_t router_dtype;    /* W_r: MOE_BF16 or MOE_F32 (must equal act_dtype)           */
   int32_t expert_dtype;    /* MOE_F32 (requires act F32) | MOE_BF16 | MOE_INT8 | MOE_INT4 */
   int32_t group_size;      /* int4: scale group along K; must be 128                    */
+  int32_t wait_kcycles;    /* limit of every pipeline wait inside the kernels, in units of
+                              1024 SM clock cycles; 0 = the default, 10^9 cycles (about
+                              half a second).  A wait that runs out sets device error 2
+                              and the kernel returns early (moe_get_device_status)      */
 } moe_config;
 
 /* Layer weights (device pointers, caller-owned).
@@ -130,12 +137,16 @@ typedef struct moe_weights {
 /* Bytes of device workspace the calls below need for this configuration (worst
  * case over routings: T*k kept slots).  0 on an invalid configuration.  The
  * workspace needs 256-byte alignment; its first 4 bytes are the device error
- * word.  Fixed size and fixed addresses make the calls capturable in a CUDA
- * graph ("MoE: dynamism the compiler cannot remove", grouped GEMM section:
- * descriptor buffers at fixed addresses with fixed maximum sizes). */
+ * word.
+ * Source: "MoE: dynamism the compiler cannot remove", grouped GEMM section --
+ * the per-expert row counts are data dependent, so the grouped kernels read
+ * them from descriptor buffers kept at fixed addresses and sized for the worst
+ * case (every one of the T*k assignments kept); a fixed size and fixed
+ * addresses are also what lets the calls be captured in a CUDA graph. */
 size_t moe_workspace_size(const moe_config* cfg);
 
-/* Zero the device error word (asynchronous). */
+/* Zero the device error word (asynchronous).  The pages have no counterpart:
+ * it resets the failure report that moe_get_device_status reads. */
 moe_status moe_clear_device_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Steps a1 + a2: RMSNorm and the router GEMM.
@@ -150,6 +161,11 @@ moe_status moe_rmsnorm_router(const moe_config* cfg, const moe_weights* w, const
                               void* stream);
 
 /* Step a3: softmax + top-k + bias + renormalisation, one warp per token.
+ * Sources: picx.dev summary of the moe-ceilings study, Sub-study 1
+ * (FusedSoftmax: the gate probabilities are accumulated in FP32 before the
+ * top-k); "MoE: dynamism the compiler cannot remove", natural implementation
+ * (router logits -> top-k indices and weights); "MoE Research", section 2
+ * (per-expert bias terms that move the selection to even out the load).
  *   logits    [T, E] float32 router logits (bias not included)
  *   bias      [E] float32 or NULL (see moe_bias_mode)
  *   topk_idx  [T, k] int32: selected experts by descending key (logit, plus the
@@ -217,7 +233,13 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const vo
                            const float* topk_gate, float* y_assign, float* y_shared,
                            void* ws, size_t ws_bytes, void* stream);
 
-/* Step a8: combine.  out[t] = residual[t] + sum_s y_shared[s, t] +
+/* Step a8: combine.
+ * Sources: "MoE: dynamism the compiler cannot remove", natural implementation
+ * (each expert's output, weighted by its gate, is added into the token's output
+ * row) and capacity section (a token slot dropped by capacity contributes
+ * nothing: the token passes through on the residual); "MoE Research", section 2
+ * (the shared experts' outputs are added for every token).
+ * out[t] = residual[t] + sum_s y_shared[s, t] +
  * sum_{j : slot_of[t*k+j] >= 0} y_assign[t*k+j], summed in FP32 in that fixed order
  * (deterministic), rounded to the activation dtype.
  *   residual [T, d] act dtype or NULL (then out is the MoE delta only)
@@ -227,6 +249,12 @@ moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32
                        void* stream);
 
 /* The whole layer: a1..a8 chained on one stream, no host synchronisation.
+ * Source: the whole chain of "MoE: dynamism the compiler cannot remove",
+ * natural implementation (pre-norm, router, top-k, dispatch to the experts,
+ * gated sum) with its capacity section, in the grouped form of that page's
+ * grouped GEMM section (one launch over all experts' rows) and the
+ * gather -> grouped GEMM -> scatter structure of "MoE at the inference level",
+ * Workarounds.
  *   x [T, d] act dtype, out [T, d] out dtype.  Optional outputs (NULL to skip):
  *   logits_out [T, E] float32, topk_idx_out [T, k] int32, counts_out [E] int32.
  * Between the down GEMM and the combine the gated routed rows of tensor-core
@@ -237,7 +265,10 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
                              void* out, void* ws, size_t ws_bytes, float* logits_out,
                              int32_t* topk_idx_out, int32_t* counts_out, void* stream);
 
-/* moe_layer_forward with per-step timing marks, for profiling: events[0] is
+/* moe_layer_forward with per-step timing marks, for profiling.
+ * Source: picx.dev summary of the moe-ceilings study, Summary and Sub-study 1
+ * (the forward is profiled module by module to find where the time goes before
+ * anything is fused).  events[0] is
  * recorded on `stream` before the first kernel and events[i] right after step i
  * (i = 1 .. moe_layer_step_count(cfg)).  The steps are RMSNorm, router, route,
  * permute, [dequantise + gather], gate/up GEMM, down GEMM, combine:
@@ -255,17 +286,28 @@ moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* 
 
 /* Synchronise `stream`, then read the device error word into *code (0 = none;
  * 1 = expert id out of range; 2 = a pipeline wait ran out).  Returns MOE_ERR_DEVICE
- * when the word is nonzero. */
+ * when the word is nonzero.
+ * The pages have no counterpart: this is the failure-detection side of the
+ * boundary.  The grouped GEMMs' pipelines wait on barriers inside the kernel
+ * (the persistent, descriptor-driven form of "MoE: dynamism the compiler cannot
+ * remove", grouped GEMM section); every such wait is bounded, and a wait that
+ * runs out, or a routed expert id outside [0, E), is reported here instead of
+ * trapping the device. */
 moe_status moe_get_device_status(const void* ws, int32_t* code, void* stream);
 
-/* Static, human-readable name of a status. */
+/* Static, human-readable name of a status (no counterpart in the pages). */
 const char* moe_status_string(moe_status s);
 
 /* Number of kernels moe_layer_forward launches for this configuration (for
- * launch accounting); 0 on an invalid configuration. */
+ * launch accounting); 0 on an invalid configuration.
+ * Source: "MoE: dynamism the compiler cannot remove", batch-1 section, and the
+ * picx.dev summary of the moe-ceilings study, Practical Implications: the MoE
+ * layer is launch bound at small batches (about a thousand launches per forward
+ * with a per-expert loop), so the number of launches is a figure to report. */
 int32_t moe_layer_launch_count(const moe_config* cfg);
 
-/* Number of steps moe_layer_forward_profiled marks (see there); 0 if invalid. */
+/* Number of steps moe_layer_forward_profiled marks (see there, and its source);
+ * 0 if invalid. */
 int32_t moe_layer_step_count(const moe_config* cfg);
 
 #ifdef __cplusplus

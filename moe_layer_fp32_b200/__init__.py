@@ -31,7 +31,7 @@ class MoeConfig(ctypes.Structure):
                 ("bias_mode", ctypes.c_int32), ("rms_eps", ctypes.c_float),
                 ("act_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
                 ("router_dtype", ctypes.c_int32), ("expert_dtype", ctypes.c_int32),
-                ("group_size", ctypes.c_int32)]
+                ("group_size", ctypes.c_int32), ("wait_kcycles", ctypes.c_int32)]
 
 
 class MoeWeights(ctypes.Structure):

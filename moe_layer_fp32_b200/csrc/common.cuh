@@ -1,6 +1,6 @@
 // Device helpers shared by the layer's kernels: error word, number conversion,
 // and thin inline-PTX wrappers for the sm_100a async machinery (mbarrier, TMA,
-// tcgen05 / TMEM).  Every wait here is bounded: it gives up after a fixed
+// tcgen05 / TMEM).  Every wait here is bounded: it gives up after a given
 // number of clock cycles, records an error code and returns false.
 #pragma once
 #include <cuda_runtime.h>
@@ -13,7 +13,11 @@ namespace moe {
 
 enum DeviceError : int32_t { DEV_OK = 0, DEV_BAD_EXPERT = 1, DEV_TIMEOUT = 2 };
 
-// a wait gives up after this many SM clock cycles (about half a second)
+// Default limit of a pipeline wait, in SM clock cycles (about half a second).
+// The layer's configuration can set a shorter one (moe_config.wait_kcycles);
+// the drains at the end of a kernel (copies and MMAs still in flight after an
+// abort) always use this one, so that nothing lands in shared memory or TMEM
+// after the block has released it.
 constexpr long long kWaitCycles = 1000000000LL;
 
 MOE_DEV void set_error(int32_t* err, int32_t code) {
@@ -97,15 +101,16 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait for the phase with the given parity to complete.  Returns false
-// (and records DEV_TIMEOUT, and raises *abort) if it did not within kWaitCycles
-// or if another role already raised *abort.
-MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort) {
+// (and records DEV_TIMEOUT, and raises *abort) if it did not within `limit`
+// clock cycles or if another role already raised *abort.
+MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort,
+                       long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       set_error(err, DEV_TIMEOUT);
       *abort = 1;
       return false;

@@ -85,6 +85,7 @@ struct TcParams {
   TcProblem prob[2];
   int n_prob;
   int32_t* err;
+  long long wait_cycles;      // limit of every pipeline wait (clock cycles)
   // Split-K for swapped tiles (nullptr: off).  When the output tiles fill at most
   // half of the grid, each is split along K into S <= kMaxSplit parts.  Each part
   // stores its FP32 accumulators to split_part, and the last part of an output tile
@@ -464,7 +465,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
           decode_work(p, prefix, BN, TN, S, tile, ti);
           const TcProblem& P = p.prob[ti.prob];
           for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-            if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
             issue_stage(tiles + stage * C::STAGE_BYTES, stage, phase, ti, P, kb, false);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
           }
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
         }
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           int okw = 1;
-          if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag) ? 1 : 0;
+          if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1, p.err, abort_flag, p.wait_cycles) ? 1 : 0;
           if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
           uint8_t* st = tiles + stage * C::STAGE_BYTES;
           if (lane == 0) issue_stage(st, stage, phase, ti, P, kb, gather);
@@ -514,13 +515,13 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
-        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag)) break;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
           if (WQ != WQ_BF16 &&
-              !mbar_wait(&deq_bar[aslot], aphase, p.err, abort_flag)) { ok = false; break; }
+              !mbar_wait(&deq_bar[aslot], aphase, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
           tc_fence_after();
           const uint32_t st_addr = smem_u32(tiles + stage * C::STAGE_BYTES);
           const uint32_t a_addr =
@@ -575,8 +576,8 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&aempty_bar[aslot], aphase ^ 1, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
+          if (!mbar_wait(&aempty_bar[aslot], aphase ^ 1, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
           uint8_t* st = tiles + stage * C::STAGE_BYTES;
           uint8_t* dst = aslots + aslot * C::A_SLOT_BYTES;
           const uint8_t* raw = st + C::RAW_OFF;
@@ -621,7 +622,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
             r = (int)(ti.out_seg + m);
           }
         }
-        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag)) break;
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
         // GATEUP: 128 features, gate in columns [0,128), up in [128,256); each half
         // of the warps takes 64 features.  DOWN: TILE_N features, half each.
@@ -713,7 +714,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
           s_scale[m] = sc;
         }
         __syncwarp();
-        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag)) break;
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
         const int n = ti.n0 + q * 32 + lane;
         const bool n_ok = n < P.n_valid;

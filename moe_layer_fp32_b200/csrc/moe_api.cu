@@ -116,6 +116,7 @@ moe_status validate(const moe_config* c) {
   if (c->router_dtype != c->act_dtype) return MOE_ERR_UNSUPPORTED;
   if (c->bias_mode < MOE_BIAS_NONE || c->bias_mode > MOE_BIAS_SELECT) return MOE_ERR_INVALID;
   if (!(c->rms_eps >= 0.f) || !std::isfinite(c->capacity_factor)) return MOE_ERR_INVALID;
+  if (c->wait_kcycles < 0) return MOE_ERR_INVALID;
   switch (c->expert_dtype) {
     case MOE_F32:
       if (c->act_dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
@@ -338,6 +339,11 @@ moe_status launch_tc_bn(int bn, int wq, const TcParams& p, cudaStream_t st) {
 }
 
 
+// limit of the pipeline waits inside the tensor-core kernels, in clock cycles
+long long wait_cycles(const moe_config* c) {
+  return c->wait_kcycles > 0 ? (long long)c->wait_kcycles * 1024 : kWaitCycles;
+}
+
 int capacity_rows(const moe_config* c) {
   if (!(c->capacity_factor > 0.f)) return INT_MAX;
   double v = std::ceil((double)c->capacity_factor * c->T * c->k / c->E);
@@ -395,6 +401,7 @@ moe_status run_router(const moe_config* c, const moe_weights* w, const void* xn,
     P.n_valid = c->E;
     p.n_prob = 1;
     p.err = err;
+    p.wait_cycles = wait_cycles(c);
     p.k_splits = ns;
     p.split_out_stride = (size_t)c->T * c->E;
     if (!map_rows(&P.tmB, xn, c->T, c->d, 128)) return MOE_ERR_CUDA;
@@ -672,6 +679,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
       p.n_prob = 2;
     }
     p.err = err;
+    p.wait_cycles = wait_cycles(c);
     p.split_part = split_part;
     p.split_cnt = split_cnt;
     s = launch_tc_bn<EPI_GATEUP>(bn, wq, p, st);
@@ -725,6 +733,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
       p.n_prob = 2;
     }
     p.err = err;
+    p.wait_cycles = wait_cycles(c);
     p.split_part = split_part;
     p.split_cnt = split_cnt;
     s = launch_tc_bn<EPI_DOWN>(bn, wq, p, st);

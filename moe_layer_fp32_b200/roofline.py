@@ -86,6 +86,26 @@ def ridge_batch(ridge_flop_per_byte: float, E: int, k: int) -> float:
 # --------------------------------------------------------------- peaks
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# a timed loop at least this long runs into the power cap: the sustained peak
+# applies; a shorter one is a burst
+SUSTAINED_AFTER_S = 2.0
+
+
+def tensor_peak(peaks: dict, timed_loop_s: float, sm_mhz=None) -> tuple:
+    """(bf16 TFLOP/s, label) that applies to a kernel timed inside a loop of
+    ``timed_loop_s`` seconds: the burst figure (a cuBLAS GEMM timed alone) for a
+    short loop, the sustained one (the same GEMM back to back for seconds, under
+    the power cap) for a loop of SUSTAINED_AFTER_S or more."""
+    src = peaks.get("source", "measured")
+    clk = f", median SM clock {sm_mhz:.0f} MHz" if sm_mhz else ""
+    if timed_loop_s >= SUSTAINED_AFTER_S and "bf16_tflops_sustained" in peaks:
+        return (float(peaks["bf16_tflops_sustained"]),
+                f"{src} bf16_tflops_sustained: the timed loop ran {timed_loop_s * 1e3:.0f} ms "
+                f"(>= {SUSTAINED_AFTER_S:.0f} s, power-capped regime{clk})")
+    return (float(peaks["bf16_tflops"]),
+            f"{src} bf16_tflops (burst): the timed loop ran {timed_loop_s * 1e3:.0f} ms "
+            f"(< {SUSTAINED_AFTER_S:.0f} s{clk})")
+
 
 def measured_peaks(path: Optional[str] = None) -> dict:
     """Peaks measured on this kind of GPU (MEASURED_PEAKS.json at the repository

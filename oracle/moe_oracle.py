@@ -11,10 +11,12 @@ round-to-nearest-even.
 
 Sources (page title, then section):
 
-* "MoE: dynamism the compiler cannot remove", the natural implementation
-  listing: router logits -> top-k indices -> a loop over experts that selects the
-  tokens routed to each expert, runs the expert and adds its output back.  The
-  oracle's ``moe_layer`` keeps that per-expert loop structure.
+* "MoE: dynamism the compiler cannot remove", natural implementation: the
+  router's logits give each token its top-k experts and weights, each selected
+  expert's output for the token is weighted by its gate and added to the
+  token's output row.  ``moe_layer`` evaluates exactly that definition: every
+  kept assignment (t, j) contributes ``g[t, j] * FFN_{idx[t, j]}(xn[t])`` to row
+  t, summed in j order after the residual and the shared experts.
 * same page, capacity section: each expert holds at most ``C * T*k/E`` tokens;
   overflow tokens skip the FFN and pass through on the residual.
 * picx.dev summary of the moe-ceilings study, Sub-study 1 (FusedSoftmax):
@@ -266,8 +268,9 @@ def expert_ffn(X, wg, wu, wd) -> np.ndarray:
 # the whole layer
 # ---------------------------------------------------------------------------
 class Weights:
-    """Expert weights (stacked per expert); each matrix is converted to float64
-    (dequantised for int8 / int4) when it is used."""
+    """Expert weights (stacked per expert, numpy arrays or host torch tensors);
+    each matrix is converted to float64 (dequantised for int8 / int4) when it is
+    used, one expert at a time."""
 
     def __init__(self, expert_dtype: str, group: int, gate, up, down,
                  s_gate=None, s_up=None, s_down=None):
@@ -276,7 +279,7 @@ class Weights:
 
     def get(self, which: str, e: int) -> np.ndarray:
         w, s = self.src[which]
-        return expert_matrix(w[e], None if s is None else s[e], self.dt, self.group)
+        return expert_matrix(_npy(w[e]), None if s is None else _npy(s[e]), self.dt, self.group)
 
     def ffn(self, e: int, X) -> np.ndarray:
         return expert_ffn(X, self.get("gate", e), self.get("up", e), self.get("down", e))
@@ -308,17 +311,19 @@ def moe_layer(x, gamma, w_router, router_bias, experts: Weights, *, k: int,
     where[rows] = np.arange(rows.size)
     out = x64[rows].copy() if residual else np.zeros((rows.size, d))
 
-    slot_of = p["slot_of"].reshape(T, k)
-    for e in range(E):                                   # per-expert loop
-        t_sel, j_sel = np.nonzero((r["idx"] == e) & (slot_of >= 0))
-        keep = where[t_sel] >= 0
-        t_sel, j_sel = t_sel[keep], j_sel[keep]
-        if t_sel.size == 0:
-            continue
-        y = experts.ffn(e, xn[t_sel])
-        out[where[t_sel]] += r["gates"][t_sel, j_sel][:, None] * y
-    for s in range(n_shared):                            # always-on experts
+    # y[t, j] = FFN_{idx[t, j]}(xn[t]) for every kept assignment of the evaluated
+    # rows; each row's FFN is independent of the others, so the rows that share an
+    # expert are evaluated together (one matmul per weight matrix)
+    kept = (p["slot_of"].reshape(T, k) >= 0) & (where[:, None] >= 0)
+    y = np.zeros((rows.size, k, d))
+    for e in np.unique(r["idx"][kept]):
+        t_sel, j_sel = np.nonzero(kept & (r["idx"] == e))
+        y[where[t_sel], j_sel] = experts.ffn(int(e), xn[t_sel])
+    for s in range(n_shared):                            # always-on experts, gate 1
         out += shared.ffn(s, xn[rows])
+    g = np.where(kept[rows], r["gates"][rows], 0.0)
+    for j in range(k):                                   # routed outputs in j order
+        out += g[:, j, None] * y[:, j]
     return dict(out=out, xn=xn, logits=logits, logits32=logits32, **r, **p)
 
 
@@ -352,8 +357,10 @@ def moe_layer_dense(x, gamma, w_router, router_bias, experts: Weights, *, k: int
 
 
 def _npy(t):
-    if t is None:
-        return None
+    """numpy view of a host tensor (floating types widened to float32, which is
+    exact for bf16); numpy arrays pass through."""
+    if t is None or isinstance(t, np.ndarray):
+        return t
     return t.float().numpy() if t.is_floating_point() else t.numpy()
 
 
@@ -364,7 +371,7 @@ def weights_from_inputs(li, shared: bool = False) -> Optional[Weights]:
     if shared and not sh.n_shared:
         return None
     pre = "sh_" if shared else ""
-    get = lambda n: _npy(getattr(li, pre + n))   # noqa: E731
+    get = lambda n: getattr(li, pre + n)   # noqa: E731  (converted per expert when used)
     return Weights(sh.expert, sh.group_size, get("w_gate" if not shared else "gate"),
                    get("w_up" if not shared else "up"), get("w_down" if not shared else "down"),
                    get("s_gate"), get("s_up"), get("s_down"))

@@ -21,6 +21,7 @@ import torch
 
 import moe_layer_fp32_b200 as M
 import moe_synth
+from moe_layer_fp32_b200.drift import route_drift
 from oracle import moe_oracle as O
 
 ROUTE_MARGIN = 1e-4
@@ -45,6 +46,7 @@ class LayerResult:
     err_ratio: float           # max|out - ref| / RMS(ref) on the compared rows
     err_ratio_delta: float     # max|out - ref| / RMS(ref - x)
     rows: np.ndarray
+    drift: dict                # swaps per token and Jaccard against the oracle's routes
 
 
 def route_mismatches(gpu_idx, oracle_idx):
@@ -79,7 +81,8 @@ def run_layer(shape, T, tokens: Optional[Sequence[int]] = None, x_stream=None,
     rms_d = float(np.sqrt(np.mean(delta ** 2)))
     rms_o = float(np.sqrt(np.mean(rep["out"] ** 2)))
     err = float(np.max(np.abs(out[rows] - rep["out"])))
-    return LayerResult(out, gl, gi, gc, int(mism.size), mmax, err / rms_o, err / rms_d, rows)
+    return LayerResult(out, gl, gi, gc, int(mism.size), mmax, err / rms_o, err / rms_d, rows,
+                       route_drift(gi, own["idx"]))
 
 
 def sample_rows(T, n=48, seed=0):

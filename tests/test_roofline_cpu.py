@@ -55,3 +55,11 @@ def test_int4_bytes_include_scales():
 def test_peaks_fallback(tmp_path):
     p = R.measured_peaks(str(tmp_path / "missing.json"))
     assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0
+
+
+def test_tensor_peak_follows_the_timed_loop_length():
+    peaks = {"bf16_tflops": 1610.9, "bf16_tflops_sustained": 1393.5, "source": "measured"}
+    v, label = R.tensor_peak(peaks, 0.2, 1965.0)
+    assert v == 1610.9 and "burst" in label and "200 ms" in label
+    v, label = R.tensor_peak(peaks, 5.0)
+    assert v == 1393.5 and "sustained" in label

@@ -69,3 +69,35 @@ def test_static_permute_rejects_batches_beyond_its_scratch():
     with pytest.raises(M.MoeError) as ei:
         M.moe_permute_static(cfg, dummy, dummy, dummy, dummy, dummy, dummy)
     assert ei.value.status == M.MOE_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("T,k,E", [(40, 6, 64), (9440, 8, 256)])
+def test_static_permute_drops_out_of_range_ids_like_moe_permute(T, k, E):
+    """Expert ids outside [0, E) are dropped (slot -1) by both entry points; the
+    static one has no workspace for the error word, so it reports nothing and
+    returns MOE_OK.  T*k = 240 takes the one-CTA kernel, 75520 the three-kernel
+    path."""
+    cfg = M.make_config(LayerShape("p", d=256, E=E, k=k, f=256, capacity_factor=1.25), T)
+    idx_h = skewed_routes(T, k, E, 99)
+    bad = np.zeros(T * k, bool)
+    flat = idx_h.reshape(-1)
+    r = np.random.default_rng(3)
+    for a in r.choice(T * k, 12, replace=False):
+        flat[a] = -1 if a % 2 else E
+        bad[a] = True
+    idx = torch.as_tensor(idx_h).cuda()
+    ref = outputs(T, k, E, -5)
+    ws = M.alloc_workspace(cfg)
+    M.moe_permute(cfg, idx, *ref[:4], ref[4], ws)
+    assert M.moe_get_device_status(ws) == 1          # the workspace entry point reports
+    got = outputs(T, k, E, 7)
+    M.moe_permute_static(cfg, idx, *got)             # raises unless MOE_OK
+    torch.cuda.synchronize()
+    slot = got[3].cpu().numpy()
+    assert np.all(slot[bad] == -1)
+    assert int(got[0].sum().item()) == T * k - int(bad.sum())
+    kept = int(ref[1][E].item())
+    for name, a, b in zip(("counts", "offsets", "perm_assign", "slot_of", "n_dropped"), ref, got):
+        if name == "perm_assign":
+            a, b = a[:kept], b[:kept]
+        assert torch.equal(a, b), name
