@@ -62,7 +62,8 @@ def parse_args():
 def workload_name(sh, T):
     names = {"olmoe": "OLMoE-1B-7B-shaped", "v2lite": "DeepSeek-V2-Lite-shaped",
              "qwen3_int4": "Qwen3-30B-A3B-shaped (int4 experts)",
-             "qwen3_int8": "Qwen3-30B-A3B-shaped (int8 experts)", "v3": "DeepSeek-V3-shaped",
+             "qwen3_int8": "Qwen3-30B-A3B-shaped (int8 experts)",
+             "qwen3_fp8": "Qwen3-30B-A3B-shaped (fp8 experts)", "v3": "DeepSeek-V3-shaped",
              "tiny": "Tiny"}
     kind = "decode" if T <= 64 else "prefill"
     return f"{names.get(sh.name, sh.name)} MoE layer forward, {kind} T={T}"
@@ -408,7 +409,8 @@ def time_layer(M, layer, x, n):
 
 SWEEP = [("olmoe", 1), ("olmoe", 16), ("olmoe", 64), ("olmoe", 4096), ("v2lite", 32),
          ("v2lite", 8192), ("qwen3_int4", 1), ("qwen3_int4", 64), ("qwen3_int4", 16384),
-         ("qwen3_int8", 1), ("qwen3_int8", 64), ("qwen3_int8", 16384), ("v3", 32), ("v3", 256),
+         ("qwen3_int8", 1), ("qwen3_int8", 64), ("qwen3_int8", 16384), ("qwen3_fp8", 1),
+         ("qwen3_fp8", 64), ("qwen3_fp8", 16384), ("v3", 32), ("v3", 256),
          ("v3", 9440), ("tiny", 64)]
 
 

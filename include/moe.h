@@ -66,7 +66,9 @@ typedef enum {
   MOE_ERR_DEVICE = 5        /* the device error word is set (moe_get_device_status)  */
 } moe_status;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_INT8 = 2, MOE_INT4 = 3 } moe_dtype;
+/* MOE_FP8: FP8 E4M3 expert weights (weight-only, like MOE_INT8) -- "MoE at the
+ * inference level ...", Workarounds: int4 / fp8 expert weights to halve the bytes. */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_INT8 = 2, MOE_INT4 = 3, MOE_FP8 = 4 } moe_dtype;
 
 /* Per-expert router bias ("MoE Research", section 2):
  *   NONE   : no bias.
@@ -95,7 +97,8 @@ typedef struct moe_config {
   int32_t out_dtype;       /* out: MOE_BF16 or MOE_F32 (MOE_F32 when act_dtype is F32);
                               the combine sums in FP32 and rounds once to this type    */
   int32_t router_dtype;    /* W_r: MOE_BF16 or MOE_F32 (must equal act_dtype)           */
-  int32_t expert_dtype;    /* MOE_F32 (requires act F32) | MOE_BF16 | MOE_INT8 | MOE_INT4 */
+  int32_t expert_dtype;    /* MOE_F32 (requires act F32) | MOE_BF16 | MOE_INT8 | MOE_INT4
+                              | MOE_FP8                                                 */
   int32_t group_size;      /* int4: scale group along K; must be 128                    */
   int32_t wait_kcycles;    /* limit of every pipeline wait inside the kernels, in units of
                               1024 SM clock cycles; 0 = the default, 10^9 cycles (about
@@ -107,15 +110,18 @@ typedef struct moe_config {
  *   rms_gamma   [d] float32
  *   w_router    [d, E]            router dtype
  *   router_bias [E] float32, or NULL (required unless bias_mode == NONE)
- *   w_gate/w_up [E, d, f]         F32/BF16: that type; INT8: int8; INT4: uint8 [E, d, f/2]
- *   w_down      [E, f, d]         F32/BF16: that type; INT8: int8; INT4: uint8 [E, f, d/2]
- *   s_gate/s_up INT8: bf16 [E, f]; INT4: bf16 [E, d/128, f]; otherwise NULL
- *   s_down      INT8: bf16 [E, d]; INT4: bf16 [E, f/128, d]; otherwise NULL
+ *   w_gate/w_up [E, d, f]         F32/BF16: that type; INT8: int8; FP8: uint8 E4M3 codes;
+ *                                 INT4: uint8 [E, d, f/2]
+ *   w_down      [E, f, d]         the same; INT4: uint8 [E, f, d/2]
+ *   s_gate/s_up INT8, FP8: bf16 [E, f]; INT4: bf16 [E, d/128, f]; otherwise NULL
+ *   s_down      INT8, FP8: bf16 [E, d]; INT4: bf16 [E, f/128, d]; otherwise NULL
  *   sh_*        the same for the n_shared shared experts ([S, ...]); NULL if S == 0
  * int8 weights are symmetric with one scale per output column; int4 weights are
  * symmetric signed 4-bit, two per byte along the contiguous dim (low nibble =
- * even column), with one scale per 128 rows of K and output column.  Either way
- * the weight the layer uses is bf16(q * s): the exact product rounded once. */
+ * even column), with one scale per 128 rows of K and output column; fp8 weights
+ * are E4M3 codes (no infinities, largest finite 448) with one scale per output
+ * column.  In every case the weight the layer uses is bf16(q * s): the exact
+ * product rounded once. */
 typedef struct moe_weights {
   const void* rms_gamma;
   const void* w_router;

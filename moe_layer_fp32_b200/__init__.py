@@ -17,10 +17,11 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
-MOE_F32, MOE_BF16, MOE_INT8, MOE_INT4 = range(4)
+MOE_F32, MOE_BF16, MOE_INT8, MOE_INT4, MOE_FP8 = range(5)
 MOE_BIAS_NONE, MOE_BIAS_LOGIT, MOE_BIAS_SELECT = range(3)
 
-DTYPE_CODE = {"f32": MOE_F32, "bf16": MOE_BF16, "int8": MOE_INT8, "int4": MOE_INT4}
+DTYPE_CODE = {"f32": MOE_F32, "bf16": MOE_BF16, "int8": MOE_INT8, "int4": MOE_INT4,
+              "fp8": MOE_FP8}
 BIAS_CODE = {"none": MOE_BIAS_NONE, "logit": MOE_BIAS_LOGIT, "select": MOE_BIAS_SELECT}
 
 

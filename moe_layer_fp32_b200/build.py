@@ -29,12 +29,14 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, defines=()) -> str:
+    """Compile the library; ``defines`` are extra NAME=VALUE build options (for
+    example MOE_PAIR_TILES=0 selects the single-CTA prefill GEMM)."""
+    if not force and not defines and up_to_date():
         return OUT
     nvcc = os.environ.get("NVCC", "nvcc")
     cmd = [nvcc, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-cudart", "static", SRC, "-o", OUT + ".tmp"]
+           "-cudart", "static", *[f"-D{d}" for d in defines], SRC, "-o", OUT + ".tmp"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -48,4 +50,5 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    defs = [a[len("--define="):] for a in sys.argv if a.startswith("--define=")]
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, defines=defs))

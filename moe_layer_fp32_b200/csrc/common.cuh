@@ -5,6 +5,7 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #define MOE_DEV __device__ __forceinline__
@@ -48,6 +49,16 @@ MOE_DEV __nv_bfloat16 bf16_from_double(double v) {
     return __float2bfloat16_rn((float)q);
   }
   return __float2bfloat16_rn((float)v);      // overflow / inf / nan
+}
+
+// Two FP8 E4M3 codes (the low byte is the first) to their exact values.  Every
+// E4M3 value, subnormals included, is an f16 value, so the hardware e4m3x2 ->
+// f16x2 conversion is exact, and so is the widening to f32.
+MOE_DEV float2 e4m3x2_to_float2(uint32_t two_codes) {
+  uint32_t h;
+  const uint16_t v = (uint16_t)(two_codes & 0xffffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 // ---------------------------------------------------------------------------
@@ -94,6 +105,19 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// try_wait with cluster-scope acquire: for barriers that the peer CTA of a pair
+// arrives on (its arrivals are cluster-scope releases)
+MOE_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.b32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -208,6 +232,70 @@ MOE_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 MOE_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs sharing one tcgen05 MMA: cta_group::2).  The
+// MMA of a pair is issued by the even CTA; it reads the A rows and the half of B
+// that each CTA holds at the same shared-memory offsets, and writes each CTA's
+// accumulator rows into that CTA's TMEM.  No TMA multicast is used: each CTA
+// loads its own operands.
+// ---------------------------------------------------------------------------
+MOE_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// all threads of both CTAs (arrive with release, wait with acquire semantics)
+MOE_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// shared::cluster address of the same shared-memory location in CTA `rank`
+MOE_DEV uint32_t mapa_shared(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// arrive on an mbarrier of another CTA of the cluster (cluster-scope release)
+MOE_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+MOE_DEV void st_shared_remote_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+MOE_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {   // one warp in each CTA
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+MOE_DEV void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+MOE_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {   // one warp in each CTA
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// the pair's MMA: D(tmem, both CTAs) (+)= A(smem, 128 rows per CTA) * B(smem, half of
+// N per CTA); issued by one thread of the even CTA
+MOE_DEV void tc2_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive once on the mbarrier at shared::cluster address `cluster_addr` (this CTA's
+// or the peer's) when the pair MMAs issued so far by this thread have completed
+MOE_DEV void tc2_commit(uint32_t cluster_addr) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          cluster_addr)
+      : "memory");
+}
 
 // Shared-memory matrix descriptor for tcgen05.mma with the 128-byte swizzle.
 //   start address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30),

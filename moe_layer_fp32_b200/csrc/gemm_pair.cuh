@@ -1,0 +1,302 @@
+// Grouped expert GEMM on CTA pairs (tcgen05 cta_group::2) for prefill tiles.
+//
+// "MoE: dynamism the compiler cannot remove", grouped GEMM section: one launch over
+// all experts' rows, each block finding its expert from the per-expert offsets.
+// Here a cluster of two CTAs takes a tile of 256 tokens of one expert: the even
+// CTA holds token rows m0 .. m0+127, the odd CTA rows m0+128 .. m0+255, and one
+// MMA of M = 256 tokens x N = 256 columns covers both.  Each CTA stages its own
+// 128 token rows and HALF of the 256 weight columns:
+//   GATEUP: the even CTA stages 128 features of W_gate, the odd CTA the same 128
+//           features of W_up, so every CTA's accumulator holds [gate | up] for its
+//           rows and the SwiGLU stays local;
+//   DOWN:   the even CTA stages output features n0 .. n0+127, the odd n0+128 ..
+//           n0+255.
+// Per 64-deep k-block an SM then moves 32 KB into shared memory and the MMA reads
+// 32 KB of it for 128 x 256 x 64 multiply-adds; the single-CTA kernel moves and
+// reads 48 KB for the same work.  Shared-memory bandwidth is what bounds the
+// single-CTA kernel, so this cuts the staged bytes per flop by a third.
+//
+// Synchronisation (no TMA multicast: every CTA loads only into its own memory and
+// signals only its own barrier, so each CTA always knows when its copies landed):
+//   full[s]   (each CTA) its producer's TMA bytes of stage s;
+//   pfull[s]  (even CTA) one arrival forwarded by the odd CTA once ITS stage s
+//             landed;  the even CTA's MMA thread waits on both;
+//   empty[s]  (each CTA) stage s consumed: the MMA thread commits to both CTAs;
+//   tfull[a]  (each CTA) accumulator a complete: commits to both CTAs;
+//   tempty[a] (even CTA) accumulator a drained: 8 epilogue warps of each CTA.
+// Every wait is bounded; a CTA that gives up raises its own and its peer's abort
+// flag, drains its own copies (and, on the even CTA, the issued MMAs), and both
+// meet at a final cluster barrier before the TMEM is released.
+#pragma once
+#include "gemm_tc.cuh"
+
+namespace moe {
+
+template <int EPI>
+struct PairConfig {
+  static constexpr int BN = 256;                                   // tokens per pair tile
+  static constexpr int TILE_N = EPI == EPI_GATEUP ? 128 : 256;     // features per tile
+  static constexpr uint32_t B_HALF = 128 * 64 * 2;   // 128 weight columns x 64 k
+  static constexpr uint32_t A_BYTES = 128 * 64 * 2;  // 128 token rows x 64 k
+  static constexpr uint32_t STAGE_BYTES = B_HALF + A_BYTES;
+  static constexpr uint32_t TOKEN_OFF = B_HALF;
+  static constexpr int STAGES = 6;
+  static constexpr uint32_t ACC_COLS = 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // A = tokens (K-major), B = weights (MN-major); M = 256 tokens, N = 256 columns
+  static constexpr uint32_t IDESC = idesc_bf16(256, 256, false, true);
+  static constexpr int THREADS = kTcBaseThreads;
+  static constexpr uint32_t BAR_BYTES = 8 * (3 * STAGES + 5) + 16 + 4 * STAGES;
+  static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
+  static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 20 * 4;
+  static constexpr uint32_t SMEM_BYTES =
+      1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+  static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 128-byte swizzle alignment");
+};
+
+// Bounded wait of a pair kernel: on time-out it also raises the peer's abort flag.
+MOE_DEV bool pair_wait(uint64_t* bar, uint32_t parity, const TcParams& p, volatile int* abort,
+                       uint32_t peer_abort) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > p.wait_cycles) {
+      set_error(p.err, DEV_TIMEOUT);
+      *abort = 1;
+      st_shared_remote_u32(peer_abort, 1);
+      return false;
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
+    k_tc_gemm_pair(const __grid_constant__ TcParams p) {
+  using C = PairConfig<EPI>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int BN = C::BN;
+  constexpr int TN = C::TILE_N;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
+  uint64_t* pfull_bar = full_bar + STAGES;
+  uint64_t* empty_bar = pfull_bar + STAGES;
+  uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
+  uint64_t* tempty_bar = tfull_bar + 2;       // [2]
+  uint64_t* drain_bar = tempty_bar + 2;       // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* issued = const_cast<int*>(abort_flag) + 2;   // [STAGES] last issued parity + 1
+  int* prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
+  float* stg_all = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(prefix + 2 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();   // 0: the CTA that issues the pair's MMAs
+  const uint32_t peer = rank ^ 1u;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&pfull_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      issued[s] = 0;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 2 * kEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int pi = 0; pi < p.n_prob; ++pi) {
+      tma_prefetch_desc(&p.prob[pi].tmA);
+      if (EPI == EPI_GATEUP) tma_prefetch_desc(&p.prob[pi].tmA2);
+      tma_prefetch_desc(&p.prob[pi].tmB);
+    }
+  }
+  // both CTAs' barriers are initialised (and the TMEM allocated) before either
+  // CTA signals the other
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t peer_abort = mapa_shared(const_cast<int*>(abort_flag), peer);
+  pdl_wait();
+  pdl_trigger();
+  if (warp >= 2 && warp - 2 < p.n_prob) {
+    const TcProblem& P = p.prob[warp - 2];
+    group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = total_tiles(p, prefix, TN);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, TN, tile, ti);
+        const TcProblem& P = p.prob[ti.prob];
+        // this CTA's half of the weight columns: GATEUP gate (even) / up (odd) at the
+        // tile's features; DOWN features n0 + 128 * rank
+        const void* wmap = (EPI == EPI_GATEUP && rank == 1) ? (const void*)&P.tmA2
+                                                             : (const void*)&P.tmA;
+        const int wn = (EPI == EPI_GATEUP) ? ti.n0 : ti.n0 + 128 * (int)rank;
+        const int brow = ti.b_row + 128 * (int)rank;
+        const int kbl = P.K / 64;
+        for (int kb = 0; kb < kbl; ++kb) {
+          if (!pair_wait(&empty_bar[stage], phase ^ 1, p, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = tiles + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          issued[stage] = (int)phase + 1;
+          tma_load_3d(st, wmap, &full_bar[stage], wn, kb * 64, ti.g);
+          tma_load_3d(st + 8192, wmap, &full_bar[stage], wn + 64, kb * 64, ti.g);
+          tma_load_2d(st + C::TOKEN_OFF, &P.tmB, &full_bar[stage], kb * 64, brow);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // -------------------------------------------------- MMA issuer (even CTA)
+      const uint32_t empty_peer = mapa_shared(empty_bar, peer);
+      const uint32_t tfull_peer = mapa_shared(tfull_bar, peer);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, TN, tile, ti);
+        const int kbl = p.prob[ti.prob].K / 64;
+        if (!pair_wait(&tempty_bar[acc], acc_phase ^ 1, p, abort_flag, peer_abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < kbl; ++kb) {
+          if (!pair_wait(&full_bar[stage], phase, p, abort_flag, peer_abort) ||
+              !pair_wait(&pfull_bar[stage], phase, p, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st_addr = smem_u32(tiles + stage * C::STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // tokens: K-major SW128, 16 k = 32 B per step, 8-row groups 1 KB apart;
+            // weights: MN-major SW128, 16 k-rows of 128 B per step, the two
+            // 64-column halves 8 KB apart, 8-row groups 1 KB apart
+            const uint64_t ad = sw128_desc(st_addr + C::TOKEN_OFF + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
+            tc2_mma_f16(d_tmem, ad, bd, C::IDESC, (kb != 0 || kk != 0) ? 1u : 0u);
+          }
+          // stage s of both CTAs is free once these MMAs have read it
+          tc2_commit(smem_u32(&empty_bar[stage]));
+          tc2_commit(empty_peer + stage * 8);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc2_commit(smem_u32(&tfull_bar[acc]));
+        tc2_commit(tfull_peer + acc * 8);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // every MMA issued above completes before TMEM or the peer's memory is released
+      tc2_commit(smem_u32(drain_bar));
+      const long long t0 = clock64();
+      while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kWaitCycles) {}
+    } else if (lane == 0) {
+      // ------------------------------------- forwarder (odd CTA): stage s landed here
+      const uint32_t pfull_peer = mapa_shared(pfull_bar, peer);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, TN, tile, ti);
+        const int kbl = p.prob[ti.prob].K / 64;
+        for (int kb = 0; kb < kbl; ++kb) {
+          if (!pair_wait(&full_bar[stage], phase, p, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_remote(pfull_peer + stage * 8);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int half = (warp - 2) >> 2;       // which half of the columns it drains
+    float* stg = stg_all + (warp - 2) * (32 * 20);
+    const uint32_t tempty_even = mapa_shared(tempty_bar, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      TileInfo ti;
+      decode_tile(p, prefix, BN, TN, tile, ti);
+      const TcProblem& P = p.prob[ti.prob];
+      const uint32_t t_base = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS;
+      int r;
+      float sc;
+      direct_row<EPI>(P, ti, 128 * (int)rank + q * 32 + lane, r, sc);
+      if (!pair_wait(&tfull_bar[acc], acc_phase, p, abort_flag, peer_abort)) break;
+      tc_fence_after();
+      direct_store<EPI, TN>(P, ti, r, sc, t_base, half, lane, stg);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(tempty_even + acc * 8);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // this CTA's copies still in flight after an abort: wait (bounded) for each
+    // stage's last load
+    for (int s = 0; s < STAGES; ++s) {
+      if (issued[s]) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&full_bar[s], (uint32_t)(issued[s] - 1)) &&
+               clock64() - t0 < kWaitCycles) {}
+      }
+    }
+  }
+  // neither CTA leaves while the pair's MMAs may still read its memory or write its
+  // TMEM (the even CTA drained them above)
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace moe

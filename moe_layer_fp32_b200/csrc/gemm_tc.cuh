@@ -41,16 +41,19 @@
 namespace moe {
 
 enum Epi : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_ROUTER = 2 };
-// weight storage: bf16, or weight-only int8 / int4 dequantised to bf16(q * s) in
-// the main loop
-enum WQuant : int { WQ_BF16 = 0, WQ_INT8 = 1, WQ_INT4 = 2 };
+// weight storage: bf16, or weight-only int8 / int4 / fp8 (E4M3) dequantised to
+// bf16(q * s) in the main loop; int8 and fp8 share one layout (a byte per weight,
+// a bf16 scale per output column)
+enum WQuant : int { WQ_BF16 = 0, WQ_INT8 = 1, WQ_INT4 = 2, WQ_FP8 = 3 };
+template <int WQ>
+struct ByteWeights { static constexpr bool value = WQ == WQ_INT8 || WQ == WQ_FP8; };
 
 constexpr int kTcBaseThreads = 320;   // producer, MMA, 8 epilogue warps
 constexpr int kEpiWarps = 8;
 // dequantisation warps for int8 / int4 weights (int4 is bound by shared-memory
 // bandwidth already at 8; int8's longer conversion gains from 16)
 template <int WQ>
-struct DeqWarps { static constexpr int value = WQ == 1 ? 16 : 8; };
+struct DeqWarps { static constexpr int value = ByteWeights<WQ>::value ? 16 : 8; };
 constexpr int kMaxGroups = 512;
 
 struct TcProblem {
@@ -128,8 +131,9 @@ struct TcConfig {
   static constexpr uint32_t A_BYTES = TcShape<EPI, DIRECT>::A_BYTES;
   static constexpr uint32_t B_BYTES = BN * 64 * 2;
   // raw quantised weight block (128 features x 64 k): int8 128 B rows, int4 64 B rows
-  static constexpr uint32_t RAW_BYTES = WQ == WQ_INT8 ? 128 * 64 : WQ == WQ_INT4 ? 64 * 64 : 0;
-  static constexpr uint32_t RAW_ROW = WQ == WQ_INT8 ? 128 : 64;
+  static constexpr uint32_t RAW_BYTES =
+      ByteWeights<WQ>::value ? 128 * 64 : WQ == WQ_INT4 ? 64 * 64 : 0;
+  static constexpr uint32_t RAW_ROW = ByteWeights<WQ>::value ? 128 : 64;
   static constexpr uint32_t SCALE_BYTES = WQ == WQ_BF16 ? 0 : 256;   // 128 bf16 scales
   // bf16 weights: one ring of TMA stages [weights NA x 16 KB | tokens].
   // int8 / int4 weights: a deep ring of TMA stages [tokens | raw weights | scales
@@ -285,7 +289,7 @@ MOE_DEV void int4x8_to_bf16(uint32_t v, const uint32_t (&s2)[4], uint32_t (&o)[4
 // Features at or beyond N were zero-filled by the TMA (q = 0, s = 0).
 template <int WQ, int NTHREADS>
 MOE_DEV void dequant_block(const uint8_t* raw, uint8_t* out, const __nv_bfloat16* ssm, int t) {
-  constexpr int RAW_ROW = WQ == WQ_INT8 ? 128 : 64;
+  constexpr int RAW_ROW = WQ == WQ_INT4 ? 64 : 128;
   constexpr int ITERS = 64 * 16 / NTHREADS;
   static_assert(64 * 16 % NTHREADS == 0, "whole chunks per thread");
   // the column chunk of thread t is the same in every iteration (16 | NTHREADS):
@@ -314,8 +318,15 @@ MOE_DEV void dequant_block(const uint8_t* raw, uint8_t* out, const __nv_bfloat16
       for (int i = 0; i < 4; ++i) {
         const uint32_t w = i < 2 ? v.x : v.y;
         const int sh = (i & 1) * 16;
-        const float q0 = (float)(int8_t)((w >> sh) & 0xff);
-        const float q1 = (float)(int8_t)((w >> (sh + 8)) & 0xff);
+        float q0, q1;
+        if (WQ == WQ_FP8) {
+          const float2 q = e4m3x2_to_float2(w >> sh);
+          q0 = q.x;
+          q1 = q.y;
+        } else {
+          q0 = (float)(int8_t)((w >> sh) & 0xff);
+          q1 = (float)(int8_t)((w >> (sh + 8)) & 0xff);
+        }
         __nv_bfloat162 h2 =
             __floats2bfloat162_rn(q0 * __low2float(s2[i]), q1 * __high2float(s2[i]));
         pk[i] = *reinterpret_cast<uint32_t*>(&h2);
@@ -323,6 +334,98 @@ MOE_DEV void dequant_block(const uint8_t* raw, uint8_t* out, const __nv_bfloat16
     }
     *reinterpret_cast<uint4*>(out + (c >> 3) * 8192 + k * 128 + (((c & 7) ^ (k & 7)) << 4)) =
         make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// Direct orientation (tokens on the MMA's M side): output row and scale of token
+// row m of the tile (r = -1 past the end of the segment).
+template <int EPI>
+MOE_DEV void direct_row(const TcProblem& P, const TileInfo& ti, int m, int& r, float& sc) {
+  r = -1;
+  sc = 1.f;
+  if (m < ti.rows) {
+    if (EPI == EPI_DOWN && P.perm_assign) {
+      r = P.perm_assign[ti.slot0 + m];
+      sc = P.gate[r];
+    } else {
+      r = (int)(ti.out_seg + m);
+    }
+  }
+}
+
+// Direct-orientation epilogue: this thread holds TMEM lane (q*32 + lane) of the
+// accumulator at t_base, i.e. one token row, whose output row is r (-1: none).
+// GATEUP: 128 features, gate in columns [0,128), up in [128,256); each half of the
+// warps takes 64 features and writes bf16 h.  DOWN: TN features, half each, scaled
+// by the gate and stored through the warp's staging tile `stg` (32 rows x 20 floats).
+template <int EPI, int TN>
+MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float sc,
+                          uint32_t t_base, int half, int lane, float* stg) {
+  constexpr int CPH = (EPI == EPI_GATEUP) ? 4 : TN / 32;   // chunks per half
+#pragma unroll 1
+  for (int c = half * CPH; c < half * CPH + CPH; ++c) {
+    const int n = ti.n0 + c * 16;
+    if (n >= P.n_valid) break;
+    float v0[16];
+    tmem_ld16(t_base + c * 16, v0);
+    float v1[16];
+    if (EPI == EPI_GATEUP) tmem_ld16(t_base + 128 + c * 16, v1);
+    tmem_wait_ld();
+    if (r >= 0 && EPI == EPI_GATEUP) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(silu_f(v0[2 * j]) * v1[2 * j],
+                                                  silu_f(v0[2 * j + 1]) * v1[2 * j + 1]);
+        pk[j] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) +
+                                            (size_t)r * P.ld_out + n);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    } else if (EPI != EPI_GATEUP) {
+      // Through a per-warp staging tile: each lane writes its row's 16 scaled values,
+      // then several lanes store one row's contiguous bytes (FP32: 4 lanes x 16 B,
+      // 8 rows per instruction; bf16: 2 lanes x 16 B, 16 rows per instruction), so
+      // every store fills whole 32-byte sectors.
+      float4* srow = reinterpret_cast<float4*>(stg + lane * 20);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        srow[j] = make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
+                              v0[4 * j + 3] * sc);
+      __syncwarp();
+      if (P.out_bf16) {
+        const int hh = (lane & 1) * 8;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int rr = (lane >> 1) + 16 * i;
+          const int rout = __shfl_sync(0xffffffffu, r, rr);
+          const float4 a = *reinterpret_cast<const float4*>(stg + rr * 20 + hh);
+          const float4 b = *reinterpret_cast<const float4*>(stg + rr * 20 + hh + 4);
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(a.z, a.w);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(b.z, b.w);
+          if (rout >= 0)
+            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) +
+                                      (size_t)rout * P.ld_out + n + hh) =
+                make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                           *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+        }
+      } else {
+        const int qq = (lane & 3) * 4;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = (lane >> 2) + 8 * i;
+          const int rout = __shfl_sync(0xffffffffu, r, rr);
+          const float4 v = *reinterpret_cast<const float4*>(stg + rr * 20 + qq);
+          if (rout >= 0)
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + (size_t)rout * P.ld_out +
+                                       n + qq) = v;
+        }
+      }
+      __syncwarp();
+    }
   }
 }
 
@@ -445,11 +548,11 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
         const void* s2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmS2 : (const void*)&P.tmS;
         tma_load_3d(raw, &P.tmA, &full_bar[stage], ti.n0 / div, kb * 64, ti.g);
         // int8: scales [G][N] (second coordinate g, third 0); int4: [G][K/128][N]
-        if (WQ == WQ_INT8) tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, ti.g, 0);
+        if (WQ != WQ_INT4) tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, ti.g, 0);
         else tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, kb / 2, ti.g);
         if (NA == 2) {
           tma_load_3d(raw + C::RAW_BYTES, m2, &full_bar[stage], n2 / div, kb * 64, ti.g);
-          if (WQ == WQ_INT8) tma_load_3d(scl + 256, s2, &full_bar[stage], n2, ti.g, 0);
+          if (WQ != WQ_INT4) tma_load_3d(scl + 256, s2, &full_bar[stage], n2, ti.g, 0);
           else tma_load_3d(scl + 256, s2, &full_bar[stage], n2, kb / 2, ti.g);
         }
       }
@@ -611,90 +714,13 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
       if (DIRECT) {
         // this thread's token row; its output row and gate are fetched before the
         // accumulator wait so that the loads overlap the MMAs
-        const int m = q * 32 + lane;
-        int r = -1;
-        float sc = 1.f;
-        if (m < ti.rows) {
-          if (EPI == EPI_DOWN && P.perm_assign) {
-            r = P.perm_assign[ti.slot0 + m];
-            sc = P.gate[r];
-          } else {
-            r = (int)(ti.out_seg + m);
-          }
-        }
+        int r;
+        float sc;
+        direct_row<EPI>(P, ti, q * 32 + lane, r, sc);
         if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
-        // GATEUP: 128 features, gate in columns [0,128), up in [128,256); each half
-        // of the warps takes 64 features.  DOWN: TILE_N features, half each.
-        constexpr int CPH = (EPI == EPI_GATEUP) ? 4 : TN / 32;   // chunks per half
-#pragma unroll 1
-        for (int c = half * CPH; c < half * CPH + CPH; ++c) {
-          const int n = ti.n0 + c * 16;
-          if (n >= P.n_valid) break;
-          float v0[16];
-          tmem_ld16(t_base + c * 16, v0);
-          float v1[16];
-          if (EPI == EPI_GATEUP) tmem_ld16(t_base + 128 + c * 16, v1);
-          tmem_wait_ld();
-          if (r >= 0 && EPI == EPI_GATEUP) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(silu_f(v0[2 * j]) * v1[2 * j],
-                                                        silu_f(v0[2 * j + 1]) * v1[2 * j + 1]);
-              pk[j] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) +
-                                                  (size_t)r * P.ld_out + n);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          } else if (EPI != EPI_GATEUP) {
-            // Through a per-warp staging tile: each lane writes its row's 16 scaled values,
-            // then several lanes store one row's contiguous bytes (FP32: 4 lanes x 16 B,
-            // 8 rows per instruction; bf16: 2 lanes x 16 B, 16 rows per instruction), so
-            // every store fills whole 32-byte sectors.
-            float* stg = reinterpret_cast<float*>(epi_row) + (warp - 2) * (32 * 20);
-            float4* srow = reinterpret_cast<float4*>(stg + lane * 20);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              srow[j] = make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
-                                    v0[4 * j + 3] * sc);
-            __syncwarp();
-            if (P.out_bf16) {
-              const int hh = (lane & 1) * 8;
-#pragma unroll
-              for (int i = 0; i < 2; ++i) {
-                const int rr = (lane >> 1) + 16 * i;
-                const int rout = __shfl_sync(0xffffffffu, r, rr);
-                const float4 a = *reinterpret_cast<const float4*>(stg + rr * 20 + hh);
-                const float4 b = *reinterpret_cast<const float4*>(stg + rr * 20 + hh + 4);
-                __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y);
-                __nv_bfloat162 h1 = __floats2bfloat162_rn(a.z, a.w);
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y);
-                __nv_bfloat162 h3 = __floats2bfloat162_rn(b.z, b.w);
-                if (rout >= 0)
-                  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) +
-                                            (size_t)rout * P.ld_out + n + hh) =
-                      make_uint4(*reinterpret_cast<uint32_t*>(&h0),
-                                 *reinterpret_cast<uint32_t*>(&h1),
-                                 *reinterpret_cast<uint32_t*>(&h2),
-                                 *reinterpret_cast<uint32_t*>(&h3));
-              }
-            } else {
-              const int qq = (lane & 3) * 4;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int rr = (lane >> 2) + 8 * i;
-                const int rout = __shfl_sync(0xffffffffu, r, rr);
-                const float4 v = *reinterpret_cast<const float4*>(stg + rr * 20 + qq);
-                if (rout >= 0)
-                  *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) +
-                                             (size_t)rout * P.ld_out + n + qq) = v;
-              }
-            }
-            __syncwarp();
-          }
-        }
+        direct_store<EPI, TN>(P, ti, r, sc, t_base, half, lane,
+                              reinterpret_cast<float*>(epi_row) + (warp - 2) * (32 * 20));
       } else {
         // swapped: this thread owns feature n; the tile's token rows and scales are
         // staged in this warp's shared-memory slice (warp-private: __syncwarp only)

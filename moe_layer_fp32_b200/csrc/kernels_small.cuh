@@ -711,14 +711,14 @@ __global__ void __launch_bounds__(256) k_perm_rank(const int32_t* __restrict__ i
 }
 
 // ---------------------------------------------------------------------------
-// Dequantise whole expert matrices to bf16 (prefill batches with int8 / int4
-// experts): w = bf16(q * s), the exact product rounded once, 8 outputs per
+// Dequantise whole expert matrices to bf16 (prefill batches with int8 / int4 /
+// fp8 experts): w = bf16(q * s), the exact product rounded once, 8 outputs per
 // thread per step.  Experts that received no token are skipped when `offsets`
 // is given.  blockIdx.y = matrix, blockIdx.z = expert.
 // ---------------------------------------------------------------------------
 struct DeqMatrix {
-  const uint8_t* q;              // int8 [G][K][N] or packed int4 [G][K][N/2]
-  const __nv_bfloat16* s;        // [G][N] (int8) or [G][K/128][N] (int4)
+  const uint8_t* q;              // int8 / fp8 [G][K][N] or packed int4 [G][K][N/2]
+  const __nv_bfloat16* s;        // [G][N] (int8, fp8) or [G][K/128][N] (int4)
   __nv_bfloat16* out;            // [G][K][N]
   const int32_t* offsets;        // [G+1] routed segments, or nullptr (dequantise all)
   int G, K, N;
@@ -728,8 +728,10 @@ struct DeqArgs {
   int n;
 };
 
-template <bool INT4>
+// KIND: 0 = int8, 1 = int4, 2 = fp8 (E4M3 codes, the int8 layout)
+template <int KIND>
 __global__ void __launch_bounds__(256) k_dequant_experts(const __grid_constant__ DeqArgs a) {
+  constexpr bool INT4 = KIND == 1;
   pdl_wait();
   pdl_trigger();
   // block (x, y, z) = 8 rows of matrix y of expert z; thread (tx, ty) = row ty,
@@ -768,6 +770,14 @@ __global__ void __launch_bounds__(256) k_dequant_experts(const __grid_constant__
       if (INT4) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) q[i] = (float)((int)(v4[u] << (28 - 4 * i)) >> 28);
+      } else if (KIND == 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t w = i < 2 ? v8[u].x : v8[u].y;
+          const float2 f = e4m3x2_to_float2(w >> ((i & 1) * 16));
+          q[2 * i] = f.x;
+          q[2 * i + 1] = f.y;
+        }
       } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "kernels_small.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_pair.cuh"
 
 using namespace moe;
 
@@ -93,9 +94,11 @@ inline int split_counters() { return num_sms() * 8; }
 // in bf16 (half the bytes the down GEMM writes and the combine reads); the
 // grouped-FFN and combine entry points exchange them in FP32.
 inline bool y_bf16(const moe_config* c) { return tc_experts(c); }
-inline bool dequant_once(const moe_config* c) {
-  return (c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4) && pick_bn(c) == 128;
+inline bool quantised(const moe_config* c) {
+  return c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4 ||
+         c->expert_dtype == MOE_FP8;
 }
+inline bool dequant_once(const moe_config* c) { return quantised(c) && pick_bn(c) == 128; }
 
 struct Layout {
   size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, split,
@@ -127,6 +130,7 @@ moe_status validate(const moe_config* c) {
       break;
     case MOE_INT8:
     case MOE_INT4:
+    case MOE_FP8:
       if (c->act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
       if (c->d % 128 || c->f % 128 || c->E % 8) return MOE_ERR_UNSUPPORTED;
       if (c->expert_dtype == MOE_INT4 && c->group_size != 128) return MOE_ERR_UNSUPPORTED;
@@ -286,13 +290,16 @@ bool map_scales(CUtensorMap* m, const moe_config* c, const void* base, int G, in
 
 // expert weight matrix [G][K][N] in the storage the GEMM reads (wq)
 bool map_expert(CUtensorMap* m, int wq, const void* base, int G, int K, int N) {
-  if (wq == WQ_INT8) return map_raw(m, base, G, K, N, 128);
+  if (wq == WQ_INT8 || wq == WQ_FP8) return map_raw(m, base, G, K, N, 128);
   if (wq == WQ_INT4) return map_raw(m, base, G, K, N / 2, 64);
   return map_weights(m, base, G, K, N);
 }
 
 inline int wq_of(const moe_config* c) {
-  return c->expert_dtype == MOE_INT8 ? WQ_INT8 : c->expert_dtype == MOE_INT4 ? WQ_INT4 : WQ_BF16;
+  return c->expert_dtype == MOE_INT8   ? WQ_INT8
+         : c->expert_dtype == MOE_INT4 ? WQ_INT4
+         : c->expert_dtype == MOE_FP8  ? WQ_FP8
+                                       : WQ_BF16;
 }
 
 // activations [R][K] bf16, K contiguous; box 64 k x BN rows
@@ -319,6 +326,25 @@ moe_status launch_tc(const TcParams& p, cudaStream_t st) {
   return check_launch();
 }
 
+// Prefill tiles of bf16 experts run on CTA pairs (256 tokens per tile, one
+// cta_group::2 MMA per k-step) unless the library is built with MOE_PAIR_TILES=0.
+#ifndef MOE_PAIR_TILES
+#define MOE_PAIR_TILES 1
+#endif
+constexpr bool kPairTiles = MOE_PAIR_TILES != 0;
+
+template <int EPI>
+moe_status launch_pair(const TcParams& p, cudaStream_t st) {
+  using C = PairConfig<EPI>;
+  auto kern = k_tc_gemm_pair<EPI>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  // an even number of CTAs: one cluster of two per pair of SMs
+  MOE_LAUNCH((kern), num_sms() / 2 * 2, C::THREADS, C::SMEM_BYTES, st, p);
+  return check_launch();
+}
+
 template <int EPI, int WQ>
 moe_status launch_tc_bn_q(int bn, const TcParams& p, cudaStream_t st) {
   switch (bn) {
@@ -326,8 +352,12 @@ moe_status launch_tc_bn_q(int bn, const TcParams& p, cudaStream_t st) {
     case 32: return launch_tc<EPI, 32, false, WQ>(p, st);
     case 64: return launch_tc<EPI, 64, false, WQ>(p, st);
     default:   // prefill tiles: tokens on MMA-M (quantised weights are dequantised first)
-      if constexpr (WQ == WQ_BF16) return launch_tc<EPI, 128, true, WQ>(p, st);
-      else return MOE_ERR_UNSUPPORTED;
+      if constexpr (WQ == WQ_BF16) {
+        if (kPairTiles) return launch_pair<EPI>(p, st);
+        return launch_tc<EPI, 128, true, WQ>(p, st);
+      } else {
+        return MOE_ERR_UNSUPPORTED;
+      }
   }
 }
 
@@ -335,6 +365,7 @@ template <int EPI>
 moe_status launch_tc_bn(int bn, int wq, const TcParams& p, cudaStream_t st) {
   if (wq == WQ_INT8) return launch_tc_bn_q<EPI, WQ_INT8>(bn, p, st);
   if (wq == WQ_INT4) return launch_tc_bn_q<EPI, WQ_INT4>(bn, p, st);
+  if (wq == WQ_FP8) return launch_tc_bn_q<EPI, WQ_FP8>(bn, p, st);
   return launch_tc_bn_q<EPI, WQ_BF16>(bn, p, st);
 }
 
@@ -538,7 +569,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   const int T = c->T, k = c->k, S = c->n_shared;
   if (!w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID;
   if (S > 0 && (!w->sh_gate || !w->sh_up || !w->sh_down || !ys)) return MOE_ERR_INVALID;
-  if (c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4) {
+  if (quantised(c)) {
     if (!w->s_gate || !w->s_up || !w->s_down) return MOE_ERR_INVALID;
     if (S > 0 && (!w->sh_s_gate || !w->sh_s_up || !w->sh_s_down)) return MOE_ERR_INVALID;
   }
@@ -611,8 +642,9 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     // 8 rows of one matrix per block (K is d or f, both multiples of 128)
     const int kmax = c->d > c->f ? c->d : c->f;
     dim3 grid(kmax / 8, a.n, c->E > S ? c->E : S);
-    if (wq == WQ_INT4) MOE_LAUNCH((k_dequant_experts<true>), grid, 256, 0, st, a);
-    else MOE_LAUNCH((k_dequant_experts<false>), grid, 256, 0, st, a);
+    if (wq == WQ_INT4) MOE_LAUNCH((k_dequant_experts<1>), grid, 256, 0, st, a);
+    else if (wq == WQ_FP8) MOE_LAUNCH((k_dequant_experts<2>), grid, 256, 0, st, a);
+    else MOE_LAUNCH((k_dequant_experts<0>), grid, 256, 0, st, a);
     if ((s = check_launch()) != MOE_OK) return s;
     wl.w_gate = dst[0]; wl.w_up = dst[1]; wl.w_down = dst[2];
     wl.sh_gate = dst[3]; wl.sh_up = dst[4]; wl.sh_down = dst[5];

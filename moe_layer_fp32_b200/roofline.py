@@ -19,12 +19,12 @@ import json
 import os
 from typing import Optional, Sequence
 
-BYTES_PER_WEIGHT = {"f32": 4.0, "bf16": 2.0, "int8": 1.0, "int4": 0.5}
+BYTES_PER_WEIGHT = {"f32": 4.0, "bf16": 2.0, "int8": 1.0, "fp8": 1.0, "int4": 0.5}
 
 
 def scale_bytes_per_expert(expert: str, d: int, f: int, group: int = 128) -> float:
     """bf16 scale bytes of one expert's three matrices."""
-    if expert == "int8":
+    if expert in ("int8", "fp8"):
         return 2.0 * (f + f + d)                      # per output column
     if expert == "int4":
         return 2.0 * (2 * (d // group) * f + (f // group) * d)

@@ -22,6 +22,8 @@ Recipe (every tensor draws from its own PCG64 stream,
     ``bias_e = ln p_e - mean(ln p)``.
 * int8 weights: symmetric, one bf16 scale per output column,
   ``s = bf16(max|w| / 127)``, ``q = clamp(rint(w / s), -127, 127)``.
+* fp8 weights: FP8 E4M3 codes, one bf16 scale per output column,
+  ``s = bf16(max|w| / 448)``, ``q = e4m3(w / s)`` (round to nearest even).
 * int4 weights: symmetric, groups of ``group_size`` along the reduction (K) dim,
   ``s = bf16(max|w| / 7)``, ``q = clamp(rint(w / s), -8, 7)``; two values per byte
   along the contiguous (output) dim, low nibble first.
@@ -61,7 +63,7 @@ class LayerShape:
     n_shared: int = 0           # always-on shared experts (hidden f each)
     act: str = "bf16"           # x / out dtype: "bf16" | "f32"
     router: str = "bf16"        # router weight dtype: "bf16" | "f32"
-    expert: str = "bf16"        # "f32" | "bf16" | "int8" | "int4"
+    expert: str = "bf16"        # "f32" | "bf16" | "int8" | "int4" | "fp8"
     renormalize: bool = True    # gates renormalised over the selected k
     bias_mode: str = "none"     # "none" | "logit" | "select"
     capacity_factor: float = 0.0  # <= 0: uncapped
@@ -90,6 +92,9 @@ PRESETS: Dict[str, LayerShape] = {
     # the same layer with int8 per-channel experts
     "qwen3_int8": LayerShape("qwen3_int8", d=2048, E=128, k=8, f=768, expert="int8",
                              seed=3, tokens=(1, 64, 16384)),
+    # the same layer with FP8 (E4M3) per-channel experts
+    "qwen3_fp8": LayerShape("qwen3_fp8", d=2048, E=128, k=8, f=768, expert="fp8",
+                            seed=3, tokens=(1, 64, 16384)),
     # DeepSeek-V3-shaped layer: 1 shared expert, Zipf(1.1) select-mode bias
     "v3": LayerShape("v3", d=7168, E=256, k=8, f=2048, n_shared=1, bias_mode="select",
                      seed=4, tokens=(32, 256, 9440)),
@@ -166,6 +171,17 @@ def quantize_int8(w: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
     return q, s
 
 
+def quantize_fp8(w: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """w[K, N] fp32 -> (q uint8 FP8 E4M3 codes [K, N], s bf16 [N]); one scale per
+    output column, ``s = bf16(max|w| / 448)``, ``q = e4m3(w / s)`` rounded to nearest
+    even and clamped to the largest finite code (448)."""
+    amax = w.abs().amax(dim=0)
+    s = (amax / 448.0).to(torch.bfloat16)
+    s = torch.where(s.float() > 0, s, torch.ones_like(s))
+    q = (w / s.float()).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8), s
+
+
 def quantize_int4(w: torch.Tensor, group: int) -> Tuple[torch.Tensor, torch.Tensor]:
     """w[K, N] fp32 -> (packed uint8 [K, N/2], s bf16 [K/group, N]).
 
@@ -190,6 +206,8 @@ def _encode(shape: LayerShape, w: np.ndarray):
     t = torch.from_numpy(w)
     if shape.expert == "int8":
         return quantize_int8(t)
+    if shape.expert == "fp8":
+        return quantize_fp8(t)
     if shape.expert == "int4":
         return quantize_int4(t, shape.group_size)
     raise ValueError(shape.expert)

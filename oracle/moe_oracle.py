@@ -42,6 +42,9 @@ Readings where the pages are silent:
   ``< cap``.  Kept slots keep their gate (no re-renormalisation).
 * Expert: SwiGLU, ``y = (silu(xn Wg) * (xn Wu)) Wd``.
 * Combine: ``out = x + sum_s shared_s(xn) + sum_{kept j} g_j * y_j``.
+* fp8 weights (E4M3 codes with one bf16 scale per output column, "MoE at the
+  inference level", Workarounds: int4/fp8 expert weights) dequantise the same
+  way, ``bf16(e4m3(q) * s)``.
 * int8 and int4 weights dequantise to ``bf16(q * s)`` (the exact product rounded
   once to bf16): the layer's tensor-core GEMMs consume bf16 weights.
 """
@@ -172,6 +175,96 @@ def route(logits32, bias, k: int, bias_mode: str, renormalize: bool,
 
 
 # ---------------------------------------------------------------------------
+# expert-choice routing (the inverted assignment)
+# ---------------------------------------------------------------------------
+def expert_choice_capacity(capacity_factor: float, T: int, k: int, E: int) -> int:
+    """Tokens each expert picks: ceil(C * T*k/E) with C = 1 when the factor is <= 0
+    (the balanced case, C = 1.0 exact), at most T."""
+    c = float(np.float32(capacity_factor))
+    if c <= 0:
+        c = 1.0
+    return int(min(T, math.ceil(c * T * k / E)))
+
+
+def expert_choice_scores(logits32, bias, bias_mode: str) -> np.ndarray:
+    """Affinity of every (token, expert): the softmax over the experts of the FP32
+    logits (plus the bias in "logit" mode), in float64, as FP32 values."""
+    if bias_mode == BIAS_SELECT:
+        raise ValueError("expert-choice routing takes no selection-only bias")
+    _, p_in = selection_keys(logits32, bias, bias_mode)
+    return round_f32(softmax64(p_in))
+
+
+def expert_choice_select(scores32, C: int) -> Dict[str, np.ndarray]:
+    """Each expert e picks the C tokens with the largest score[t, e] (ties to the
+    lower token; NaN scores below every number).
+
+    tok[e, c]    the c-th picked token of expert e, in ascending token order
+    gate[e, c]   its score (the gate of that assignment)
+    slot[t, e]   e*C + c if token t was picked by e, else -1
+    margin[e]    gap between the C-th and (C+1)-th largest scores of e (inf if C == T)
+    """
+    s = np.asarray(scores32, dtype=np.float32)
+    T, E = s.shape
+    key = np.where(np.isnan(s), -np.inf, s).astype(np.float64)
+    tok = np.empty((E, C), dtype=np.int64)
+    gate = np.empty((E, C), dtype=np.float64)
+    slot = np.full((T, E), -1, dtype=np.int64)
+    margin = np.full(E, np.inf)
+    tokens = np.arange(T)
+    for e in range(E):
+        order = np.lexsort((tokens, -key[:, e]))          # score descending, token ascending
+        picked = np.sort(order[:C])
+        tok[e] = picked
+        gate[e] = s[picked, e]
+        slot[picked, e] = e * C + np.arange(C)
+        if C < T:
+            margin[e] = key[order[C - 1], e] - key[order[C], e]
+    return dict(tok=tok.astype(np.int32), gate=gate, slot=slot.astype(np.int32), margin=margin)
+
+
+def moe_layer_expert_choice(x, gamma, w_router, router_bias, experts: "Weights", *, k: int,
+                            act: str = "bf16", rms_eps: float = 1e-6,
+                            bias_mode: str = BIAS_NONE, capacity_factor: float = 0.0,
+                            shared: Optional["Weights"] = None, n_shared: int = 0,
+                            forced_scores=None, tokens: Optional[Sequence[int]] = None,
+                            residual: bool = True) -> Dict[str, np.ndarray]:
+    """Forward of one MoE layer under expert-choice routing ("MoE: dynamism the
+    compiler cannot remove", capacity section: instead of each token picking k
+    experts, each expert picks its top T*k/E tokens, so every expert holds exactly
+    C = T*k/E rows; a token may get several experts or none):
+
+        out[t] = x[t] + sum_s FFN_s(xn_t) + sum_{e : t picked by e} score[t, e] FFN_e(xn_t)
+
+    with the routed terms added in ascending e.  ``forced_scores`` replaces the
+    oracle's FP32 scores by given ones (selection replay)."""
+    x64 = np.asarray(x, np.float64)
+    T, d = x64.shape
+    E = np.asarray(w_router).shape[1]
+    xn = rmsnorm(x64, gamma, rms_eps, act)
+    logits = router_logits(xn, w_router)
+    logits32 = logits.astype(np.float32)
+    scores = expert_choice_scores(logits32, router_bias, bias_mode)
+    if forced_scores is not None:
+        scores = np.asarray(forced_scores, dtype=np.float32)
+    C = expert_choice_capacity(capacity_factor, T, k, E)
+    sel = expert_choice_select(scores, C)
+    rows = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    where = np.full(T, -1, dtype=np.int64)
+    where[rows] = np.arange(rows.size)
+    out = x64[rows].copy() if residual else np.zeros((rows.size, d))
+    for s_ in range(n_shared):
+        out += shared.ffn(s_, xn[rows])
+    for e in range(E):                                   # routed terms in ascending e
+        t_sel = sel["tok"][e][where[sel["tok"][e]] >= 0]
+        if t_sel.size == 0:
+            continue
+        g = sel["gate"][e][where[sel["tok"][e]] >= 0]
+        out[where[t_sel]] += g[:, None] * experts.ffn(e, xn[t_sel])
+    return dict(out=out, xn=xn, logits=logits, logits32=logits32, scores=scores, C=C, **sel)
+
+
+# ---------------------------------------------------------------------------
 # a4 / a5: histogram, scan, capacity and the stable permutation
 # ---------------------------------------------------------------------------
 def capacity(capacity_factor: float, T: int, k: int, E: int) -> Optional[int]:
@@ -238,12 +331,33 @@ def dequant_int4(packed, s, group: int) -> np.ndarray:
     return round_bf16(q * sk)
 
 
+def decode_e4m3(codes) -> np.ndarray:
+    """FP8 E4M3 codes (uint8) -> float64, from the format's definition: bit 7 sign,
+    bits 6..3 biased exponent (bias 7), bits 2..0 mantissa; exponent 0 encodes the
+    subnormals m/8 * 2^-6; this variant has no infinities and exponent 15 with
+    mantissa 7 encodes NaN (largest finite value 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequant_fp8(q, s) -> np.ndarray:
+    """w[K, N] = bf16(e4m3(q[K, N]) * s[N])."""
+    return round_bf16(decode_e4m3(q) * np.asarray(s, np.float64)[None, :])
+
+
 def expert_matrix(w, s, expert_dtype: str, group: int = 128) -> np.ndarray:
     """One expert's [K, N] weight matrix in float64."""
     if expert_dtype in ("bf16", "f32"):
         return np.asarray(w, np.float64)
     if expert_dtype == "int8":
         return dequant_int8(w, s)
+    if expert_dtype == "fp8":
+        return dequant_fp8(w, s)
     if expert_dtype == "int4":
         return dequant_int4(w, s, group)
     raise ValueError(expert_dtype)
@@ -375,6 +489,17 @@ def weights_from_inputs(li, shared: bool = False) -> Optional[Weights]:
     return Weights(sh.expert, sh.group_size, get("w_gate" if not shared else "gate"),
                    get("w_up" if not shared else "up"), get("w_down" if not shared else "down"),
                    get("s_gate"), get("s_up"), get("s_down"))
+
+
+def layer_expert_choice_from_inputs(li, x, **kw) -> Dict[str, np.ndarray]:
+    """Run ``moe_layer_expert_choice`` on a ``moe_synth.LayerInputs``."""
+    sh = li.shape
+    args = dict(k=sh.k, act=sh.act, rms_eps=sh.rms_eps, bias_mode=sh.bias_mode,
+                capacity_factor=sh.capacity_factor, shared=weights_from_inputs(li, shared=True),
+                n_shared=sh.n_shared)
+    args.update(kw)
+    return moe_layer_expert_choice(_npy(x), _npy(li.gamma), _npy(li.w_router),
+                                   _npy(li.router_bias), weights_from_inputs(li), **args)
 
 
 def layer_from_inputs(li, x, **kw) -> Dict[str, np.ndarray]:

@@ -7,7 +7,7 @@ Tolerances (each derived from the arithmetic of the path):
   the oracle's k-th/(k+1)-th key margin is below 1e-4;
 * bf16 experts: max|out - out_oracle| / RMS(out_oracle) <= 1e-2 on the FP32
   layer output, against the oracle re-run with the GPU's routes; int8 / int4
-  experts: <= 3e-2 (the same oracle, same dequantised weights); fp32 experts:
+  / fp8 experts: <= 3e-2 (the same oracle, same dequantised weights); fp32 experts:
   <= 1e-5.  The ratio against RMS(out_oracle - x) (the MoE delta alone) is
   reported beside it and held under DELTA_GUARD.
 """
@@ -25,8 +25,8 @@ from moe_layer_fp32_b200.drift import route_drift
 from oracle import moe_oracle as O
 
 ROUTE_MARGIN = 1e-4
-TOL = {"f32": 1e-5, "bf16": 1e-2, "int8": 3e-2, "int4": 3e-2}
-DELTA_GUARD = {"f32": 1e-4, "bf16": 3e-2, "int8": 6e-2, "int4": 6e-2}
+TOL = {"f32": 1e-5, "bf16": 1e-2, "int8": 3e-2, "int4": 3e-2, "fp8": 3e-2}
+DELTA_GUARD = {"f32": 1e-4, "bf16": 3e-2, "int8": 6e-2, "int4": 6e-2, "fp8": 6e-2}
 
 
 def inputs_on_device(shape, T, x_stream=None):

@@ -140,7 +140,8 @@ def test_make_weights_maps_every_layer_tensor():
 LAUNCHES = [("tiny", 64, 7), ("olmoe", 1, 6), ("olmoe", 16, 6), ("olmoe", 64, 7),
             ("olmoe", 4096, 10), ("v2lite", 32, 6), ("v2lite", 8192, 10),
             ("qwen3_int4", 1, 7), ("qwen3_int4", 64, 8), ("qwen3_int4", 16384, 11),
-            ("qwen3_int8", 16384, 11), ("v3", 32, 6), ("v3", 256, 7), ("v3", 9440, 10)]
+            ("qwen3_int8", 16384, 11), ("qwen3_fp8", 64, 8), ("qwen3_fp8", 16384, 11),
+            ("v3", 32, 6), ("v3", 256, 7), ("v3", 9440, 10)]
 
 
 @pytest.mark.parametrize("preset,T,n", LAUNCHES)

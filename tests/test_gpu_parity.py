@@ -34,6 +34,16 @@ SMALL = {
                                expert="int8", seed=18),
     # tensor-core router with K split into 4 parts (partial logits added by the route)
     "bf16_tc_router_split": LayerShape("bf16_router_split", d=1024, E=64, k=4, f=256, seed=20),
+    # prefill tiles under Zipf-skewed routing and a shared expert: 256-token pair
+    # tiles whose odd CTA holds no rows, tiles with a few rows, experts with none
+    "bf16_prefill_skew": LayerShape("bf16_prefill_skew", d=256, E=16, k=4, f=384, n_shared=1,
+                                    bias_mode="select", seed=21),
+    # FP8 (E4M3) experts: decode tiles (in-loop dequantisation, split K) and
+    # prefill tiles (dequantised once), with a shared expert and capacity
+    "fp8_decode": LayerShape("fp8_decode", d=384, E=32, k=6, f=256, n_shared=1, expert="fp8",
+                             bias_mode="logit", seed=22),
+    "fp8_prefill": LayerShape("fp8_prefill", d=512, E=8, k=2, f=384, expert="fp8",
+                              capacity_factor=1.25, seed=23),
     # FP32 experts with f not a multiple of 4 (scalar weight columns in gate/up)
     "f32_odd_f": LayerShape("f32_odd_f", d=136, E=6, k=2, f=130, n_shared=1, act="f32",
                             router="f32", expert="f32", capacity_factor=1.5,
@@ -42,7 +52,8 @@ SMALL = {
 SMALL_T = {"bf16_plain": 100, "bf16_shared_cap": 77, "bf16_select_tc_router": 200,
            "bf16_prefill_tiles": 1000, "f32_tiny": 64, "int4_decode": 20, "int8_decode": 50,
            "int4_prefill": 900, "int8_prefill": 700, "f32_odd_f": 37,
-           "bf16_tc_router_split": 300}
+           "bf16_tc_router_split": 300, "bf16_prefill_skew": 700, "fp8_decode": 40,
+           "fp8_prefill": 800}
 
 
 @pytest.fixture(autouse=True)
@@ -155,7 +166,8 @@ def test_permute_flags_out_of_range_expert():
 
 # --------------------------------------------------------------------- a6 + a7
 @pytest.mark.parametrize("name", ["bf16_plain", "bf16_shared_cap", "bf16_prefill_tiles", "f32_tiny",
-                                  "int4_decode", "int8_decode", "int4_prefill", "int8_prefill"])
+                                  "int4_decode", "int8_decode", "int4_prefill", "int8_prefill",
+                                  "bf16_prefill_skew", "fp8_decode", "fp8_prefill"])
 def test_grouped_ffn_matches_oracle_per_assignment(name):
     sh, T = SMALL[name], SMALL_T[name]
     li, x, dli, dx = inputs_on_device(sh, T)
@@ -294,7 +306,8 @@ def test_bf16_output_is_rounding_of_fp32_output():
 # --------------------------------------------------------------------- full sizes
 FULL = [("olmoe", 1), ("olmoe", 16), ("olmoe", 64), ("olmoe", 4096),
         ("v2lite", 32), ("v2lite", 8192), ("qwen3_int4", 1), ("qwen3_int4", 64),
-        ("qwen3_int4", 16384), ("qwen3_int8", 1), ("qwen3_int8", 64), ("qwen3_int8", 16384)]
+        ("qwen3_int4", 16384), ("qwen3_int8", 1), ("qwen3_int8", 64), ("qwen3_int8", 16384),
+        ("qwen3_fp8", 1), ("qwen3_fp8", 64), ("qwen3_fp8", 16384)]
 
 
 @pytest.mark.parametrize("preset,T", FULL)

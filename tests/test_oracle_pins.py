@@ -265,6 +265,33 @@ def test_quantised_weights_within_quantisation_bound():
     np.testing.assert_array_equal(dq4, O.round_bf16(dq4))
 
 
+def test_e4m3_decode_matches_torch_float8_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.decode_e4m3(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+    # closed forms: 1.0, the largest finite value, the smallest subnormal, a sign
+    assert O.decode_e4m3([0x38])[0] == 1.0 and O.decode_e4m3([0x7E])[0] == 448.0
+    assert O.decode_e4m3([0x01])[0] == 2.0 ** -9 and O.decode_e4m3([0xB8])[0] == -1.0
+    assert np.isnan(O.decode_e4m3([0x7F, 0xFF])).all()
+
+
+def test_fp8_weights_within_quantisation_bound():
+    w = torch.from_numpy(rng(13).standard_normal((256, 64)).astype(np.float32)) * 0.05
+    q, s = moe_synth.quantize_fp8(w)
+    dq = O.dequant_fp8(q.numpy(), s.float().numpy())
+    # e4m3 keeps 3 mantissa bits: relative error <= 2^-4 for normals, absolute
+    # <= 2^-10 s below the normal range; then one bf16 rounding of q*s
+    sf = s.float().numpy()[None, :]
+    bound = np.abs(w.numpy()) * 2.0 ** -4 + sf * 2.0 ** -10 + np.abs(dq) * 2.0 ** -8
+    assert np.all(np.abs(dq - w.numpy()) <= bound * (1 + 1e-6))
+    np.testing.assert_array_equal(dq, O.round_bf16(dq))
+    # the column maximum maps to (nearly) the largest code
+    assert np.all(np.abs(O.decode_e4m3(q.numpy())).max(axis=0) >= 416)
+
+
 # ---------------------------------------------------------------------------
 # a6 / a7 expert FFN, a8 combine, the whole layer
 # ---------------------------------------------------------------------------

@@ -5,6 +5,7 @@ import numpy as np
 import pytest
 
 from oracle import moe_oracle as O
+from tests import test_oracle_expert_choice as EC
 from tests import test_oracle_pins as P
 
 
@@ -71,6 +72,25 @@ def _route_gates_unrenormalised(logits32, bias, k, bias_mode, renormalize, force
 _real_route = O.route
 
 
+_real_ec_select = O.expert_choice_select
+
+
+def _ec_ties_to_higher_token(scores32, C):
+    s = np.asarray(scores32, np.float32)
+    r = _real_ec_select(s[::-1], C)             # reversed token order: ties go high
+    T = s.shape[0]
+    tok = np.sort(T - 1 - r["tok"], axis=1).astype(np.int32)
+    return dict(r, tok=tok, gate=np.take_along_axis(s.T, tok, axis=1).astype(np.float64))
+
+
+def _ec_decode_e4m3_bias_8(codes):
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -7, (1.0 + m / 8.0) * np.exp2(e - 8.0))
+    return np.where(c & 0x80, -1.0, 1.0) * mag
+
+
 MUTANTS = [
     ("rmsnorm", _rms_sum_not_mean, P.test_rmsnorm_matches_torch_rms_norm),
     ("rmsnorm", _rms_no_eps, P.test_rmsnorm_eps_matters_for_tiny_rows),
@@ -82,6 +102,9 @@ MUTANTS = [
     ("softmax64", _softmax_no_shift_wrong_axis, P.test_softmax_matches_torch),
     ("permute", _permute_keeps_one_extra, lambda: P.test_permute_matches_brute_force(1.0)),
     ("route", _route_gates_unrenormalised, P.test_gates_renormalised_and_bias_modes),
+    ("expert_choice_select", _ec_ties_to_higher_token,
+     EC.test_selection_matches_a_library_sort_with_ties),
+    ("decode_e4m3", _ec_decode_e4m3_bias_8, P.test_e4m3_decode_matches_torch_float8_on_every_code),
 ]
 
 
