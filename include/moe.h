@@ -78,6 +78,18 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_INT8 = 2, MOE_INT4 = 3, MOE_FP8 = 
  *            gates are the softmax of the unbiased logits. */
 typedef enum { MOE_BIAS_NONE = 0, MOE_BIAS_LOGIT = 1, MOE_BIAS_SELECT = 2 } moe_bias_mode;
 
+/* Routing ("MoE: dynamism the compiler cannot remove", capacity section):
+ *   TOPK           : each token picks its top-k experts (the layer of the pages);
+ *   EXPERT_CHOICE  : each expert picks the C = ceil(C_f * T*k/E) tokens (C_f = the
+ *                    capacity factor, 1 when <= 0; at most T) with the largest gate
+ *                    probability -- the softmax over the experts of the token's FP32
+ *                    logits (plus the bias in LOGIT mode); that probability is the
+ *                    assignment's gate.  Every expert holds exactly C rows; a token
+ *                    may get several experts or none.  Ties at an expert's C-th
+ *                    score go to the lower token.  Not with SELECT bias or FP32
+ *                    experts. */
+typedef enum { MOE_ROUTE_TOPK = 0, MOE_ROUTE_EXPERT_CHOICE = 1 } moe_routing;
+
 /* Layer configuration.  All fields are 32-bit so that the layout is the same
  * from every language. */
 typedef struct moe_config {
@@ -104,6 +116,7 @@ typedef struct moe_config {
                               1024 SM clock cycles; 0 = the default, 10^9 cycles (about
                               half a second).  A wait that runs out sets device error 2
                               and the kernel returns early (moe_get_device_status)      */
+  int32_t routing;         /* moe_routing (0 = top-k)                                    */
 } moe_config;
 
 /* Layer weights (device pointers, caller-owned).
@@ -185,6 +198,29 @@ moe_status moe_rmsnorm_router(const moe_config* cfg, const moe_weights* w, const
 moe_status moe_route(const moe_config* cfg, const float* logits, const float* bias,
                      int32_t* topk_idx, float* topk_gate, void* stream);
 
+/* Expert-choice routing (cfg->routing == MOE_ROUTE_EXPERT_CHOICE): the routing
+ * and permutation steps of that mode.
+ * Source: "MoE: dynamism the compiler cannot remove", capacity section -- each
+ * expert picks its top T*k/E tokens, which balances the load by construction.
+ *   logits     [T, E] float32 router logits (bias not included)
+ *   bias       [E] float32 or NULL (LOGIT mode adds it before the softmax)
+ *   scores_out [T, E] float32 or NULL: the FP32 softmax over the experts, on which
+ *              the picks are taken
+ *   tok        [E*C] int32: slot e*C + c holds the c-th token expert e picked, in
+ *              ascending token order (C = moe_expert_choice_capacity(cfg))
+ *   gate       [E*C] float32: that token's score for expert e
+ *   slot_te    [T, E] int32: the slot of (token, expert), or -1 if not picked
+ *   ws         workspace (the scores are kept there expert-major)
+ * The picks are deterministic and, given identical FP32 scores, bit-exact to any
+ * correct implementation of the rule above. */
+moe_status moe_route_expert_choice(const moe_config* cfg, const float* logits, const float* bias,
+                                   float* scores_out, int32_t* tok, float* gate,
+                                   int32_t* slot_te, void* ws, size_t ws_bytes, void* stream);
+
+/* Tokens each expert picks under expert-choice routing (0 for a top-k or an
+ * invalid configuration).  Source: as moe_route_expert_choice. */
+int32_t moe_expert_choice_capacity(const moe_config* cfg);
+
 /* Steps a4 + a5: per-expert histogram, prefix scan, capacity and the stable
  * permutation ("MoE Research", section 3: grouped GEMM and sorting).  No global
  * atomics; deterministic.
@@ -263,6 +299,10 @@ moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32
  * Workarounds.
  *   x [T, d] act dtype, out [T, d] out dtype.  Optional outputs (NULL to skip):
  *   logits_out [T, E] float32, topk_idx_out [T, k] int32, counts_out [E] int32.
+ * With expert-choice routing the chain is RMSNorm, router, scores, the experts'
+ * picks, the grouped GEMMs over the E*C picks and a combine that adds, per token,
+ * the rows of the experts that picked it in ascending expert order; topk_idx_out
+ * must then be NULL and counts_out receives C for every expert.
  * Between the down GEMM and the combine the gated routed rows of tensor-core
  * experts are kept in bf16 (the round-to-nearest-even of the FP32 rows that
  * moe_grouped_ffn returns), so the result equals moe_combine applied to those

@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
 MOE_F32, MOE_BF16, MOE_INT8, MOE_INT4, MOE_FP8 = range(5)
 MOE_BIAS_NONE, MOE_BIAS_LOGIT, MOE_BIAS_SELECT = range(3)
+MOE_ROUTE_TOPK, MOE_ROUTE_EXPERT_CHOICE = range(2)
+ROUTING_CODE = {"topk": MOE_ROUTE_TOPK, "expert_choice": MOE_ROUTE_EXPERT_CHOICE}
 
 DTYPE_CODE = {"f32": MOE_F32, "bf16": MOE_BF16, "int8": MOE_INT8, "int4": MOE_INT4,
               "fp8": MOE_FP8}
@@ -32,7 +34,8 @@ class MoeConfig(ctypes.Structure):
                 ("bias_mode", ctypes.c_int32), ("rms_eps", ctypes.c_float),
                 ("act_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
                 ("router_dtype", ctypes.c_int32), ("expert_dtype", ctypes.c_int32),
-                ("group_size", ctypes.c_int32), ("wait_kcycles", ctypes.c_int32)]
+                ("group_size", ctypes.c_int32), ("wait_kcycles", ctypes.c_int32),
+                ("routing", ctypes.c_int32)]
 
 
 class MoeWeights(ctypes.Structure):
@@ -57,6 +60,9 @@ _SIGS = {
     "moe_rmsnorm_router": (ctypes.c_int, [_CFG, _WTS, _VP, _VP, _F32P, _VP, _SZ, _VP]),
     "moe_route": (ctypes.c_int, [_CFG, _F32P, _F32P, _I32P, _F32P, _VP]),
     "moe_permute": (ctypes.c_int, [_CFG, _I32P, _I32P, _I32P, _I32P, _I32P, _I32P, _VP, _SZ, _VP]),
+    "moe_route_expert_choice": (ctypes.c_int, [_CFG, _F32P, _F32P, _F32P, _I32P, _F32P, _I32P,
+                                               _VP, _SZ, _VP]),
+    "moe_expert_choice_capacity": (ctypes.c_int32, [_CFG]),
     "moe_permute_static": (ctypes.c_int, [_CFG, _I32P, _I32P, _I32P, _I32P, _I32P, _I32P, _VP]),
     "moe_grouped_ffn": (ctypes.c_int, [_CFG, _WTS, _VP, _I32P, _I32P, _F32P, _F32P, _F32P, _VP, _SZ, _VP]),
     "moe_combine": (ctypes.c_int, [_CFG, _F32P, _I32P, _F32P, _VP, _VP, _VP]),
@@ -116,7 +122,8 @@ def make_config(shape, T: int, out_dtype: Optional[str] = None) -> MoeConfig:
                      renormalize=int(bool(shape.renormalize)), bias_mode=BIAS_CODE[shape.bias_mode],
                      rms_eps=float(shape.rms_eps), act_dtype=DTYPE_CODE[shape.act],
                      out_dtype=DTYPE_CODE[out], router_dtype=DTYPE_CODE[shape.router],
-                     expert_dtype=DTYPE_CODE[shape.expert], group_size=int(shape.group_size))
+                     expert_dtype=DTYPE_CODE[shape.expert], group_size=int(shape.group_size),
+                     routing=ROUTING_CODE[getattr(shape, "routing", "topk")])
 
 
 def make_weights(li) -> MoeWeights:
@@ -170,6 +177,16 @@ def moe_permute_static(cfg, topk_idx, counts, offsets, perm_assign, slot_of, n_d
     _check("moe_permute_static", lib().moe_permute_static(
         ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(offsets), _p(perm_assign), _p(slot_of),
         _p(n_dropped), _stream(stream)))
+
+
+def moe_route_expert_choice(cfg, logits, bias, scores_out, tok, gate, slot_te, ws, stream=None):
+    _check("moe_route_expert_choice", lib().moe_route_expert_choice(
+        ctypes.byref(cfg), _p(logits), _p(bias), _p(scores_out), _p(tok), _p(gate), _p(slot_te),
+        _p(ws), ws.numel(), _stream(stream)))
+
+
+def moe_expert_choice_capacity(cfg) -> int:
+    return int(lib().moe_expert_choice_capacity(ctypes.byref(cfg)))
 
 
 def moe_grouped_ffn(cfg, w: MoeWeights, xn, offsets, perm_assign, topk_gate, y_assign, y_shared,

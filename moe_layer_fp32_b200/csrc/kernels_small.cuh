@@ -282,17 +282,14 @@ MOE_DEV bool key_better(float ka, int ea, float kb, int eb) {
   return ka > kb || (ka == kb && ea < eb);
 }
 
-// Routes token t with the calling warp.  The router partials of the ns K-slices
-// are added in slice order; their loads are issued 8 at a time so that they
-// overlap instead of each waiting for the previous add.
+// Logits of token t for the calling lane's experts (lane, lane + 32, ...): the
+// router partials of the ns K-slices added in slice order; their loads are issued
+// SU slices at a time for all of the lane's experts together, so that they overlap
+// instead of each waiting for the previous add.
 template <int EPL>
-MOE_DEV void route_token(const float* part, int ns, int T, int E, int k, const float* bias,
-                         int mode, int renorm, int32_t* idx, float* gate, float* logits_out,
-                         int t, int lane) {
-  // logits: the ns slice partials of this lane's experts, loaded SU slices at a time
-  // for all of them together, each added in slice order
+MOE_DEV void router_logits_of_lane(const float* part, int ns, int T, int E, int t, int lane,
+                                   float (&lg)[EPL]) {
   constexpr int SU = EPL <= 4 ? 4 : EPL <= 8 ? 2 : 1;
-  float lg[EPL];
   const size_t sstride = (size_t)T * E;
   const float* pt = part + (size_t)t * E + lane;
 #pragma unroll
@@ -310,6 +307,15 @@ MOE_DEV void route_token(const float* part, int ns, int T, int E, int k, const f
       for (int u = 0; u < SU; ++u)
         if (s0 + u < ns) lg[i] += v[i][u];
   }
+}
+
+// Routes token t with the calling warp.
+template <int EPL>
+MOE_DEV void route_token(const float* part, int ns, int T, int E, int k, const float* bias,
+                         int mode, int renorm, int32_t* idx, float* gate, float* logits_out,
+                         int t, int lane) {
+  float lg[EPL];
+  router_logits_of_lane<EPL>(part, ns, T, E, t, lane, lg);
   float key[EPL], pin[EPL];
   float mx = -INFINITY;
 #pragma unroll

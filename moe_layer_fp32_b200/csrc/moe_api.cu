@@ -14,6 +14,7 @@
 #include "kernels_small.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_pair.cuh"
+#include "kernels_ec.cuh"
 
 using namespace moe;
 
@@ -62,9 +63,22 @@ inline int router_slice(const moe_config* c, int ns) {
   return (s + 7) / 8 * 8;
 }
 
+// Expert-choice routing: every expert picks C = ceil(C_f * T*k/E) tokens (C_f = 1
+// when capacity_factor <= 0), at most T.
+inline bool expert_choice(const moe_config* c) { return c->routing == MOE_ROUTE_EXPERT_CHOICE; }
+int ec_capacity(const moe_config* c) {
+  const double cf = c->capacity_factor > 0.f ? (double)c->capacity_factor : 1.0;
+  const double v = std::ceil(cf * c->T * c->k / c->E);
+  return v >= (double)c->T ? c->T : (int)v;
+}
+// routed rows the expert GEMMs hold at most: T*k assignments, or E*C picks
+inline size_t n_slots(const moe_config* c) {
+  return expert_choice(c) ? (size_t)c->E * ec_capacity(c) : (size_t)c->T * c->k;
+}
+
 // token-tile width of the expert GEMMs from the mean rows per expert
 int pick_bn(const moe_config* c) {
-  const double mean = (double)c->T * c->k / c->E;
+  const double mean = (double)n_slots(c) / c->E;
   if (mean <= 16) return 16;
   if (mean <= 32) return 32;
   if (mean <= 64) return 64;
@@ -102,7 +116,7 @@ inline bool dequant_once(const moe_config* c) { return quantised(c) && pick_bn(c
 
 struct Layout {
   size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, split,
-      splitcnt, h, y, ys, deq,
+      splitcnt, h, y, ys, deq, sct,
       total;
   int ns;
 };
@@ -120,6 +134,15 @@ moe_status validate(const moe_config* c) {
   if (c->bias_mode < MOE_BIAS_NONE || c->bias_mode > MOE_BIAS_SELECT) return MOE_ERR_INVALID;
   if (!(c->rms_eps >= 0.f) || !std::isfinite(c->capacity_factor)) return MOE_ERR_INVALID;
   if (c->wait_kcycles < 0) return MOE_ERR_INVALID;
+  if (c->routing != MOE_ROUTE_TOPK && c->routing != MOE_ROUTE_EXPERT_CHOICE)
+    return MOE_ERR_INVALID;
+  if (c->routing == MOE_ROUTE_EXPERT_CHOICE) {
+    // the expert picks rank tokens by their gate probability: a selection-only bias
+    // has no meaning there; the FP32 (CUDA-core) experts take the top-k path only
+    if (c->bias_mode == MOE_BIAS_SELECT) return MOE_ERR_UNSUPPORTED;
+    if (c->expert_dtype == MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if ((double)c->E * c->T > (double)(1 << 30)) return MOE_ERR_INVALID;
+  }
   switch (c->expert_dtype) {
     case MOE_F32:
       if (c->act_dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
@@ -151,21 +174,27 @@ Layout layout(const moe_config* c) {
   L.err = o;      o = align_up(o + 16);
   L.xn = o;       o = align_up(o + T * d * act);
   L.part = o;     o = align_up(o + (size_t)L.ns * T * E * 4);
-  L.idx = o;      o = align_up(o + T * k * 4);
-  L.gate = o;     o = align_up(o + T * k * 4);
+  // routed rows: T*k assignments (top-k) or E*C picks (expert choice); with expert
+  // choice idx / gate / perm hold the picks' token / gate / output row, slot the
+  // token x expert slot map and sct the scores expert-major
+  const size_t R = n_slots(c);
+  const size_t nslot = expert_choice(c) ? T * E : T * k;
+  L.idx = o;      o = align_up(o + R * 4);
+  L.gate = o;     o = align_up(o + R * 4);
   L.counts = o;   o = align_up(o + E * 4);
   L.offsets = o;  o = align_up(o + (E + 1) * 4);
-  L.perm = o;     o = align_up(o + T * k * 4);
-  L.slot = o;     o = align_up(o + T * k * 4);
+  L.perm = o;     o = align_up(o + R * 4);
+  L.slot = o;     o = align_up(o + nslot * 4);
   L.dropped = o;  o = align_up(o + 16);
   L.blk = o;      o = align_up(o + (size_t)E * ((T * k + kPermChunk - 1) / kPermChunk) * 4);
-  L.xp = o;       o = align_up(o + (tc_experts(c) && !gather_in_gemm(c) ? T * k * d * act : 0));
+  L.xp = o;       o = align_up(o + (tc_experts(c) && !gather_in_gemm(c) ? R * d * act : 0));
   L.split = o;    o = align_up(o + (split_k(c) ? (size_t)num_sms() * 2 * pick_bn(c) * 128 * 4 : 0));
   L.splitcnt = o; o = align_up(o + (split_k(c) ? (size_t)split_counters() * 4 : 0));
-  L.h = o;        o = align_up(o + (T * k + S * T) * f * hb);
-  L.y = o;        o = align_up(o + T * k * d * (y_bf16(c) ? 2 : 4));
+  L.h = o;        o = align_up(o + (R + S * T) * f * hb);
+  L.y = o;        o = align_up(o + R * d * (y_bf16(c) ? 2 : 4));
   L.ys = o;       o = align_up(o + S * T * d * 4);
   L.deq = o;      o = align_up(o + (dequant_once(c) ? (E + S) * 3 * d * f * 2 : 0));
+  L.sct = o;      o = align_up(o + (expert_choice(c) ? T * E * 4 : 0));
   L.total = o;
   return L;
 }
@@ -558,8 +587,18 @@ moe_status launch_simt(const SimtArgs& a, int grid, cudaStream_t st) {
   return check_launch();
 }
 
+// Routed rows of the expert GEMMs: slot s (< offsets[E]) gathers token
+// src[s] / src_k of xn, and the down GEMM stores its row, scaled by gate[dst[s]],
+// as row dst[s] of y.  Top-k: src = dst = perm_assign, src_k = k.  Expert choice:
+// src = the picked tokens (src_k = 1), dst = the identity.
+struct RoutedRows {
+  const int32_t* src;
+  int src_k;
+  const int32_t* dst;
+};
+
 moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
-                   const int32_t* offsets, const int32_t* perm, const float* gate, void* y,
+                   const int32_t* offsets, RoutedRows rr, const float* gate, void* y,
                    float* ys, void* ws, cudaStream_t st, Marks* mk = nullptr,
                    bool counters_zeroed = false, bool rows_bf16 = false) {
   Marks none;
@@ -567,6 +606,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   const Layout L = layout(c);
   int32_t* err = at<int32_t>(ws, L.err);
   const int T = c->T, k = c->k, S = c->n_shared;
+  const int32_t* perm = rr.dst;
   if (!w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID;
   if (S > 0 && (!w->sh_gate || !w->sh_up || !w->sh_down || !ys)) return MOE_ERR_INVALID;
   if (quantised(c)) {
@@ -615,7 +655,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   }
   __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
   const int bn = pick_bn(c);
-  const int R = T * k;
+  const int R = (int)n_slots(c);
   int wq = wq_of(c);
   moe_weights wl = *w;                     // the weights the GEMMs read
   moe_status s = MOE_OK;
@@ -660,7 +700,8 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   if (!g4) {
     // 64 warps per SM, so that many rows are in flight at once
     MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 8 * num_sms(), 256, 0, st,
-               static_cast<const __nv_bfloat16*>(xn), perm, offsets + c->E, k, c->d, xp);
+               static_cast<const __nv_bfloat16*>(xn), rr.src, offsets + c->E, rr.src_k, c->d,
+               xp);
     if ((s = check_launch()) != MOE_OK) return s;
   }
   mk->mark(st);   // end of the (optional) dequantisation and gather step
@@ -672,8 +713,8 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     if (g4) {
       // routed rows: slot s reads token perm[s] / k of xn, four rows per copy
       if (!map_rows(&P.tmB, xn, T, c->d, 1)) return MOE_ERR_CUDA;
-      P.gather_rows = perm;
-      P.gather_k = k;
+      P.gather_rows = rr.src;
+      P.gather_k = rr.src_k;
     } else if (!map_rows(&P.tmB, xp, R, c->d, bn)) {
       return MOE_ERR_CUDA;
     }
@@ -815,6 +856,57 @@ moe_status run_combine(const moe_config* c, const void* y, bool rows_bf16, const
   return launch_combine<1>(c, y, rows_bf16, slot, ys, res, out, st);
 }
 
+template <int VEC>
+moe_status launch_combine_ec(const moe_config* c, const void* y, bool rows_bf16,
+                             const int32_t* slot_te, const float* ys, const void* res, void* out,
+                             cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  auto rb = static_cast<const bf*>(res);
+  const int T = c->T, E = c->E, S = c->n_shared, d = c->d;
+  if (!rows_bf16) return MOE_ERR_UNSUPPORTED;   // tensor-core experts: bf16 rows
+  auto yb = static_cast<const bf*>(y);
+  if (c->out_dtype == MOE_BF16)
+    MOE_LAUNCH((k_combine_ec<bf, bf, bf, VEC>), T, 256, 0, st, yb, slot_te, E, ys, S, rb,
+               static_cast<bf*>(out), T, d);
+  else
+    MOE_LAUNCH((k_combine_ec<bf, float, bf, VEC>), T, 256, 0, st, yb, slot_te, E, ys, S, rb,
+               static_cast<float*>(out), T, d);
+  return check_launch();
+}
+
+moe_status run_combine_ec(const moe_config* c, const void* y, bool rows_bf16,
+                          const int32_t* slot_te, const float* ys, const void* res, void* out,
+                          cudaStream_t st) {
+  auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  if (a16(y) && a16(ys) && a16(res) && a16(out))
+    return launch_combine_ec<4>(c, y, rows_bf16, slot_te, ys, res, out, st);
+  return launch_combine_ec<1>(c, y, rows_bf16, slot_te, ys, res, out, st);
+}
+
+// Expert-choice routing from router partials (ns K-slices): FP32 scores, then each
+// expert's C picks.  tok / gate / yrow [E*C], offsets [E+1], counts [E], slot_te [T, E].
+moe_status run_route_ec(const moe_config* c, const float* part, int ns, const float* bias,
+                        float* scores_t, float* scores_out, float* logits_out, int32_t* tok,
+                        float* gate, int32_t* yrow, int32_t* offsets, int32_t* counts,
+                        int32_t* slot_te, cudaStream_t st, Marks* mk = nullptr) {
+  const int mode = c->bias_mode;
+  if (mode != MOE_BIAS_NONE && !bias) return MOE_ERR_INVALID;
+  const int blocks = (c->T + 7) / 8;
+#define MOE_EC_SCORES(EPL)                                                                 \
+  MOE_LAUNCH((k_ec_scores<EPL>), blocks, 256, 0, st, part, ns, c->T, c->E, bias, mode,     \
+             scores_t, scores_out, logits_out)
+  if (c->E <= 32) MOE_EC_SCORES(1);
+  else if (c->E <= 64) MOE_EC_SCORES(2);
+  else if (c->E <= 128) MOE_EC_SCORES(4);
+  else if (c->E <= 256) MOE_EC_SCORES(8);
+  else MOE_EC_SCORES(16);
+#undef MOE_EC_SCORES
+  if (mk) mk->mark(st);   // end of the routing step (scores)
+  MOE_LAUNCH((k_ec_select), c->E, 1024, 0, st, scores_t, c->T, c->E, ec_capacity(c), tok, gate,
+             yrow, offsets, counts, slot_te);
+  return check_launch();
+}
+
 moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const void* x,
                               void* out, void* ws, size_t ws_bytes, float* logits_out,
                               int32_t* topk_idx_out, int32_t* counts_out, cudaStream_t st,
@@ -844,6 +936,25 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
   mk->mark(st);
   if ((s = run_router(cfg, w, xn, part, L.ns, err, st)) != MOE_OK) return s;
   mk->mark(st);
+  if (expert_choice(cfg)) {
+    // scores (the routing step), the experts' picks (the permutation step), the
+    // expert GEMMs over the E*C picks, and the per-token combine
+    if (topk_idx_out) return MOE_ERR_INVALID;
+    int32_t* tok = at<int32_t>(ws, L.idx);
+    int32_t* yrow = at<int32_t>(ws, L.perm);
+    int32_t* slot_te = at<int32_t>(ws, L.slot);
+    if ((s = run_route_ec(cfg, part, L.ns, static_cast<const float*>(w->router_bias),
+                          at<float>(ws, L.sct), nullptr, logits_out, tok, gate, yrow, offsets,
+                          counts, slot_te, st, mk)) != MOE_OK)
+      return s;
+    mk->mark(st);
+    if ((s = run_ffn(cfg, w, xn, offsets, RoutedRows{tok, 1, yrow}, gate, y, ys, ws, st, mk,
+                     true, y_bf16(cfg))) != MOE_OK)
+      return s;
+    s = run_combine_ec(cfg, y, y_bf16(cfg), slot_te, ys, x, out, st);
+    mk->mark(st);
+    return s;
+  }
   if (fused_route_permute(cfg)) {
     // one launch; the permutation step has no time of its own in the profile
     if ((s = run_route_permute(cfg, part, L.ns, static_cast<const float*>(w->router_bias), idx,
@@ -861,8 +972,8 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
       return s;
   }
   mk->mark(st);
-  if ((s = run_ffn(cfg, w, xn, offsets, perm, gate, y, ys, ws, st, mk, true, y_bf16(cfg))) !=
-      MOE_OK)
+  if ((s = run_ffn(cfg, w, xn, offsets, RoutedRows{perm, cfg->k, perm}, gate, y, ys, ws, st, mk,
+                   true, y_bf16(cfg))) != MOE_OK)
     return s;
   s = run_combine(cfg, y, y_bf16(cfg), slot, ys, x, out, st);
   mk->mark(st);
@@ -936,7 +1047,27 @@ moe_status moe_route(const moe_config* cfg, const float* logits, const float* bi
   moe_status s = validate(cfg);
   if (s != MOE_OK) return s;
   if (!logits || !topk_idx || !topk_gate) return MOE_ERR_INVALID;
+  if (expert_choice(cfg)) return MOE_ERR_INVALID;   // moe_route_expert_choice
   return run_route(cfg, logits, 1, bias, topk_idx, topk_gate, nullptr, S_(stream));
+}
+
+int32_t moe_expert_choice_capacity(const moe_config* cfg) {
+  if (validate(cfg) != MOE_OK || !expert_choice(cfg)) return 0;
+  return ec_capacity(cfg);
+}
+
+moe_status moe_route_expert_choice(const moe_config* cfg, const float* logits, const float* bias,
+                                   float* scores_out, int32_t* tok, float* gate,
+                                   int32_t* slot_te, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = validate(cfg);
+  if (s != MOE_OK) return s;
+  if (!expert_choice(cfg)) return MOE_ERR_INVALID;
+  if (!logits || !tok || !gate || !slot_te) return MOE_ERR_INVALID;
+  if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
+  const Layout L = layout(cfg);
+  return run_route_ec(cfg, logits, 1, bias, at<float>(ws, L.sct), scores_out, nullptr, tok, gate,
+                      at<int32_t>(ws, L.perm), at<int32_t>(ws, L.offsets),
+                      at<int32_t>(ws, L.counts), slot_te, S_(stream));
 }
 
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
@@ -997,8 +1128,9 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const vo
   if (s != MOE_OK) return s;
   if (!w || !xn || !offsets || !perm_assign || !topk_gate || !y_assign) return MOE_ERR_INVALID;
   if ((s = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return s;
-  return run_ffn(cfg, w, xn, offsets, perm_assign, topk_gate, y_assign, y_shared, ws,
-                 S_(stream));
+  if (expert_choice(cfg)) return MOE_ERR_UNSUPPORTED;   // the layer forward only
+  return run_ffn(cfg, w, xn, offsets, RoutedRows{perm_assign, cfg->k, perm_assign}, topk_gate,
+                 y_assign, y_shared, ws, S_(stream));
 }
 
 moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32_t* slot_of,
@@ -1051,6 +1183,7 @@ const char* moe_status_string(moe_status s) {
 
 int32_t moe_layer_step_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
+  // expert choice: rmsnorm, router, scores, picks, [gather], gate/up, down, combine
   // rmsnorm, router, route, permute, [dequantise + gather], gate/up, down, combine
   return tc_experts(cfg) ? 8 : 7;
 }
@@ -1061,8 +1194,10 @@ int32_t moe_layer_launch_count(const moe_config* cfg) {
   // own launch, three for large batches, or none when it shares the routing
   // launch), and for tensor-core experts at wide tiles the row gather and (int8 /
   // int4) the one-pass dequantisation
-  const int perm = fused_route_permute(cfg) ? 0 : cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
   const int gather = tc_experts(cfg) && !gather_in_gemm(cfg) ? 1 : 0;
+  if (expert_choice(cfg))   // rmsnorm, router, scores, picks, gate/up, down, combine
+    return 7 + gather + (dequant_once(cfg) ? 1 : 0);
+  const int perm = fused_route_permute(cfg) ? 0 : cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
   return 6 + perm + gather + (dequant_once(cfg) ? 1 : 0);
 }
 

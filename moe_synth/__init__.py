@@ -71,6 +71,7 @@ class LayerShape:
     group_size: int = 128       # int4 group along K
     seed: int = 0
     tokens: Tuple[int, ...] = (64,)
+    routing: str = "topk"       # "topk" | "expert_choice"
 
     def with_(self, **kw) -> "LayerShape":
         return dataclasses.replace(self, **kw)

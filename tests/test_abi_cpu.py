@@ -151,3 +151,20 @@ def test_launch_and_step_counts(lib, preset, T, n):
     assert M.moe_layer_launch_count(cfg) == n
     # profiled steps: 7 for FP32 experts, 8 with the [dequantise + gather] step
     assert M.moe_layer_step_count(cfg) == (7 if sh.expert == "f32" else 8)
+
+
+def test_expert_choice_configuration_on_the_host(lib):
+    sh = moe_synth.PRESETS["olmoe"].with_(routing="expert_choice", bias_mode="logit")
+    cfg = M.make_config(sh, 4096)
+    assert M.moe_expert_choice_capacity(cfg) == 4096 * 8 // 64
+    assert M.moe_workspace_size(cfg) > 0
+    # rmsnorm, router, scores, picks, gather, gate/up, down, combine
+    assert M.moe_layer_launch_count(cfg) == 8
+    cfg.capacity_factor = 1.5
+    assert M.moe_expert_choice_capacity(cfg) == 768
+    # a selection-only bias and FP32 experts are refused; top-k configs have no C
+    assert M.moe_workspace_size(M.make_config(sh.with_(bias_mode="select"), 16)) == 0
+    assert M.moe_expert_choice_capacity(M.make_config(moe_synth.PRESETS["olmoe"], 16)) == 0
+    bad = M.make_config(sh, 16)
+    bad.routing = 2
+    assert M.moe_workspace_size(bad) == 0
