@@ -165,7 +165,10 @@ typedef struct moe_weights {
 size_t moe_workspace_size(const moe_config* cfg);
 
 /* Zero the device error word (asynchronous).  The pages have no counterpart:
- * it resets the failure report that moe_get_device_status reads. */
+ * it resets the failure report that moe_get_device_status reads, and the state
+ * the single-launch decode layer keeps in the workspace's first 256 bytes (its
+ * grid-barrier words).  Call it after a device error before the workspace is used
+ * again. */
 moe_status moe_clear_device_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Steps a1 + a2: RMSNorm and the router GEMM.
@@ -290,7 +293,13 @@ moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32
                        const float* y_shared, const void* residual, void* out,
                        void* stream);
 
-/* The whole layer: a1..a8 chained on one stream, no host synchronisation.
+/* The whole layer: a1..a8 on one stream, no host synchronisation.
+ * Decode batches (T <= 32) of bf16 experts with a bf16 router of at most 256
+ * experts and 16-byte aligned tensors run as ONE cooperative launch of one CTA per
+ * SM ("MoE: dynamism the compiler cannot remove", batch-1 section: the layer is
+ * launch bound at small batches), its steps separated by bounded grid-wide
+ * barriers in the workspace; every other configuration runs as a chain of
+ * kernels (moe_layer_launch_count).
  * Source: the whole chain of "MoE: dynamism the compiler cannot remove",
  * natural implementation (pre-norm, router, top-k, dispatch to the experts,
  * gated sum) with its capacity section, in the grouped form of that page's

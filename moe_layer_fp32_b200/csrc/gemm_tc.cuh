@@ -177,7 +177,7 @@ struct TcConfig {
       (EPI == EPI_DOWN && DIRECT) ? kEpiWarps * 32 * 20 * 4 : kEpiWarps * 128 * 8;
   static constexpr uint32_t SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + A_REGION + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+  static_assert(SMEM_BYTES + 64 <= 227 * 1024, "shared memory per CTA (dynamic + static)");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
   static_assert(!DIRECT || BN == 128, "direct tiles hold 128 tokens");
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 128-byte swizzle alignment");
@@ -429,15 +429,20 @@ MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float s
   }
 }
 
+// The grouped GEMM of one CTA over the work items cta, cta + ncta, ...: barrier
+// set-up in its shared memory (`smem`, 1024-byte aligned, C::SMEM_BYTES - 1024
+// bytes), the warp roles, and after an abort the drain of this CTA's copies still
+// in flight.  The caller has allocated C::TMEM_COLS columns of TMEM, whose address
+// is at *tmem_slot once the CTA has synchronised.  with_pdl: wait for the previous
+// kernel of the stream (programmatic dependent launch) before reading global
+// memory.  All threads of the CTA call it; it returns after a __syncthreads, with
+// every MMA it issued complete and every barrier idle.
 template <int EPI, int BN, bool DIRECT, int WQ>
-__global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
-    k_tc_gemm(const __grid_constant__ TcParams p) {
+MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_slot, int cta,
+                         int ncta, bool with_pdl) {
   using C = TcConfig<EPI, BN, DIRECT, WQ>;
   constexpr int NA = C::NA;
   constexpr int STAGES = C::STAGES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
   uint8_t* aslots = tiles + STAGES * C::STAGE_BYTES;   // dequantised weights (int8 / int4)
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(aslots + C::A_REGION);
@@ -447,8 +452,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
   uint64_t* drain_bar = tempty_bar + 2;       // [1]
   uint64_t* deq_bar = drain_bar + 1;          // [2] dequantised slot filled
   uint64_t* aempty_bar = deq_bar + 2;         // [2] dequantised slot consumed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aempty_bar + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(aempty_bar + 2) + 1;
   int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
   int* prefix = reinterpret_cast<int*>(
       reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
@@ -478,10 +482,6 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
-  }
   if (warp == 0 && lane == 0) {
     for (int pi = 0; pi < p.n_prob; ++pi) {
       tma_prefetch_desc(&p.prob[pi].tmA);
@@ -491,8 +491,10 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
   }
   // everything above touched only this CTA's shared memory, TMEM and the kernel
   // parameters; from here on the previous kernel's outputs are read
-  pdl_wait();
-  pdl_trigger();
+  if (with_pdl) {
+    pdl_wait();
+    pdl_trigger();
+  }
   if (warp >= 2 && warp - 2 < p.n_prob) {
     const TcProblem& P = p.prob[warp - 2];
     group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1));
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
   if (kCanSplit && p.split_part != nullptr && out_tiles > 0) {
     int kbmin = p.prob[0].K / 64;
     if (p.n_prob > 1 && p.prob[1].K / 64 < kbmin) kbmin = p.prob[1].K / 64;
-    S = (int)gridDim.x / out_tiles;
+    S = ncta / out_tiles;
     if (S > kMaxSplit) S = kMaxSplit;
     if (S > kbmin / 2) S = kbmin / 2;
     if (S < 1) S = 1;
@@ -563,7 +565,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
     bool ok = true;
     if (!any_gather) {
       if (lane == 0) {
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int tile = cta; tile < total && ok; tile += ncta) {
           TileInfo ti;
           decode_work(p, prefix, BN, TN, S, tile, ti);
           const TcProblem& P = p.prob[ti.prob];
@@ -575,7 +577,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
         }
       }
     } else {
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = cta; tile < total && ok; tile += ncta) {
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
         const TcProblem& P = p.prob[ti.prob];
@@ -615,7 +617,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = cta; tile < total && ok; tile += ncta) {
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag, p.wait_cycles)) break;
@@ -675,7 +677,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
       int aslot = 0;
       uint32_t aphase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = cta; tile < total && ok; tile += ncta) {
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
@@ -706,7 +708,7 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
     float* s_scale = epi_scale + (warp - 2) * 128;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int tile = cta; tile < total; tile += ncta) {
       TileInfo ti;
       decode_work(p, prefix, BN, TN, S, tile, ti);
       const TcProblem& P = p.prob[ti.prob];
@@ -850,9 +852,24 @@ __global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+}
+
+template <int EPI, int BN, bool DIRECT, int WQ>
+__global__ void __launch_bounds__(TcConfig<EPI, BN, DIRECT, WQ>::THREADS, 1)
+    k_tc_gemm(const __grid_constant__ TcParams p) {
+  using C = TcConfig<EPI, BN, DIRECT, WQ>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_slot;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if ((threadIdx.x >> 5) == 1) {
+    tmem_alloc(&tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_gemm_run<EPI, BN, DIRECT, WQ>(p, smem, &tmem_slot, blockIdx.x, gridDim.x, true);
+  if ((threadIdx.x >> 5) == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    tmem_dealloc(tmem_slot, C::TMEM_COLS);
   }
 }
 

@@ -105,25 +105,23 @@ MOE_DEV void unpack8(const uint4& u, float (&f)[8]) {
   for (int i = 0; i < 4; ++i) { f[2 * i] = __low2float(h[i]); f[2 * i + 1] = __high2float(h[i]); }
 }
 
-template <int MAXV>
-__global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __restrict__ x,
-                                                       const float* __restrict__ gamma,
-                                                       __nv_bfloat16* __restrict__ xn, int d,
-                                                       double eps, int32_t* __restrict__ zero,
-                                                       int nzero) {
-  pdl_wait();
-  pdl_trigger();
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
-  __shared__ double red[8];
+// One token row, vectorised: thread i of the NT calling threads keeps up to MAXV
+// 16-byte vectors of the row in registers between the sum of squares and the
+// scaling pass (d up to NT * MAXV * 8).  `red` is a shared scratch of NT / 32
+// doubles.  Same arithmetic as k_rmsnorm; all NT threads call it.
+template <int NT, int MAXV>
+MOE_DEV void rmsnorm_row_bf16v(const __nv_bfloat16* __restrict__ xrow,
+                               const float* __restrict__ gamma,
+                               __nv_bfloat16* __restrict__ xnrow, int d, double eps,
+                               double* red) {
   const int nv = d / 8;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)blockIdx.x * d);
-  uint4* outr = reinterpret_cast<uint4*>(xn + (size_t)blockIdx.x * d);
+  const uint4* xr = reinterpret_cast<const uint4*>(xrow);
+  uint4* outr = reinterpret_cast<uint4*>(xnrow);
   uint4 buf[MAXV];
   double s = 0.0;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
-    const int v = threadIdx.x + i * 256;
+    const int v = threadIdx.x + i * NT;
     if (v < nv) {
       buf[i] = xr[v];
       float f[8];
@@ -137,11 +135,11 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __re
   __syncthreads();
   double tot = 0.0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) tot += red[w];
+  for (int w = 0; w < NT / 32; ++w) tot += red[w];
   const double r = 1.0 / sqrt(tot / d + eps);
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
-    const int v = threadIdx.x + i * 256;
+    const int v = threadIdx.x + i * NT;
     if (v < nv) {
       float f[8];
       unpack8(buf[i], f);
@@ -155,6 +153,22 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __re
       outr[v] = o;
     }
   }
+  __syncthreads();   // red may be reused
+}
+
+template <int MAXV>
+__global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __restrict__ x,
+                                                       const float* __restrict__ gamma,
+                                                       __nv_bfloat16* __restrict__ xn, int d,
+                                                       double eps, int32_t* __restrict__ zero,
+                                                       int nzero) {
+  pdl_wait();
+  pdl_trigger();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
+  __shared__ double red[8];
+  rmsnorm_row_bf16v<256, MAXV>(x + (size_t)blockIdx.x * d, gamma, xn + (size_t)blockIdx.x * d, d,
+                               eps, red);
 }
 
 // ---------------------------------------------------------------------------
@@ -207,20 +221,19 @@ __global__ void __launch_bounds__(256) k_router_split(const TA* __restrict__ xn,
 // arithmetic.  Thread t always meets the same 8-column group (256 is a multiple
 // of E/8), keeps TT x 8 partial sums in registers, and the threads of a column
 // group are summed in a fixed order through shared memory.
-template <int TT>
-__global__ void __launch_bounds__(256) k_router_vec(const __nv_bfloat16* __restrict__ xn,
-                                                    const __nv_bfloat16* __restrict__ wr,
-                                                    float* __restrict__ part, int T, int d,
-                                                    int E, int rows) {
-  extern __shared__ float sm_r[];
+// One router tile for TT tokens from t0 and K-slice `slice` of `rows` rows, by
+// the first 256 of the calling threads (every calling thread must call it; NT is
+// their number).  sm_r: TT * rows + 256 * 8 floats of shared memory.
+template <int TT, int NT>
+MOE_DEV void router_vec_tile(const __nv_bfloat16* __restrict__ xn,
+                             const __nv_bfloat16* __restrict__ wr, float* __restrict__ part,
+                             int T, int d, int E, int rows, int t0, int slice, float* sm_r) {
   float* xs = sm_r;                      // [TT][rows]
   float* red = sm_r + TT * rows;         // [256][8]
-  pdl_wait();
-  pdl_trigger();
-  const int t0 = blockIdx.x * TT;
-  const int k0 = blockIdx.y * rows;
+  const int tid = threadIdx.x;
+  const int k0 = slice * rows;
   const int kn = min(rows, d - k0);
-  for (int i = threadIdx.x; i < TT * rows; i += 256) {
+  for (int i = tid; i < TT * rows; i += NT) {
     const int tt = i / rows, kk = i % rows;
     xs[i] = (t0 + tt < T && kk < kn) ? __bfloat162float(xn[(size_t)(t0 + tt) * d + k0 + kk]) : 0.f;
   }
@@ -233,25 +246,27 @@ __global__ void __launch_bounds__(256) k_router_vec(const __nv_bfloat16* __restr
   for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[tt][j] = 0.f;
-  for (int v0 = threadIdx.x; v0 < nvec; v0 += 4 * 256) {
-    uint4 w[4];
+  if (tid < 256) {
+    for (int v0 = tid; v0 < nvec; v0 += 4 * 256) {
+      uint4 w[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int v = v0 + u * 256;
-      w[u] = v < nvec ? wv[v] : make_uint4(0, 0, 0, 0);
-    }
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * 256;
+        w[u] = v < nvec ? wv[v] : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int v = v0 + u * 256;
-      if (v < nvec) {
-        float f[8];
-        unpack8(w[u], f);
-        const int i = v / cgs;
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * 256;
+        if (v < nvec) {
+          float f[8];
+          unpack8(w[u], f);
+          const int i = v / cgs;
 #pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
-          const float x = xs[tt * rows + i];
+          for (int tt = 0; tt < TT; ++tt) {
+            const float x = xs[tt * rows + i];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[tt][j] = fmaf(x, f[j], acc[tt][j]);
+            for (int j = 0; j < 8; ++j) acc[tt][j] = fmaf(x, f[j], acc[tt][j]);
+          }
         }
       }
     }
@@ -259,17 +274,36 @@ __global__ void __launch_bounds__(256) k_router_vec(const __nv_bfloat16* __restr
   const int per = 256 / cgs;   // threads per column group
   for (int tt = 0; tt < TT; ++tt) {
     if (t0 + tt >= T) break;
+    if (tid < 256) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) red[threadIdx.x * 8 + j] = acc[tt][j];
+      for (int j = 0; j < 8; ++j) red[tid * 8 + j] = acc[tt][j];
+    }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += 256) {
+    for (int e = tid; e < E; e += NT) {
       const int g = e / 8, j = e % 8;
       float s = 0.f;
       for (int m = 0; m < per; ++m) s += red[(g + m * cgs) * 8 + j];
-      part[((size_t)blockIdx.y * T + t0 + tt) * E + e] = s;
+      part[((size_t)slice * T + t0 + tt) * E + e] = s;
     }
     __syncthreads();
   }
+}
+
+// a2 for small batches with a bf16 router: CTA (blockIdx.x, blockIdx.y) takes TT
+// tokens and `rows` consecutive rows of W_r -- one contiguous block of rows * E
+// bf16 -- streamed as 16-byte vectors, every load of a thread issued before its
+// arithmetic.  Thread t always meets the same 8-column group (256 is a multiple
+// of E/8), keeps TT x 8 partial sums in registers, and the threads of a column
+// group are summed in a fixed order through shared memory.
+template <int TT>
+__global__ void __launch_bounds__(256) k_router_vec(const __nv_bfloat16* __restrict__ xn,
+                                                    const __nv_bfloat16* __restrict__ wr,
+                                                    float* __restrict__ part, int T, int d,
+                                                    int E, int rows) {
+  extern __shared__ float sm_r[];
+  pdl_wait();
+  pdl_trigger();
+  router_vec_tile<TT, 256>(xn, wr, part, T, d, E, rows, blockIdx.x * TT, blockIdx.y, sm_r);
 }
 
 // ---------------------------------------------------------------------------
@@ -887,21 +921,16 @@ MOE_DEV void storev(__nv_bfloat16* p, const float (&v)[VEC]) {
   }
 }
 
+// Element group i (token i / (d / VEC), VEC columns) of the combine.  The rows of
+// JB assignments are loaded together, unconditionally (a dropped slot's row is
+// read but not added; past k the token's first row is re-read), so that their
+// memory latencies overlap; the adds then follow in j order.
 template <typename TA, typename TO, typename TY, int VEC>
-__global__ void __launch_bounds__(256) k_combine(const TY* __restrict__ y,
-                                                 const int32_t* __restrict__ slot_of,
-                                                 const float* __restrict__ ys, int S,
-                                                 const TA* __restrict__ res, TO* __restrict__ out,
-                                                 int T, int d, int k) {
-  pdl_wait();
-  pdl_trigger();
-  // The rows of JB assignments are loaded together, unconditionally (a dropped
-  // slot's row is read but not added; past k the token's first row is re-read), so
-  // that their memory latencies overlap; the adds then follow in j order.
+MOE_DEV void combine_elems(const TY* __restrict__ y, const int32_t* __restrict__ slot_of,
+                           const float* __restrict__ ys, int S, const TA* __restrict__ res,
+                           TO* __restrict__ out, int T, int d, int k, size_t i) {
   constexpr int JB = 8;
   const int q = d / VEC;
-  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (size_t)T * q) return;
   const int t = (int)(i / q);
   const int c = (int)(i % q) * VEC;
   float acc[VEC];
@@ -931,6 +960,19 @@ __global__ void __launch_bounds__(256) k_combine(const TY* __restrict__ y,
       }
   }
   storev<VEC>(out + (size_t)t * d + c, acc);
+}
+
+template <typename TA, typename TO, typename TY, int VEC>
+__global__ void __launch_bounds__(256) k_combine(const TY* __restrict__ y,
+                                                 const int32_t* __restrict__ slot_of,
+                                                 const float* __restrict__ ys, int S,
+                                                 const TA* __restrict__ res, TO* __restrict__ out,
+                                                 int T, int d, int k) {
+  pdl_wait();
+  pdl_trigger();
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (size_t)T * (d / VEC)) return;
+  combine_elems<TA, TO, TY, VEC>(y, slot_of, ys, S, res, out, T, d, k, i);
 }
 
 // ---------------------------------------------------------------------------

@@ -15,6 +15,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_pair.cuh"
 #include "kernels_ec.cuh"
+#include "decode_layer.cuh"
 
 using namespace moe;
 
@@ -362,6 +363,29 @@ moe_status launch_tc(const TcParams& p, cudaStream_t st) {
 #endif
 constexpr bool kPairTiles = MOE_PAIR_TILES != 0;
 
+// CTA pairs that can be resident at once.  A cluster's two CTAs must sit in one
+// GPC, so a GPC with an odd number of free SMs leaves one idle: the persistent
+// grid must not ask for more pairs than fit, or the last ones would run as a
+// second wave after the others have finished their share of the tiles.
+template <int EPI>
+int resident_pairs() {
+  static int cached[8] = {};   // per device, on first use
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 8 && cached[dev] > 0) return cached[dev];
+  using C = PairConfig<EPI>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms() / 2 * 2);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (void*)k_tc_gemm_pair<EPI>, &cfg) != cudaSuccess || n < 1)
+    n = 0;
+  if (n > num_sms() / 2) n = num_sms() / 2;
+  if (dev < 8 && n > 0) cached[dev] = n;
+  return n;
+}
+
 template <int EPI>
 moe_status launch_pair(const TcParams& p, cudaStream_t st) {
   using C = PairConfig<EPI>;
@@ -369,8 +393,9 @@ moe_status launch_pair(const TcParams& p, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  // an even number of CTAs: one cluster of two per pair of SMs
-  MOE_LAUNCH((kern), num_sms() / 2 * 2, C::THREADS, C::SMEM_BYTES, st, p);
+  const int pairs = resident_pairs<EPI>();
+  if (pairs < 1) return MOE_ERR_CUDA;
+  MOE_LAUNCH((kern), 2 * pairs, C::THREADS, C::SMEM_BYTES, st, p);
   return check_launch();
 }
 
@@ -597,6 +622,127 @@ struct RoutedRows {
   const int32_t* dst;
 };
 
+// Parameters of the grouped gate/up GEMM: the routed problem (rows gathered by the
+// GEMM from xn through rr.src, or read from the gathered rows xp) and the shared
+// experts' problem (every token of xn).
+moe_status gateup_params(const moe_config* c, const moe_weights* w, const moe_weights& wl, int wq,
+                         const void* xn, const void* xp, const int32_t* offsets, RoutedRows rr,
+                         __nv_bfloat16* h, float* split_part, int32_t* split_cnt, int32_t* err,
+                         TcParams& p) {
+  const int T = c->T, S = c->n_shared, bn = pick_bn(c), R = (int)n_slots(c);
+  const bool g4 = gather_in_gemm(c);
+  p = TcParams{};
+  TcProblem& P = p.prob[0];
+  if (!map_expert(&P.tmA, wq, wl.w_gate, c->E, c->d, c->f)) return MOE_ERR_CUDA;
+  if (!map_expert(&P.tmA2, wq, wl.w_up, c->E, c->d, c->f)) return MOE_ERR_CUDA;
+  if (g4) {
+    // routed rows: slot s reads token perm[s] / k of xn, four rows per copy
+    if (!map_rows(&P.tmB, xn, T, c->d, 1)) return MOE_ERR_CUDA;
+    P.gather_rows = rr.src;
+    P.gather_k = rr.src_k;
+  } else if (!map_rows(&P.tmB, xp, R, c->d, bn)) {
+    return MOE_ERR_CUDA;
+  }
+  if (wq != WQ_BF16 && (!map_scales(&P.tmS, c, w->s_gate, c->E, c->d, c->f) ||
+                        !map_scales(&P.tmS2, c, w->s_up, c->E, c->d, c->f)))
+    return MOE_ERR_CUDA;
+  P.offsets = offsets;
+  P.G = c->E;
+  P.N = c->f;
+  P.K = c->d;
+  P.out = h;
+  P.out_row_base = 0;
+  P.ld_out = c->f;
+  P.n_valid = c->f;
+  p.n_prob = 1;
+  if (S > 0) {
+    TcProblem& Q = p.prob[1];
+    if (!map_expert(&Q.tmA, wq, wl.sh_gate, S, c->d, c->f)) return MOE_ERR_CUDA;
+    if (!map_expert(&Q.tmA2, wq, wl.sh_up, S, c->d, c->f)) return MOE_ERR_CUDA;
+    if (!map_rows(&Q.tmB, xn, T, c->d, bn)) return MOE_ERR_CUDA;
+    if (wq != WQ_BF16 && (!map_scales(&Q.tmS, c, w->sh_s_gate, S, c->d, c->f) ||
+                          !map_scales(&Q.tmS2, c, w->sh_s_up, S, c->d, c->f)))
+      return MOE_ERR_CUDA;
+    Q.offsets = nullptr;
+    Q.G = S;
+    Q.uniform_rows = T;
+    Q.b_row_base = 0;
+    Q.b_group_stride = 0;
+    Q.N = c->f;
+    Q.K = c->d;
+    Q.out = h;
+    Q.out_row_base = (size_t)R;
+    Q.ld_out = c->f;
+    Q.n_valid = c->f;
+    p.n_prob = 2;
+  }
+  p.err = err;
+  p.wait_cycles = wait_cycles(c);
+  p.split_part = split_part;
+  p.split_cnt = split_cnt;
+  return MOE_OK;
+}
+
+// Parameters of the grouped down GEMM: routed rows of h to rows rr.dst of y scaled
+// by their gate, and the shared experts' rows of h to ys.
+moe_status down_params(const moe_config* c, const moe_weights* w, const moe_weights& wl, int wq,
+                       const int32_t* offsets, RoutedRows rr, const float* gate,
+                       const __nv_bfloat16* h, void* y, bool rows_bf16, float* ys,
+                       float* split_part, int32_t* split_cnt, int32_t* err, TcParams& p) {
+  const int T = c->T, S = c->n_shared, bn = pick_bn(c), R = (int)n_slots(c);
+  const int32_t* perm = rr.dst;
+  p = TcParams{};
+  TcProblem& P = p.prob[0];
+  if (!map_expert(&P.tmA, wq, wl.w_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
+  P.tmA2 = P.tmA;
+  if (wq != WQ_BF16) {
+    if (!map_scales(&P.tmS, c, w->s_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
+    P.tmS2 = P.tmS;
+  }
+  if (!map_rows(&P.tmB, h, R + S * T, c->f, bn)) return MOE_ERR_CUDA;
+  P.offsets = offsets;
+  P.G = c->E;
+  P.N = c->d;
+  P.K = c->f;
+  P.out = y;
+  P.out_bf16 = rows_bf16 ? 1 : 0;
+  P.out_row_base = 0;
+  P.ld_out = c->d;
+  P.perm_assign = perm;
+  P.gate = gate;
+  P.n_valid = c->d;
+  p.n_prob = 1;
+  if (S > 0) {
+    TcProblem& Q = p.prob[1];
+    if (!map_expert(&Q.tmA, wq, wl.sh_down, S, c->f, c->d)) return MOE_ERR_CUDA;
+    Q.tmA2 = Q.tmA;
+    if (wq != WQ_BF16) {
+      if (!map_scales(&Q.tmS, c, w->sh_s_down, S, c->f, c->d)) return MOE_ERR_CUDA;
+      Q.tmS2 = Q.tmS;
+    }
+    Q.tmB = P.tmB;
+    Q.offsets = nullptr;
+    Q.G = S;
+    Q.uniform_rows = T;
+    Q.b_row_base = R;
+    Q.b_group_stride = T;
+    Q.N = c->d;
+    Q.K = c->f;
+    Q.out = ys;
+    Q.out_row_base = 0;
+    Q.ld_out = c->d;
+    Q.perm_assign = nullptr;
+    Q.gate = nullptr;
+    Q.n_valid = c->d;
+    p.n_prob = 2;
+  }
+  p.err = err;
+  p.wait_cycles = wait_cycles(c);
+  p.split_part = split_part;
+  p.split_cnt = split_cnt;
+  return MOE_OK;
+}
+
 moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
                    const int32_t* offsets, RoutedRows rr, const float* gate, void* y,
                    float* ys, void* ws, cudaStream_t st, Marks* mk = nullptr,
@@ -706,109 +852,19 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   }
   mk->mark(st);   // end of the (optional) dequantisation and gather step
   {
-    TcParams p{};
-    TcProblem& P = p.prob[0];
-    if (!map_expert(&P.tmA, wq, wl.w_gate, c->E, c->d, c->f)) return MOE_ERR_CUDA;
-    if (!map_expert(&P.tmA2, wq, wl.w_up, c->E, c->d, c->f)) return MOE_ERR_CUDA;
-    if (g4) {
-      // routed rows: slot s reads token perm[s] / k of xn, four rows per copy
-      if (!map_rows(&P.tmB, xn, T, c->d, 1)) return MOE_ERR_CUDA;
-      P.gather_rows = rr.src;
-      P.gather_k = rr.src_k;
-    } else if (!map_rows(&P.tmB, xp, R, c->d, bn)) {
-      return MOE_ERR_CUDA;
-    }
-    if (wq != WQ_BF16 && (!map_scales(&P.tmS, c, w->s_gate, c->E, c->d, c->f) ||
-                          !map_scales(&P.tmS2, c, w->s_up, c->E, c->d, c->f)))
-      return MOE_ERR_CUDA;
-    P.offsets = offsets;
-    P.G = c->E;
-    P.N = c->f;
-    P.K = c->d;
-    P.out = h;
-    P.out_row_base = 0;
-    P.ld_out = c->f;
-    P.n_valid = c->f;
-    p.n_prob = 1;
-    if (S > 0) {
-      TcProblem& Q = p.prob[1];
-      if (!map_expert(&Q.tmA, wq, wl.sh_gate, S, c->d, c->f)) return MOE_ERR_CUDA;
-      if (!map_expert(&Q.tmA2, wq, wl.sh_up, S, c->d, c->f)) return MOE_ERR_CUDA;
-      if (!map_rows(&Q.tmB, xn, T, c->d, bn)) return MOE_ERR_CUDA;
-      if (wq != WQ_BF16 && (!map_scales(&Q.tmS, c, w->sh_s_gate, S, c->d, c->f) ||
-                            !map_scales(&Q.tmS2, c, w->sh_s_up, S, c->d, c->f)))
-        return MOE_ERR_CUDA;
-      Q.offsets = nullptr;
-      Q.G = S;
-      Q.uniform_rows = T;
-      Q.b_row_base = 0;
-      Q.b_group_stride = 0;
-      Q.N = c->f;
-      Q.K = c->d;
-      Q.out = h;
-      Q.out_row_base = (size_t)R;
-      Q.ld_out = c->f;
-      Q.n_valid = c->f;
-      p.n_prob = 2;
-    }
-    p.err = err;
-    p.wait_cycles = wait_cycles(c);
-    p.split_part = split_part;
-    p.split_cnt = split_cnt;
+    TcParams p;
+    if ((s = gateup_params(c, w, wl, wq, xn, xp, offsets, rr, h, split_part, split_cnt, err, p)) !=
+        MOE_OK)
+      return s;
     s = launch_tc_bn<EPI_GATEUP>(bn, wq, p, st);
     if (s != MOE_OK) return s;
     mk->mark(st);
   }
   {
-    TcParams p{};
-    TcProblem& P = p.prob[0];
-    if (!map_expert(&P.tmA, wq, wl.w_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
-    P.tmA2 = P.tmA;
-    if (wq != WQ_BF16) {
-      if (!map_scales(&P.tmS, c, w->s_down, c->E, c->f, c->d)) return MOE_ERR_CUDA;
-      P.tmS2 = P.tmS;
-    }
-    if (!map_rows(&P.tmB, h, R + S * T, c->f, bn)) return MOE_ERR_CUDA;
-    P.offsets = offsets;
-    P.G = c->E;
-    P.N = c->d;
-    P.K = c->f;
-    P.out = y;
-    P.out_bf16 = rows_bf16 ? 1 : 0;
-    P.out_row_base = 0;
-    P.ld_out = c->d;
-    P.perm_assign = perm;
-    P.gate = gate;
-    P.n_valid = c->d;
-    p.n_prob = 1;
-    if (S > 0) {
-      TcProblem& Q = p.prob[1];
-      if (!map_expert(&Q.tmA, wq, wl.sh_down, S, c->f, c->d)) return MOE_ERR_CUDA;
-      Q.tmA2 = Q.tmA;
-      if (wq != WQ_BF16) {
-        if (!map_scales(&Q.tmS, c, w->sh_s_down, S, c->f, c->d)) return MOE_ERR_CUDA;
-        Q.tmS2 = Q.tmS;
-      }
-      Q.tmB = P.tmB;
-      Q.offsets = nullptr;
-      Q.G = S;
-      Q.uniform_rows = T;
-      Q.b_row_base = R;
-      Q.b_group_stride = T;
-      Q.N = c->d;
-      Q.K = c->f;
-      Q.out = ys;
-      Q.out_row_base = 0;
-      Q.ld_out = c->d;
-      Q.perm_assign = nullptr;
-      Q.gate = nullptr;
-      Q.n_valid = c->d;
-      p.n_prob = 2;
-    }
-    p.err = err;
-    p.wait_cycles = wait_cycles(c);
-    p.split_part = split_part;
-    p.split_cnt = split_cnt;
+    TcParams p;
+    if ((s = down_params(c, w, wl, wq, offsets, rr, gate, h, y, rows_bf16, ys, split_part,
+                         split_cnt, err, p)) != MOE_OK)
+      return s;
     s = launch_tc_bn<EPI_DOWN>(bn, wq, p, st);
     mk->mark(st);
   }
@@ -907,6 +963,110 @@ moe_status run_route_ec(const moe_config* c, const float* part, int ns, const fl
   return check_launch();
 }
 
+// ------------------------------------------------------ single-launch decode layer
+// Offset of the decode kernel's grid-barrier words in the workspace (inside the
+// first 256 bytes, which moe_clear_device_status zeroes).
+constexpr size_t kGridBarOff = 64;
+
+// The whole layer in one cooperative launch: decode batches (T <= 32) of bf16
+// experts with a bf16 router of at most 256 experts, 16-byte aligned tensors.
+bool single_launch(const moe_config* c) {
+  return !expert_choice(c) && c->T <= kDecodeMaxT && c->expert_dtype == MOE_BF16 &&
+         vec_router(c) && c->E <= 256 && gather_in_gemm(c) && c->d <= kDecodeThreads * 4 * 8;
+}
+
+template <int EPL, int BN>
+moe_status launch_decode(const DecodeParams& dp, cudaStream_t st) {
+  using CG = TcConfig<EPI_GATEUP, BN, false, WQ_BF16>;
+  using CD = TcConfig<EPI_DOWN, BN, false, WQ_BF16>;
+  constexpr uint32_t smem = CG::SMEM_BYTES > CD::SMEM_BYTES ? CG::SMEM_BYTES : CD::SMEM_BYTES;
+  auto kern = k_decode_layer<EPL, BN, 4>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  // every CTA must be resident at once (the grid barriers): one per SM
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecodeThreads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return MOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeCooperative;
+  a[0].val.cooperative = 1;
+  cfg.attrs = a;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, dp) != cudaSuccess) return MOE_ERR_CUDA;
+  return check_launch();
+}
+
+moe_status run_decode_layer(const moe_config* c, const moe_weights* w, const void* x, void* out,
+                            void* ws, float* logits_out, int32_t* idx, int32_t* counts,
+                            cudaStream_t st) {
+  const Layout L = layout(c);
+  DecodeParams dp{};
+  int32_t* err = at<int32_t>(ws, L.err);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  float* gate = at<float>(ws, L.gate);
+  __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
+  void* xn = at<void>(ws, L.xn);
+  void* y = at<void>(ws, L.y);
+  float* ys = c->n_shared ? at<float>(ws, L.ys) : nullptr;
+  const RoutedRows rr{perm, c->k, perm};
+  moe_status s;
+  if ((s = gateup_params(c, w, *w, WQ_BF16, xn, nullptr, offsets, rr, h, nullptr, nullptr, err,
+                         dp.gu)) != MOE_OK)
+    return s;
+  if ((s = down_params(c, w, *w, WQ_BF16, offsets, rr, gate, h, y, true, ys, nullptr, nullptr,
+                       err, dp.dn)) != MOE_OK)
+    return s;
+  dp.x = static_cast<const __nv_bfloat16*>(x);
+  dp.gamma = static_cast<const float*>(w->rms_gamma);
+  dp.w_router = static_cast<const __nv_bfloat16*>(w->w_router);
+  dp.bias = static_cast<const float*>(w->router_bias);
+  dp.xn = static_cast<__nv_bfloat16*>(xn);
+  dp.part = at<float>(ws, L.part);
+  dp.idx = idx;
+  dp.gate = gate;
+  dp.counts = counts;
+  dp.offsets = offsets;
+  dp.perm = perm;
+  dp.slot = at<int32_t>(ws, L.slot);
+  dp.dropped = at<int32_t>(ws, L.dropped);
+  dp.logits_out = logits_out;
+  dp.y = static_cast<const __nv_bfloat16*>(y);
+  dp.ys = ys;
+  dp.out = out;
+  dp.out_f32 = c->out_dtype == MOE_F32 ? 1 : 0;
+  dp.err = err;
+  dp.grid_bar = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kGridBarOff);
+  dp.wait_cycles = wait_cycles(c);
+  dp.eps = (double)c->rms_eps;
+  dp.T = c->T;
+  dp.d = c->d;
+  dp.E = c->E;
+  dp.k = c->k;
+  dp.S = c->n_shared;
+  dp.mode = c->bias_mode;
+  dp.renorm = c->renormalize ? 1 : 0;
+  dp.cap = capacity_rows(c);
+  dp.ns = L.ns;
+  dp.rows = kRouterSlice;
+  const int bn = pick_bn(c);
+#define MOE_DECODE(EPL)                                                        \
+  return bn == 16 ? launch_decode<EPL, 16>(dp, st) : launch_decode<EPL, 32>(dp, st)
+  if (c->E <= 32) MOE_DECODE(1);
+  if (c->E <= 64) MOE_DECODE(2);
+  if (c->E <= 128) MOE_DECODE(4);
+  MOE_DECODE(8);
+#undef MOE_DECODE
+}
+
 moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const void* x,
                               void* out, void* ws, size_t ws_bytes, float* logits_out,
                               int32_t* topk_idx_out, int32_t* counts_out, cudaStream_t st,
@@ -928,6 +1088,14 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
   int32_t* slot = at<int32_t>(ws, L.slot);
   void* y = at<void>(ws, L.y);
   float* ys = cfg->n_shared ? at<float>(ws, L.ys) : nullptr;
+  if (!mk->ev && single_launch(cfg)) {
+    auto a16 = [](const void* q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    const void* ops[] = {x, out, w->rms_gamma, w->w_router, w->w_gate, w->w_up, w->w_down,
+                         w->sh_gate, w->sh_up, w->sh_down};
+    bool aligned = true;
+    for (const void* o : ops) aligned = aligned && a16(o);
+    if (aligned) return run_decode_layer(cfg, w, x, out, ws, logits_out, idx, counts, st);
+  }
   mk->mark(st);
   int32_t* split_cnt = split_k(cfg) ? at<int32_t>(ws, L.splitcnt) : nullptr;
   if ((s = run_rmsnorm(cfg, w, x, xn, st, split_cnt, split_cnt ? split_counters() : 0)) !=
@@ -1016,7 +1184,9 @@ size_t moe_workspace_size(const moe_config* cfg) {
 
 moe_status moe_clear_device_status(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < 16) return MOE_ERR_WORKSPACE;
-  return cudaMemsetAsync(ws, 0, 16, S_(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  // the error word, and the single-launch decode layer's grid-barrier words
+  const size_t n = ws_bytes < 256 ? 16 : 256;
+  return cudaMemsetAsync(ws, 0, n, S_(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_rmsnorm_router(const moe_config* cfg, const moe_weights* w, const void* x,
@@ -1190,6 +1360,7 @@ int32_t moe_layer_step_count(const moe_config* cfg) {
 
 int32_t moe_layer_launch_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
+  if (single_launch(cfg)) return 1;   // with 16-byte aligned tensors
   // rmsnorm, router, route, gate/up, down and combine, plus the permutation (its
   // own launch, three for large batches, or none when it shares the routing
   // launch), and for tensor-core experts at wide tiles the row gather and (int8 /

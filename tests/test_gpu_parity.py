@@ -415,3 +415,42 @@ def test_misaligned_tensors():
     with pytest.raises(M.MoeError) as e:
         M.moe_grouped_ffn(cfg, w, xn, offs, perm, gate, y, ys, ws)
     assert e.value.status == M.MOE_ERR_INVALID
+
+
+# --------------------------------------------------------------------- single launch
+DECODE_ONE_LAUNCH = {
+    "olmoe_like": (LayerShape("d1", d=2048, E=64, k=8, f=1024, bias_mode="logit", seed=51), 1),
+    "shared_cap": (LayerShape("d2", d=1024, E=32, k=6, f=512, n_shared=2, capacity_factor=1.0,
+                              seed=52), 32),
+    "select_256": (LayerShape("d3", d=768, E=256, k=8, f=256, n_shared=1, bias_mode="select",
+                              seed=53), 17),
+    "wide_tiles": (LayerShape("d4", d=512, E=8, k=8, f=384, seed=54), 32),
+}
+
+
+@pytest.mark.parametrize("name", list(DECODE_ONE_LAUNCH))
+def test_single_launch_decode_layer_equals_the_kernel_chain(name):
+    """Decode batches of bf16 experts run as one cooperative launch; the profiled
+    entry point runs the same layer as a chain of kernels.  The two give the same
+    bits (the RMSNorm sum of squares of bf16 inputs is exact in double, and the
+    GEMM tiles are the same), the same routes, and the oracle's result."""
+    sh, T = DECODE_ONE_LAUNCH[name]
+    li, x, dli, dx = inputs_on_device(sh, T)
+    layer = M.MoELayer(dli, T, out_dtype="f32")
+    assert M.moe_layer_launch_count(layer.cfg) == 1
+    idx = torch.empty(T, sh.k, dtype=torch.int32, device="cuda")
+    one = layer.forward(dx, topk_idx=idx).clone()
+    assert M.moe_get_device_status(layer.ws) == 0
+    evs = [torch.cuda.Event(enable_timing=True)
+           for _ in range(M.moe_layer_step_count(layer.cfg) + 1)]
+    chain = torch.empty_like(one)
+    M.moe_layer_forward_profiled(layer.cfg, layer.w, dx, chain, layer.ws, evs)
+    assert M.moe_get_device_status(layer.ws) == 0
+    assert torch.equal(one, chain)
+    # and twice in a row (the grid-barrier words are left ready for the next call)
+    again = layer.forward(dx)
+    assert torch.equal(again, one)
+    res = run_layer(sh, T)
+    assert res.max_margin_mismatch < ROUTE_MARGIN
+    assert res.err_ratio <= TOL[sh.expert], res.err_ratio
+    print(f"{name}: err/rms(out) {res.err_ratio:.3e}, err/rms(delta) {res.err_ratio_delta:.3e}")
