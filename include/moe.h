@@ -123,18 +123,20 @@ typedef struct moe_config {
  *   rms_gamma   [d] float32
  *   w_router    [d, E]            router dtype
  *   router_bias [E] float32, or NULL (required unless bias_mode == NONE)
- *   w_gate/w_up [E, d, f]         F32/BF16: that type; INT8: int8; FP8: uint8 E4M3 codes;
- *                                 INT4: uint8 [E, d, f/2]
- *   w_down      [E, f, d]         the same; INT4: uint8 [E, f, d/2]
+ *   w_gate/w_up F32/BF16: [E, d, f] of that type (W[k][n], n contiguous).
+ *               INT8: int8 [E, f, d]; FP8: uint8 E4M3 codes [E, f, d]; INT4: uint8
+ *               [E, f, d/2] -- quantised codes are stored transposed, the reduction
+ *               dim d contiguous (code q[n][k] is weight W[k][n])
+ *   w_down      F32/BF16: [E, f, d]; INT8 / FP8: [E, d, f]; INT4: uint8 [E, d, f/2]
  *   s_gate/s_up INT8, FP8: bf16 [E, f]; INT4: bf16 [E, d/128, f]; otherwise NULL
  *   s_down      INT8, FP8: bf16 [E, d]; INT4: bf16 [E, f/128, d]; otherwise NULL
  *   sh_*        the same for the n_shared shared experts ([S, ...]); NULL if S == 0
  * int8 weights are symmetric with one scale per output column; int4 weights are
- * symmetric signed 4-bit, two per byte along the contiguous dim (low nibble =
- * even column), with one scale per 128 rows of K and output column; fp8 weights
- * are E4M3 codes (no infinities, largest finite 448) with one scale per output
- * column.  In every case the weight the layer uses is bf16(q * s): the exact
- * product rounded once. */
+ * symmetric signed 4-bit, two per byte along the contiguous (reduction) dim, low
+ * nibble = even k, with one scale per 128 rows of K and output column; fp8
+ * weights are E4M3 codes (no infinities, largest finite 448) with one scale per
+ * output column.  In every case the weight the layer uses is bf16(q * s): the
+ * exact product rounded once, formed inside the expert GEMM's main loop. */
 typedef struct moe_weights {
   const void* rms_gamma;
   const void* w_router;
@@ -323,16 +325,17 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
 /* moe_layer_forward with per-step timing marks, for profiling.
  * Source: picx.dev summary of the moe-ceilings study, Summary and Sub-study 1
  * (the forward is profiled module by module to find where the time goes before
- * anything is fused).  events[0] is
- * recorded on `stream` before the first kernel and events[i] right after step i
- * (i = 1 .. moe_layer_step_count(cfg)).  The steps are RMSNorm, router, route,
- * permute, [dequantise + gather], gate/up GEMM, down GEMM, combine:
+ * anything is fused).  It always runs the layer as a chain of kernels, also
+ * for the decode batches that moe_layer_forward runs as a single launch.
+ * events[0] is recorded on `stream` before the first kernel and events[i] right
+ * after step i (i = 1 .. moe_layer_step_count(cfg)).  The steps are RMSNorm,
+ * router, route, permute, [gather], gate/up GEMM, down GEMM, combine (expert
+ * choice: route = the scores, permute = the experts' picks):
  *   - up to 32 tokens the route launch also builds the permutation, and the
  *     permute step is empty;
  *   - the bracketed step exists for tensor-core experts: it gathers the routed
- *     token rows (and, at prefill batch sizes, dequantises int8/int4 experts),
- *     except on bf16 decode tiles, where the gate/up GEMM gathers them itself
- *     and the step is empty.
+ *     token rows, except on bf16 decode tiles, where the gate/up GEMM gathers
+ *     them itself and the step is empty.
  * `events` holds caller-created cudaEvent_t handles (as void*); n_events must be
  * at least moe_layer_step_count(cfg) + 1.  No optional outputs. */
 moe_status moe_layer_forward_profiled(const moe_config* cfg, const moe_weights* w,

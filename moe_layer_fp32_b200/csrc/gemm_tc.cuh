@@ -50,10 +50,6 @@ struct ByteWeights { static constexpr bool value = WQ == WQ_INT8 || WQ == WQ_FP8
 
 constexpr int kTcBaseThreads = 320;   // producer, MMA, 8 epilogue warps
 constexpr int kEpiWarps = 8;
-// dequantisation warps for int8 / int4 weights (int4 is bound by shared-memory
-// bandwidth already at 8; int8's longer conversion gains from 16)
-template <int WQ>
-struct DeqWarps { static constexpr int value = ByteWeights<WQ>::value ? 16 : 8; };
 constexpr int kMaxGroups = 512;
 
 struct TcProblem {
@@ -130,18 +126,17 @@ struct TcConfig {
   static constexpr int TILE_N = TcShape<EPI, DIRECT>::TILE_N;
   static constexpr uint32_t A_BYTES = TcShape<EPI, DIRECT>::A_BYTES;
   static constexpr uint32_t B_BYTES = BN * 64 * 2;
-  // raw quantised weight block (128 features x 64 k): int8 128 B rows, int4 64 B rows
-  static constexpr uint32_t RAW_BYTES =
-      ByteWeights<WQ>::value ? 128 * 64 : WQ == WQ_INT4 ? 64 * 64 : 0;
-  static constexpr uint32_t RAW_ROW = ByteWeights<WQ>::value ? 128 : 64;
+  // raw quantised weight block of 128 features x 64 k, stored K-contiguous: one row
+  // of 64 codes per feature (int8 / fp8: 64 B, int4: 32 B)
+  static constexpr uint32_t RAW_ROW = ByteWeights<WQ>::value ? 64 : WQ == WQ_INT4 ? 32 : 0;
+  static constexpr uint32_t RAW_BYTES = 128 * RAW_ROW;
   static constexpr uint32_t SCALE_BYTES = WQ == WQ_BF16 ? 0 : 256;   // 128 bf16 scales
   // bf16 weights: one ring of TMA stages [weights NA x 16 KB | tokens].
-  // int8 / int4 weights: a deep ring of TMA stages [tokens | raw weights | scales
-  // in a 1 KB slot] (so that enough weight bytes are in flight to cover HBM
-  // latency) and AS slots of dequantised bf16 weights that the dequantisation
-  // warps fill and the MMA drains.  Every stage and slot is 1024-byte aligned.
-  static constexpr int AS = WQ == WQ_BF16 ? 0 : 2;
-  static constexpr uint32_t A_SLOT_BYTES = NA * A_BYTES;
+  // int8 / int4 / fp8 weights: a deep ring of TMA stages [tokens | raw weights |
+  // scales in a 1 KB slot] (so that enough weight bytes are in flight to cover
+  // HBM latency); the dequantisation warps expand each block into one of two TMEM
+  // slots of bf16 weights, from which the MMA takes its A operand.  Every stage
+  // is 1024-byte aligned.
   static constexpr uint32_t STAGE_BYTES =
       WQ == WQ_BF16 ? NA * A_BYTES + B_BYTES : B_BYTES + NA * RAW_BYTES + 1024;
   static constexpr uint32_t TOKEN_OFF = WQ == WQ_BF16 ? NA * A_BYTES : 0;
@@ -150,23 +145,31 @@ struct TcConfig {
   // bytes the TMA delivers per stage
   static constexpr uint32_t TX_BYTES =
       WQ == WQ_BF16 ? STAGE_BYTES : B_BYTES + NA * (RAW_BYTES + SCALE_BYTES);
-  static constexpr int DEQ_WARPS = DeqWarps<WQ>::value;
-  static constexpr int THREADS = kTcBaseThreads + (WQ == WQ_BF16 ? 0 : 32 * DEQ_WARPS);
-  static constexpr int STAGES_RAW = (200 * 1024 - AS * A_SLOT_BYTES) / STAGE_BYTES;
+  // one dequantisation thread per feature of each weight block: 4 warps per block,
+  // each warp on the TMEM lane quadrant its warp index allows
+  static constexpr int DEQ_WARPS = WQ == WQ_BF16 ? 0 : 4 * NA;
+  static constexpr int THREADS = kTcBaseThreads + 32 * DEQ_WARPS;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
   static constexpr int STAGE_CAP = WQ == WQ_BF16 ? 8 : 16;
   static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
-  static constexpr uint32_t A_REGION = AS * A_SLOT_BYTES;
+  static constexpr uint32_t A_REGION = 0;
   static constexpr uint32_t ACC_COLS = NA * BN;
-  static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS;
+  // TMEM: two accumulators, then (quantised weights) two slots of NA bf16 weight
+  // blocks, 128 lanes x 32 columns each (64 k, two per 32-bit column)
+  static constexpr uint32_t A_COL0 = 2 * ACC_COLS;
+  static constexpr uint32_t A_SLOT_COLS = WQ == WQ_BF16 ? 0 : NA * 32;
+  static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS + 2 * A_SLOT_COLS;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                         : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-  // swapped: A = weights (MN-major), B = tokens (K-major), M = 128 features, N = BN,
-  //          one MMA per weight block;
+  // swapped: A = weights, M = 128 features, N = BN tokens (K-major), one MMA per
+  //          weight block; bf16 weights come from shared memory (MN-major), the
+  //          dequantised ones from TMEM (K-major);
   // direct:  A = tokens (K-major), B = all NA weight blocks at once (MN-major, the
   //          blocks 16 KB apart = two 64-feature boxes each at the 8 KB leading
   //          offset), M = 128 tokens, N = 128 * NA
-  static constexpr uint32_t IDESC = DIRECT ? idesc_bf16(128, 128 * NA, false, true)
-                                           : idesc_bf16(128, BN, true, false);
+  static constexpr uint32_t IDESC = DIRECT            ? idesc_bf16(128, 128 * NA, false, true)
+                                    : WQ == WQ_BF16 ? idesc_bf16(128, BN, true, false)
+                                                    : idesc_bf16(128, BN, false, false);
   // barriers + bookkeeping after the tiles
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * 2) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
@@ -180,6 +183,7 @@ struct TcConfig {
   static_assert(SMEM_BYTES + 64 <= 227 * 1024, "shared memory per CTA (dynamic + static)");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
   static_assert(!DIRECT || BN == 128, "direct tiles hold 128 tokens");
+  static_assert(WQ == WQ_BF16 || !DIRECT, "quantised weights take the swapped tiles");
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 128-byte swizzle alignment");
   static_assert(NA * SCALE_BYTES <= 1024, "scale slot");
   static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
@@ -281,59 +285,75 @@ MOE_DEV void int4x8_to_bf16(uint32_t v, const uint32_t (&s2)[4], uint32_t (&o)[4
   }
 }
 
-// Dequantise one raw weight block (128 features x 64 k of tile (g, n, kb)) into the
-// bf16 MN-major layout with the 128-byte swizzle that a TMA load would have
-// produced: 16-byte chunk cc (8 features) of k-row k of 64-feature half h sits at
-// h * 8192 + k * 128 + ((cc ^ (k & 7)) << 4).  Value = bf16(q * s), the exact
-// product rounded once; the block's 128 scales were loaded by the TMA with it.
-// Features at or beyond N were zero-filled by the TMA (q = 0, s = 0).
-template <int WQ, int NTHREADS>
-MOE_DEV void dequant_block(const uint8_t* raw, uint8_t* out, const __nv_bfloat16* ssm, int t) {
-  constexpr int RAW_ROW = WQ == WQ_INT4 ? 64 : 128;
-  constexpr int ITERS = 64 * 16 / NTHREADS;
-  static_assert(64 * 16 % NTHREADS == 0, "whole chunks per thread");
-  // the column chunk of thread t is the same in every iteration (16 | NTHREADS):
-  // load its scales once, then all raw words, then convert
-  const int c = t & 15;
-  const uint4 sv = *reinterpret_cast<const uint4*>(ssm + c * 8);
-  uint32_t w4[ITERS];
-  uint2 w8[ITERS];
+// One feature's 64 codes of a k-block (stored K-contiguous in shared memory: int4
+// 32 bytes, int8 / fp8 64 bytes) to 32 bf16x2 words, k = 2c in the low half of
+// word c, each value bf16(q * s): the exact product rounded once.  The 16-byte
+// pieces are read in a lane-rotated order so that the 8 lanes of each quarter-warp
+// cover all 32 banks.
+template <int WQ>
+MOE_DEV void dequant_row(const uint8_t* row, __nv_bfloat16 s, int lane, uint32_t (&o)[32]) {
+  if (WQ == WQ_INT4) {
+    // load j reads piece (j + r) & 1; swap back when r = 1
+    const int r = (lane >> 2) & 1;
+    uint4 v[2];
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int k = (t + it * NTHREADS) >> 4;
-    if (WQ == WQ_INT4) w4[it] = *reinterpret_cast<const uint32_t*>(raw + k * RAW_ROW + c * 4);
-    else w8[it] = *reinterpret_cast<const uint2*>(raw + k * RAW_ROW + c * 8);
-  }
+    for (int j = 0; j < 2; ++j) v[j] = *reinterpret_cast<const uint4*>(row + 16 * ((j + r) & 1));
+    if (r) {
+      const uint4 t = v[0];
+      v[0] = v[1];
+      v[1] = t;
+    }
+    const uint32_t s2 = (uint32_t)__bfloat16_as_ushort(s) * 0x10001u;
+    const uint32_t sp[4] = {s2, s2, s2, s2};
+    const uint32_t wd[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int k = (t + it * NTHREADS) >> 4;
-    uint32_t pk[4];
-    if (WQ == WQ_INT4) {
-      const uint32_t s2[4] = {sv.x, sv.y, sv.z, sv.w};
-      int4x8_to_bf16(w4[it], s2, pk);
-    } else {
-      const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv);
-      const uint2 v = w8[it];
+    for (int i = 0; i < 8; ++i) {
+      uint32_t q4[4];
+      int4x8_to_bf16(wd[i], sp, q4);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t w = i < 2 ? v.x : v.y;
-        const int sh = (i & 1) * 16;
+      for (int j = 0; j < 4; ++j) o[4 * i + j] = q4[j];
+    }
+  } else {
+    // load j reads piece (j + r) & 3; rotate back by r (two conditional rotations)
+    const int r = (lane >> 1) & 3;
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(row + 16 * ((j + r) & 3));
+    if (r & 1) {
+      const uint4 t = v[3];
+      v[3] = v[2];
+      v[2] = v[1];
+      v[1] = v[0];
+      v[0] = t;
+    }
+    if (r & 2) {
+      uint4 t = v[0];
+      v[0] = v[2];
+      v[2] = t;
+      t = v[1];
+      v[1] = v[3];
+      v[3] = t;
+    }
+    const float sf = __bfloat162float(s);
+    const uint32_t wd[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                             v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
         float q0, q1;
         if (WQ == WQ_FP8) {
-          const float2 q = e4m3x2_to_float2(w >> sh);
+          const float2 q = e4m3x2_to_float2(wd[i] >> (16 * h));
           q0 = q.x;
           q1 = q.y;
         } else {
-          q0 = (float)(int8_t)((w >> sh) & 0xff);
-          q1 = (float)(int8_t)((w >> (sh + 8)) & 0xff);
+          q0 = (float)(int8_t)((wd[i] >> (16 * h)) & 0xff);
+          q1 = (float)(int8_t)((wd[i] >> (16 * h + 8)) & 0xff);
         }
-        __nv_bfloat162 h2 =
-            __floats2bfloat162_rn(q0 * __low2float(s2[i]), q1 * __high2float(s2[i]));
-        pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+        __nv_bfloat162 r = __floats2bfloat162_rn(q0 * sf, q1 * sf);
+        o[2 * i + h] = *reinterpret_cast<uint32_t*>(&r);
       }
     }
-    *reinterpret_cast<uint4*>(out + (c >> 3) * 8192 + k * 128 + (((c & 7) ^ (k & 7)) << 4)) =
-        make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
 }
 
@@ -444,8 +464,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   constexpr int NA = C::NA;
   constexpr int STAGES = C::STAGES;
   uint8_t* tiles = smem;
-  uint8_t* aslots = tiles + STAGES * C::STAGE_BYTES;   // dequantised weights (int8 / int4)
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(aslots + C::A_REGION);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;       // [2]
@@ -543,17 +562,18 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
           tma_load_3d(st + C::A_BYTES + 8192, m2, &full_bar[stage], n2 + 64, kb * 64, ti.g);
         }
       } else {
-        // raw bytes: x is the byte column (two int4 values per byte)
+        // raw codes stored K-contiguous [G][N][K bytes]: x is the byte offset of the
+        // k-block within a feature's row, y the first feature
         uint8_t* raw = st + C::RAW_OFF;
         uint8_t* scl = st + C::SCALE_OFF;
-        const int div = WQ == WQ_INT4 ? 2 : 1;
+        const int kx = kb * (int)C::RAW_ROW;
         const void* s2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmS2 : (const void*)&P.tmS;
-        tma_load_3d(raw, &P.tmA, &full_bar[stage], ti.n0 / div, kb * 64, ti.g);
+        tma_load_3d(raw, &P.tmA, &full_bar[stage], kx, ti.n0, ti.g);
         // int8: scales [G][N] (second coordinate g, third 0); int4: [G][K/128][N]
         if (WQ != WQ_INT4) tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, ti.g, 0);
         else tma_load_3d(scl, &P.tmS, &full_bar[stage], ti.n0, kb / 2, ti.g);
         if (NA == 2) {
-          tma_load_3d(raw + C::RAW_BYTES, m2, &full_bar[stage], n2 / div, kb * 64, ti.g);
+          tma_load_3d(raw + C::RAW_BYTES, m2, &full_bar[stage], kx, n2, ti.g);
           if (WQ != WQ_INT4) tma_load_3d(scl + 256, s2, &full_bar[stage], n2, ti.g, 0);
           else tma_load_3d(scl + 256, s2, &full_bar[stage], n2, kb / 2, ti.g);
         }
@@ -629,23 +649,27 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
               !mbar_wait(&deq_bar[aslot], aphase, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
           tc_fence_after();
           const uint32_t st_addr = smem_u32(tiles + stage * C::STAGE_BYTES);
-          const uint32_t a_addr =
-              WQ == WQ_BF16 ? st_addr : smem_u32(aslots + aslot * C::A_SLOT_BYTES);
           const uint32_t b_addr = st_addr + C::TOKEN_OFF;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             // weights: MN-major SW128, 16 k-rows of 128 B per MMA step; the two
             //    64-feature halves sit 8 KB apart (leading offset), 8-row groups 1 KB
             //    apart.  tokens: K-major SW128, 16 k = 32 B per step, 8-row groups 1 KB.
+            //    Dequantised weights: TMEM, 8 columns (16 k) per step.
             const uint64_t xd = sw128_desc(b_addr + kk * 32, 16, 1024);
-            const uint64_t wd = sw128_desc(a_addr + kk * 2048, 8192, 1024);
             const uint32_t accum = (kb != ti.kb0 || kk != 0);
-            if (DIRECT) {
+            if (WQ != WQ_BF16) {
+              const uint32_t a_tm = tmem_base + C::A_COL0 + aslot * C::A_SLOT_COLS + kk * 8;
+              tc_mma_f16_tmem_a(d_tmem, a_tm, xd, C::IDESC, accum);
+              if (NA == 2) tc_mma_f16_tmem_a(d_tmem + BN, a_tm + 32, xd, C::IDESC, accum);
+            } else if (DIRECT) {
+              const uint64_t wd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
               tc_mma_f16(d_tmem, xd, wd, C::IDESC, accum);   // N = 128 * NA at once
             } else {
+              const uint64_t wd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
               tc_mma_f16(d_tmem, wd, xd, C::IDESC, accum);
               if (NA == 2) {
-                const uint64_t wd2 = sw128_desc(a_addr + C::A_BYTES + kk * 2048, 8192, 1024);
+                const uint64_t wd2 = sw128_desc(st_addr + C::A_BYTES + kk * 2048, 8192, 1024);
                 tc_mma_f16(d_tmem + BN, wd2, xd, C::IDESC, accum);
               }
             }
@@ -671,7 +695,11 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   } else if (warp >= 2 + kEpiWarps) {
     // ------------------------------------------------------------ dequantisation
     if (WQ != WQ_BF16) {
-      const int dt = threadIdx.x - 32 * (2 + kEpiWarps);
+      // warp w expands weight block (w - 10) / 4 for the 32 features of its TMEM lane
+      // quadrant w % 4: one thread per feature, its 64 codes of the k-block
+      const int blk = (warp - 2 - kEpiWarps) >> 2;
+      const int qd = warp & 3;
+      const int feat = qd * 32 + lane;
       int stage = 0;
       uint32_t phase = 0;
       int aslot = 0;
@@ -683,16 +711,18 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
           if (!mbar_wait(&aempty_bar[aslot], aphase ^ 1, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
-          uint8_t* st = tiles + stage * C::STAGE_BYTES;
-          uint8_t* dst = aslots + aslot * C::A_SLOT_BYTES;
-          const uint8_t* raw = st + C::RAW_OFF;
-          const __nv_bfloat16* scl = reinterpret_cast<const __nv_bfloat16*>(st + C::SCALE_OFF);
-#pragma unroll
-          for (int i = 0; i < NA; ++i)
-            dequant_block<WQ, 32 * C::DEQ_WARPS>(raw + i * C::RAW_BYTES, dst + i * C::A_BYTES,
-                                                 scl + 128 * i, dt);
-          // generic-proxy stores must be visible to the tensor core (async proxy)
-          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint8_t* st = tiles + stage * C::STAGE_BYTES;
+          const uint8_t* row = st + C::RAW_OFF + blk * C::RAW_BYTES + feat * C::RAW_ROW;
+          const __nv_bfloat16 sc =
+              reinterpret_cast<const __nv_bfloat16*>(st + C::SCALE_OFF)[128 * blk + feat];
+          uint32_t w[32];
+          dequant_row<WQ>(row, sc, lane, w);
+          tmem_st32(tmem_base + ((uint32_t)(qd * 32) << 16) + C::A_COL0 +
+                        aslot * C::A_SLOT_COLS + blk * 32,
+                    w);
+          tmem_wait_st();
+          tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&deq_bar[aslot]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }

@@ -1,8 +1,7 @@
 // CUDA-core kernels of the layer: RMSNorm (a1), the split-K router for small
 // batches (a2), softmax/top-k routing (a3), histogram + scan + permutation
-// (a4/a5), the one-pass dequantisation of int8/int4 experts, the row gather for
-// prefill tiles, the combine (a8), and the FP32 grouped SwiGLU FFN used when the
-// expert weights are fp32.
+// (a4/a5), the row gather for prefill tiles, the combine (a8), and the FP32
+// grouped SwiGLU FFN used when the expert weights are fp32.
 #pragma once
 #include <type_traits>
 #include "common.cuh"
@@ -746,93 +745,6 @@ __global__ void __launch_bounds__(256) k_perm_rank(const int32_t* __restrict__ i
       } else {
         slot_of[a] = -1;
       }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Dequantise whole expert matrices to bf16 (prefill batches with int8 / int4 /
-// fp8 experts): w = bf16(q * s), the exact product rounded once, 8 outputs per
-// thread per step.  Experts that received no token are skipped when `offsets`
-// is given.  blockIdx.y = matrix, blockIdx.z = expert.
-// ---------------------------------------------------------------------------
-struct DeqMatrix {
-  const uint8_t* q;              // int8 / fp8 [G][K][N] or packed int4 [G][K][N/2]
-  const __nv_bfloat16* s;        // [G][N] (int8, fp8) or [G][K/128][N] (int4)
-  __nv_bfloat16* out;            // [G][K][N]
-  const int32_t* offsets;        // [G+1] routed segments, or nullptr (dequantise all)
-  int G, K, N;
-};
-struct DeqArgs {
-  DeqMatrix m[6];
-  int n;
-};
-
-// KIND: 0 = int8, 1 = int4, 2 = fp8 (E4M3 codes, the int8 layout)
-template <int KIND>
-__global__ void __launch_bounds__(256) k_dequant_experts(const __grid_constant__ DeqArgs a) {
-  constexpr bool INT4 = KIND == 1;
-  pdl_wait();
-  pdl_trigger();
-  // block (x, y, z) = 8 rows of matrix y of expert z; thread (tx, ty) = row ty,
-  // 8-column chunks tx, tx + 32, ...
-  const DeqMatrix& M = a.m[blockIdx.y];
-  const int g = blockIdx.z;
-  if (g >= M.G) return;
-  if (M.offsets && M.offsets[g + 1] == M.offsets[g]) return;
-  const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (k >= M.K) return;
-  const int nch = M.N / 8;
-  const __nv_bfloat16* srow =
-      INT4 ? M.s + ((size_t)g * (M.K / 128) + k / 128) * M.N : M.s + (size_t)g * M.N;
-  const uint8_t* qrow = M.q + ((size_t)g * M.K + k) * (INT4 ? M.N / 2 : M.N);
-  __nv_bfloat16* orow = M.out + ((size_t)g * M.K + k) * M.N;
-  constexpr int U = 4;
-  for (int c0 = threadIdx.x & 31; c0 < nch; c0 += 32 * U) {
-    uint4 sv[U];
-    uint32_t v4[U];
-    uint2 v8[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + 32 * u;
-      if (c < nch) {
-        sv[u] = *reinterpret_cast<const uint4*>(srow + c * 8);
-        if (INT4) v4[u] = *reinterpret_cast<const uint32_t*>(qrow + c * 4);
-        else v8[u] = *reinterpret_cast<const uint2*>(qrow + c * 8);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + 32 * u;
-      if (c >= nch) break;
-      const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv[u]);
-      float q[8];
-      if (INT4) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = (float)((int)(v4[u] << (28 - 4 * i)) >> 28);
-      } else if (KIND == 2) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t w = i < 2 ? v8[u].x : v8[u].y;
-          const float2 f = e4m3x2_to_float2(w >> ((i & 1) * 16));
-          q[2 * i] = f.x;
-          q[2 * i + 1] = f.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          q[i] = (float)(int8_t)((v8[u].x >> (8 * i)) & 0xff);
-          q[4 + i] = (float)(int8_t)((v8[u].y >> (8 * i)) & 0xff);
-        }
-      }
-      uint32_t pk[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(q[2 * i] * __low2float(s2[i]),
-                                                  q[2 * i + 1] * __high2float(s2[i]));
-        pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-      }
-      *reinterpret_cast<uint4*>(orow + c * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
 }

@@ -77,13 +77,21 @@ inline size_t n_slots(const moe_config* c) {
   return expert_choice(c) ? (size_t)c->E * ec_capacity(c) : (size_t)c->T * c->k;
 }
 
-// token-tile width of the expert GEMMs from the mean rows per expert
+inline bool quantised(const moe_config* c) {
+  return c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4 ||
+         c->expert_dtype == MOE_FP8;
+}
+
+// token-tile width of the expert GEMMs from the mean rows per expert.  Quantised
+// experts keep the weights on the MMA's M side at every batch; their widest tile
+// holds 96 tokens (two accumulators of 2 x 96 columns and two slots of dequantised
+// weights fill the 512 TMEM columns).
 int pick_bn(const moe_config* c) {
   const double mean = (double)n_slots(c) / c->E;
   if (mean <= 16) return 16;
   if (mean <= 32) return 32;
   if (mean <= 64) return 64;
-  return 128;
+  return quantised(c) ? 96 : 128;
 }
 // Quantised experts at prefill tile widths are dequantised once to bf16 in the
 // workspace (the in-loop dequantisation would repeat for every token tile of an
@@ -109,15 +117,11 @@ inline int split_counters() { return num_sms() * 8; }
 // in bf16 (half the bytes the down GEMM writes and the combine reads); the
 // grouped-FFN and combine entry points exchange them in FP32.
 inline bool y_bf16(const moe_config* c) { return tc_experts(c); }
-inline bool quantised(const moe_config* c) {
-  return c->expert_dtype == MOE_INT8 || c->expert_dtype == MOE_INT4 ||
-         c->expert_dtype == MOE_FP8;
-}
-inline bool dequant_once(const moe_config* c) { return quantised(c) && pick_bn(c) == 128; }
+
 
 struct Layout {
   size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, split,
-      splitcnt, h, y, ys, deq, sct,
+      splitcnt, h, y, ys, sct,
       total;
   int ns;
 };
@@ -194,7 +198,6 @@ Layout layout(const moe_config* c) {
   L.h = o;        o = align_up(o + (R + S * T) * f * hb);
   L.y = o;        o = align_up(o + R * d * (y_bf16(c) ? 2 : 4));
   L.ys = o;       o = align_up(o + S * T * d * 4);
-  L.deq = o;      o = align_up(o + (dequant_once(c) ? (E + S) * 3 * d * f * 2 : 0));
   L.sct = o;      o = align_up(o + (expert_choice(c) ? T * E * 4 : 0));
   L.total = o;
   return L;
@@ -287,14 +290,15 @@ bool map_weights(CUtensorMap* m, const void* base, int G, int K, int N) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// raw quantised weights [G][K][NB] bytes (NB = N for int8, N/2 for int4), no
-// swizzle; box = one 128-feature block x 64 k
-bool map_raw(CUtensorMap* m, const void* base, int G, int K, int NB, int box_bytes) {
+// raw quantised codes stored K-contiguous, [G][N][KB] bytes (KB = K for int8 /
+// fp8, K/2 for int4), no swizzle; box = the codes of one 64-deep k-block
+// (row_bytes) for 128 features
+bool map_raw(CUtensorMap* m, const void* base, int G, int N, int KB, int row_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || !base) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)NB, (cuuint64_t)K, (cuuint64_t)G};
-  cuuint64_t strides[2] = {(cuuint64_t)NB, (cuuint64_t)K * NB};
-  cuuint32_t box[3] = {(cuuint32_t)box_bytes, 64, 1};
+  cuuint64_t dims[3] = {(cuuint64_t)KB, (cuuint64_t)N, (cuuint64_t)G};
+  cuuint64_t strides[2] = {(cuuint64_t)KB, (cuuint64_t)N * KB};
+  cuuint32_t box[3] = {(cuuint32_t)row_bytes, 128, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -318,10 +322,11 @@ bool map_scales(CUtensorMap* m, const moe_config* c, const void* base, int G, in
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// expert weight matrix [G][K][N] in the storage the GEMM reads (wq)
+// expert weight matrix of K x N in the storage the GEMM reads (wq): bf16 [G][K][N],
+// quantised codes [G][N][K] (int4 [G][N][K/2])
 bool map_expert(CUtensorMap* m, int wq, const void* base, int G, int K, int N) {
-  if (wq == WQ_INT8 || wq == WQ_FP8) return map_raw(m, base, G, K, N, 128);
-  if (wq == WQ_INT4) return map_raw(m, base, G, K, N / 2, 64);
+  if (wq == WQ_INT8 || wq == WQ_FP8) return map_raw(m, base, G, N, K, 64);
+  if (wq == WQ_INT4) return map_raw(m, base, G, N, K / 2, 32);
   return map_weights(m, base, G, K, N);
 }
 
@@ -405,12 +410,12 @@ moe_status launch_tc_bn_q(int bn, const TcParams& p, cudaStream_t st) {
     case 16: return launch_tc<EPI, 16, false, WQ>(p, st);
     case 32: return launch_tc<EPI, 32, false, WQ>(p, st);
     case 64: return launch_tc<EPI, 64, false, WQ>(p, st);
-    default:   // prefill tiles: tokens on MMA-M (quantised weights are dequantised first)
-      if constexpr (WQ == WQ_BF16) {
+    default:   // prefill tiles
+      if constexpr (WQ == WQ_BF16) {   // tokens on MMA-M
         if (kPairTiles) return launch_pair<EPI>(p, st);
         return launch_tc<EPI, 128, true, WQ>(p, st);
-      } else {
-        return MOE_ERR_UNSUPPORTED;
+      } else {                         // quantised: weights on M, 96 tokens on N
+        return launch_tc<EPI, 96, false, WQ>(p, st);
       }
   }
 }
@@ -788,8 +793,8 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     mk->mark(st);
     return s;
   }
-  // tensor-core experts: [dequantise once], [gather the routed rows into xp], then
-  // gate/up and down on the tensor cores.  The TMA (and the vector loads of the
+  // tensor-core experts: [gather the routed rows into xp], then gate/up and down on
+  // the tensor cores (quantised weights are expanded inside their main loop).  The TMA (and the vector loads of the
   // gather and dequantisation kernels) need 16-byte aligned operands.
   {
     auto a16 = [](const void* q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
@@ -802,40 +807,9 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
   const int bn = pick_bn(c);
   const int R = (int)n_slots(c);
-  int wq = wq_of(c);
-  moe_weights wl = *w;                     // the weights the GEMMs read
+  const int wq = wq_of(c);
+  const moe_weights& wl = *w;
   moe_status s = MOE_OK;
-  if (dequant_once(c)) {
-    const size_t per = (size_t)c->d * c->f;
-    __nv_bfloat16* base = at<__nv_bfloat16>(ws, L.deq);
-    __nv_bfloat16* dst[6];
-    for (int i = 0; i < 3; ++i) dst[i] = base + (size_t)i * c->E * per;
-    for (int i = 0; i < 3; ++i) dst[3 + i] = base + (size_t)3 * c->E * per + (size_t)i * S * per;
-    DeqArgs a{};
-    const void* srcq[6] = {w->w_gate, w->w_up, w->w_down, w->sh_gate, w->sh_up, w->sh_down};
-    const void* srcs[6] = {w->s_gate, w->s_up, w->s_down, w->sh_s_gate, w->sh_s_up, w->sh_s_down};
-    a.n = S > 0 ? 6 : 3;
-    for (int i = 0; i < a.n; ++i) {
-      DeqMatrix& m = a.m[i];
-      m.q = static_cast<const uint8_t*>(srcq[i]);
-      m.s = static_cast<const __nv_bfloat16*>(srcs[i]);
-      m.out = dst[i];
-      m.offsets = i < 3 ? offsets : nullptr;
-      m.G = i < 3 ? c->E : S;
-      m.K = (i % 3 == 2) ? c->f : c->d;
-      m.N = (i % 3 == 2) ? c->d : c->f;
-    }
-    // 8 rows of one matrix per block (K is d or f, both multiples of 128)
-    const int kmax = c->d > c->f ? c->d : c->f;
-    dim3 grid(kmax / 8, a.n, c->E > S ? c->E : S);
-    if (wq == WQ_INT4) MOE_LAUNCH((k_dequant_experts<1>), grid, 256, 0, st, a);
-    else if (wq == WQ_FP8) MOE_LAUNCH((k_dequant_experts<2>), grid, 256, 0, st, a);
-    else MOE_LAUNCH((k_dequant_experts<0>), grid, 256, 0, st, a);
-    if ((s = check_launch()) != MOE_OK) return s;
-    wl.w_gate = dst[0]; wl.w_up = dst[1]; wl.w_down = dst[2];
-    wl.sh_gate = dst[3]; wl.sh_up = dst[4]; wl.sh_down = dst[5];
-    wq = WQ_BF16;
-  }
   const bool g4 = gather_in_gemm(c);
   float* split_part = split_k(c) ? at<float>(ws, L.split) : nullptr;
   int32_t* split_cnt = split_k(c) ? at<int32_t>(ws, L.splitcnt) : nullptr;
@@ -850,7 +824,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
                xp);
     if ((s = check_launch()) != MOE_OK) return s;
   }
-  mk->mark(st);   // end of the (optional) dequantisation and gather step
+  mk->mark(st);   // end of the (optional) gather step
   {
     TcParams p;
     if ((s = gateup_params(c, w, wl, wq, xn, xp, offsets, rr, h, split_part, split_cnt, err, p)) !=
@@ -1363,13 +1337,12 @@ int32_t moe_layer_launch_count(const moe_config* cfg) {
   if (single_launch(cfg)) return 1;   // with 16-byte aligned tensors
   // rmsnorm, router, route, gate/up, down and combine, plus the permutation (its
   // own launch, three for large batches, or none when it shares the routing
-  // launch), and for tensor-core experts at wide tiles the row gather and (int8 /
-  // int4) the one-pass dequantisation
+  // launch), and for tensor-core experts at wide tiles the row gather
   const int gather = tc_experts(cfg) && !gather_in_gemm(cfg) ? 1 : 0;
   if (expert_choice(cfg))   // rmsnorm, router, scores, picks, gate/up, down, combine
-    return 7 + gather + (dequant_once(cfg) ? 1 : 0);
+    return 7 + gather;
   const int perm = fused_route_permute(cfg) ? 0 : cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
-  return 6 + perm + gather + (dequant_once(cfg) ? 1 : 0);
+  return 6 + perm + gather;
 }
 
 }  // extern "C"

@@ -22,16 +22,21 @@ Recipe (every tensor draws from its own PCG64 stream,
     ``bias_e = ln p_e - mean(ln p)``.
 * int8 weights: symmetric, one bf16 scale per output column,
   ``s = bf16(max|w| / 127)``, ``q = clamp(rint(w / s), -127, 127)``.
+* Quantised codes (int8, int4, fp8) are stored with the reduction dim K
+  contiguous, i.e. as the transpose of the [K, N] weight: ``[E, N, K]`` (int4:
+  ``[E, N, K/2]``), so that one output feature's codes of a K block are adjacent.
 * fp8 weights: FP8 E4M3 codes, one bf16 scale per output column,
   ``s = bf16(max|w| / 448)``, ``q = e4m3(w / s)`` (round to nearest even).
 * int4 weights: symmetric, groups of ``group_size`` along the reduction (K) dim,
   ``s = bf16(max|w| / 7)``, ``q = clamp(rint(w / s), -8, 7)``; two values per byte
-  along the contiguous (output) dim, low nibble first.
+  along the contiguous (K) dim, low nibble first.
 
 Weight layouts follow the layer's statement of the problem: ``W_r[d, E]``,
 ``W_gate/W_up[E, d, f]``, ``W_down[E, f, d]``; shared experts ``[S, d, f]`` and
-``[S, f, d]``.  int8 scales are ``[E, f]`` (gate/up) and ``[E, d]`` (down); int4
-scales are ``[E, d/G, f]`` (gate/up) and ``[E, f/G, d]`` (down).
+``[S, f, d]``; quantised codes transposed (``[E, f, d]`` and ``[E, d, f]``, int4
+with the last dim halved).  int8 / fp8 scales are ``[E, f]`` (gate/up) and
+``[E, d]`` (down); int4 scales are ``[E, d/G, f]`` (gate/up) and ``[E, f/G, d]``
+(down).
 """
 from __future__ import annotations
 
@@ -164,30 +169,32 @@ def master_expert(shape: LayerShape, which: str, e: int, shared: bool = False) -
 
 
 def quantize_int8(w: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
-    """w[K, N] fp32 -> (q int8 [K, N], s bf16 [N]); one scale per output column."""
+    """w[K, N] fp32 -> (q int8 stored [N, K], s bf16 [N]); one scale per output
+    column.  The codes are stored with K contiguous (the transpose of w)."""
     amax = w.abs().amax(dim=0)
     s = (amax / 127.0).to(torch.bfloat16)
     s = torch.where(s.float() > 0, s, torch.ones_like(s))
     q = torch.round(w / s.float()).clamp_(-127, 127).to(torch.int8)
-    return q, s
+    return q.t().contiguous(), s
 
 
 def quantize_fp8(w: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
-    """w[K, N] fp32 -> (q uint8 FP8 E4M3 codes [K, N], s bf16 [N]); one scale per
-    output column, ``s = bf16(max|w| / 448)``, ``q = e4m3(w / s)`` rounded to nearest
-    even and clamped to the largest finite code (448)."""
+    """w[K, N] fp32 -> (q uint8 FP8 E4M3 codes stored [N, K], s bf16 [N]); one scale
+    per output column, ``s = bf16(max|w| / 448)``, ``q = e4m3(w / s)`` rounded to
+    nearest even and clamped to the largest finite code (448); K contiguous."""
     amax = w.abs().amax(dim=0)
     s = (amax / 448.0).to(torch.bfloat16)
     s = torch.where(s.float() > 0, s, torch.ones_like(s))
     q = (w / s.float()).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn)
-    return q.view(torch.uint8), s
+    return q.view(torch.uint8).t().contiguous(), s
 
 
 def quantize_int4(w: torch.Tensor, group: int) -> Tuple[torch.Tensor, torch.Tensor]:
-    """w[K, N] fp32 -> (packed uint8 [K, N/2], s bf16 [K/group, N]).
+    """w[K, N] fp32 -> (packed uint8 [N, K/2], s bf16 [K/group, N]).
 
-    Groups of ``group`` rows along K share a scale per column; byte j of a row
-    holds column 2j in its low nibble and column 2j+1 in its high nibble.
+    Groups of ``group`` rows along K share a scale per column.  The codes are
+    stored with K contiguous (the transpose of w): byte j of row n holds k = 2j in
+    its low nibble and k = 2j+1 in its high nibble.
     """
     K, N = w.shape
     wg = w.view(K // group, group, N)
@@ -195,9 +202,10 @@ def quantize_int4(w: torch.Tensor, group: int) -> Tuple[torch.Tensor, torch.Tens
     s = (amax / 7.0).to(torch.bfloat16)
     s = torch.where(s.float() > 0, s, torch.ones_like(s))
     q = torch.round(wg / s.float().unsqueeze(1)).clamp_(-8, 7).to(torch.int16).view(K, N)
-    lo = (q[:, 0::2] & 0xF)
-    hi = (q[:, 1::2] & 0xF) << 4
-    return (lo | hi).to(torch.uint8), s
+    qt = q.t()
+    lo = (qt[:, 0::2] & 0xF)
+    hi = (qt[:, 1::2] & 0xF) << 4
+    return (lo | hi).to(torch.uint8).contiguous(), s
 
 
 def _encode(shape: LayerShape, w: np.ndarray):

@@ -309,7 +309,7 @@ def permute(idx, E: int, capacity_factor: float = 0.0) -> Dict[str, np.ndarray]:
 # expert weights as the layer sees them
 # ---------------------------------------------------------------------------
 def unpack_int4(packed) -> np.ndarray:
-    """uint8 [K, N/2] -> int [K, N]; low nibble = even column, two's complement."""
+    """uint8 [R, C/2] -> int [R, C]; low nibble = even column, two's complement."""
     p = np.asarray(packed, dtype=np.uint8).astype(np.int64)
     lo = p & 0xF
     hi = (p >> 4) & 0xF
@@ -320,13 +320,14 @@ def unpack_int4(packed) -> np.ndarray:
 
 
 def dequant_int8(q, s) -> np.ndarray:
-    """w[K, N] = bf16(q[K, N] * s[N])."""
-    return round_bf16(np.asarray(q, np.float64) * np.asarray(s, np.float64)[None, :])
+    """w[K, N] = bf16(q[n, k] * s[n]) from codes stored K-contiguous, q[N, K]."""
+    return round_bf16(np.asarray(q, np.float64).T * np.asarray(s, np.float64)[None, :])
 
 
 def dequant_int4(packed, s, group: int) -> np.ndarray:
-    """w[K, N] = bf16(q[K, N] * s[K // group, N])."""
-    q = unpack_int4(packed).astype(np.float64)
+    """w[K, N] = bf16(q[n, k] * s[k // group, n]) from packed codes stored
+    K-contiguous, packed[N, K/2]."""
+    q = unpack_int4(packed).astype(np.float64).T
     sk = np.repeat(np.asarray(s, np.float64), group, axis=0)
     return round_bf16(q * sk)
 
@@ -346,8 +347,8 @@ def decode_e4m3(codes) -> np.ndarray:
 
 
 def dequant_fp8(q, s) -> np.ndarray:
-    """w[K, N] = bf16(e4m3(q[K, N]) * s[N])."""
-    return round_bf16(decode_e4m3(q) * np.asarray(s, np.float64)[None, :])
+    """w[K, N] = bf16(e4m3(q[n, k]) * s[n]) from codes stored K-contiguous, q[N, K]."""
+    return round_bf16(decode_e4m3(q).T * np.asarray(s, np.float64)[None, :])
 
 
 def expert_matrix(w, s, expert_dtype: str, group: int = 128) -> np.ndarray:

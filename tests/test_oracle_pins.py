@@ -288,8 +288,9 @@ def test_fp8_weights_within_quantisation_bound():
     bound = np.abs(w.numpy()) * 2.0 ** -4 + sf * 2.0 ** -10 + np.abs(dq) * 2.0 ** -8
     assert np.all(np.abs(dq - w.numpy()) <= bound * (1 + 1e-6))
     np.testing.assert_array_equal(dq, O.round_bf16(dq))
-    # the column maximum maps to (nearly) the largest code
-    assert np.all(np.abs(O.decode_e4m3(q.numpy())).max(axis=0) >= 416)
+    # each output column's maximum maps to (nearly) the largest code; the codes are
+    # stored K-contiguous, one row per output column
+    assert np.all(np.abs(O.decode_e4m3(q.numpy())).max(axis=1) >= 416)
 
 
 # ---------------------------------------------------------------------------
