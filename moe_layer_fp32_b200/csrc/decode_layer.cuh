@@ -71,16 +71,18 @@ MOE_DEV bool grid_barrier(unsigned* bar, int nblocks, long long limit, int32_t* 
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    volatile unsigned* gen = bar + 1;
-    const unsigned g = *gen;
+    const unsigned g = ld_acquire_gpu(bar + 1);
+    // the arrival releases this CTA's writes (ordered after the CTA barrier by the
+    // fence); the last one acquires everyone's, resets the count and publishes the
+    // new generation, which every waiter acquires
     __threadfence();
-    if (atomicAdd(bar, 1u) == (unsigned)nblocks - 1) {
+    if (atom_add_acq_rel_gpu(bar, 1u) == (unsigned)nblocks - 1) {
       atomicExch(bar, 0u);
-      __threadfence();
-      atomicAdd(bar + 1, 1u);
+      atom_add_acq_rel_gpu(bar + 1, 1u);
     } else {
       const long long t0 = clock64();
-      while (*gen == g) {
+      while (ld_acquire_gpu(bar + 1) == g) {
+        __nanosleep(32);
         if (clock64() - t0 > limit) {
           set_error(err, DEV_TIMEOUT);
           ok = 0;
@@ -88,7 +90,6 @@ MOE_DEV bool grid_barrier(unsigned* bar, int nblocks, long long limit, int32_t* 
         }
       }
     }
-    __threadfence();
     if (*reinterpret_cast<volatile int32_t*>(err) == DEV_TIMEOUT) ok = 0;
     *s_ok = ok;
   }

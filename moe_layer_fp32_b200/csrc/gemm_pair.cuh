@@ -16,17 +16,20 @@
 // reads 48 KB for the same work.  Shared-memory bandwidth is what bounds the
 // single-CTA kernel, so this cuts the staged bytes per flop by a third.
 //
-// Synchronisation (no TMA multicast: every CTA loads only into its own memory and
-// signals only its own barrier, so each CTA always knows when its copies landed):
-//   full[s]   (each CTA) its producer's TMA bytes of stage s;
-//   pfull[s]  (even CTA) one arrival forwarded by the odd CTA once ITS stage s
-//             landed;  the even CTA's MMA thread waits on both;
+// Synchronisation (no TMA multicast: each CTA loads only into its own memory):
+//   full[s]   (even CTA) stage s of BOTH CTAs: the even producer arms it with both
+//             CTAs' bytes, and each CTA's TMA loads complete on it (the pair form
+//             of the copy, whose barrier may sit in the peer);
 //   empty[s]  (each CTA) stage s consumed: the MMA thread commits to both CTAs;
 //   tfull[a]  (each CTA) accumulator a complete: commits to both CTAs;
 //   tempty[a] (even CTA) accumulator a drained: 8 epilogue warps of each CTA.
 // Every wait is bounded; a CTA that gives up raises its own and its peer's abort
-// flag, drains its own copies (and, on the even CTA, the issued MMAs), and both
-// meet at a final cluster barrier before the TMEM is released.
+// flag.  After an abort the even CTA drains its issued MMAs and the stages it
+// armed (which cover the odd CTA's copies of those stages); the odd CTA, which
+// cannot observe its copies on the peer's barrier, waits a fixed 2^21 cycles
+// (about a millisecond, orders of magnitude above a copy's latency) for any copy
+// of a stage the even CTA did not arm; both then meet at a final cluster barrier
+// before the TMEM is released.
 #pragma once
 #include "gemm_tc.cuh"
 
@@ -46,7 +49,7 @@ struct PairConfig {
   // A = tokens (K-major), B = weights (MN-major); M = 256 tokens, N = 256 columns
   static constexpr uint32_t IDESC = idesc_bf16(256, 256, false, true);
   static constexpr int THREADS = kTcBaseThreads;
-  static constexpr uint32_t BAR_BYTES = 8 * (3 * STAGES + 5) + 16 + 4 * STAGES;
+  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 20 * 4;
   static constexpr uint32_t SMEM_BYTES =
@@ -84,8 +87,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
-  uint64_t* pfull_bar = full_bar + STAGES;
-  uint64_t* empty_bar = pfull_bar + STAGES;
+  uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;       // [2]
   uint64_t* drain_bar = tempty_bar + 2;       // [1]
@@ -104,7 +106,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&pfull_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
       issued[s] = 0;
     }
@@ -148,6 +149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    const uint32_t full_even = mapa_shared(full_bar, 0);
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -169,11 +171,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
             break;
           }
           uint8_t* st = tiles + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          // the even CTA arms the stage for both CTAs' bytes
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE_BYTES);
           issued[stage] = (int)phase + 1;
-          tma_load_3d(st, wmap, &full_bar[stage], wn, kb * 64, ti.g);
-          tma_load_3d(st + 8192, wmap, &full_bar[stage], wn + 64, kb * 64, ti.g);
-          tma_load_2d(st + C::TOKEN_OFF, &P.tmB, &full_bar[stage], kb * 64, brow);
+          const uint32_t fb = full_even + stage * 8;
+          tma_load_3d_pair(st, wmap, fb, wn, kb * 64, ti.g);
+          tma_load_3d_pair(st + 8192, wmap, fb, wn + 64, kb * 64, ti.g);
+          tma_load_2d_pair(st + C::TOKEN_OFF, &P.tmB, fb, kb * 64, brow);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -197,8 +201,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
         for (int kb = 0; kb < kbl; ++kb) {
-          if (!pair_wait(&full_bar[stage], phase, p, abort_flag, peer_abort) ||
-              !pair_wait(&pfull_bar[stage], phase, p, abort_flag, peer_abort)) {
+          if (!pair_wait(&full_bar[stage], phase, p, abort_flag, peer_abort)) {
             ok = false;
             break;
           }
@@ -228,25 +231,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       tc2_commit(smem_u32(drain_bar));
       const long long t0 = clock64();
       while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kWaitCycles) {}
-    } else if (lane == 0) {
-      // ------------------------------------- forwarder (odd CTA): stage s landed here
-      const uint32_t pfull_peer = mapa_shared(pfull_bar, peer);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = pair; tile < total && ok; tile += npairs) {
-        TileInfo ti;
-        decode_tile(p, prefix, BN, TN, tile, ti);
-        const int kbl = p.prob[ti.prob].K / 64;
-        for (int kb = 0; kb < kbl; ++kb) {
-          if (!pair_wait(&full_bar[stage], phase, p, abort_flag, peer_abort)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_remote(pfull_peer + stage * 8);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        }
-      }
     }
     __syncwarp();
   } else {
@@ -279,14 +263,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
   // ---------------------------------------------------------------- teardown
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) {
-    // this CTA's copies still in flight after an abort: wait (bounded) for each
-    // stage's last load
-    for (int s = 0; s < STAGES; ++s) {
-      if (issued[s]) {
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&full_bar[s], (uint32_t)(issued[s] - 1)) &&
-               clock64() - t0 < kWaitCycles) {}
+    if (rank == 0) {
+      // the stages this CTA armed (both CTAs' copies): wait (bounded) for the
+      // last phase of each
+      for (int s = 0; s < STAGES; ++s) {
+        if (issued[s]) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait_cluster(&full_bar[s], (uint32_t)(issued[s] - 1)) &&
+                 clock64() - t0 < kWaitCycles) {}
+        }
       }
+    } else {
+      // copies of this CTA complete on the peer's barrier: give any still in
+      // flight a fixed, generous time to land
+      const long long t0 = clock64();
+      while (clock64() - t0 < (1ll << 21)) {}
     }
   }
   // neither CTA leaves while the pair's MMAs may still read its memory or write its
