@@ -248,6 +248,19 @@ MOE_DEV int total_tiles(const TcParams& p, const int* prefix, int TN) {
 
 MOE_DEV float silu_f(float u) { return __fdividef(u, 1.f + __expf(-u)); }
 
+// Tokens a swapped tile's MMA covers: its rows rounded up to the MMA's N step of
+// 16, at most the tile width BN.  A tile of a lightly loaded expert then costs MMA
+// time (and, with the in-GEMM gather, copies) for its own rows only, while the
+// heavily loaded experts get wide tiles that stream their weights fewer times.
+MOE_DEV int tile_n(int rows, int BN) {
+  const int n = (rows + 15) & ~15;
+  return n < 16 ? 16 : n > BN ? BN : n;
+}
+// the instruction descriptor with its N field (bits 17..22, N >> 3) replaced
+MOE_DEV uint32_t idesc_with_n(uint32_t idesc, int n) {
+  return (idesc & ~(0x3Fu << 17)) | ((uint32_t)(n >> 3) << 17);
+}
+
 // Dequantise one raw weight block (128 features x 64 k of tile (g, n, kb)) into the
 // bf16 MN-major layout with the 128-byte swizzle that a TMA load would have
 // produced: 16-byte chunk cc (8 features) of k-row k of 64-feature half h sits at
@@ -525,7 +538,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   constexpr int TN = C::TILE_N;
   const int out_tiles = total_tiles(p, prefix, TN);
   // split-K is compiled into the narrow swapped expert tiles only
-  constexpr bool kCanSplit = !DIRECT && EPI != EPI_ROUTER && BN <= 32;
+  constexpr bool kCanSplit = !DIRECT && EPI != EPI_ROUTER && BN <= 64;
   int S = 1;
   if (EPI == EPI_ROUTER && p.k_splits > 1) S = p.k_splits;
   if (kCanSplit && p.split_part != nullptr && out_tiles > 0) {
@@ -549,7 +562,10 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
     // arm stage `stage` of tile ti, k-block kb, and request everything but gathered rows
     auto issue_stage = [&](uint8_t* st, int stage, uint32_t phase, const TileInfo& ti,
                            const TcProblem& P, int kb, bool gather) {
-      mbar_arrive_expect_tx(&full_bar[stage], C::TX_BYTES);
+      // gathered rows: only the tile's own (rounded up to 16), 128 B each
+      mbar_arrive_expect_tx(&full_bar[stage],
+                            gather ? C::TX_BYTES - C::B_BYTES + 128u * tile_n(ti.rows, BN)
+                                   : C::TX_BYTES);
       issued[stage] = (int)phase + 1;
       // GATEUP: the up matrix at the same features; wide DOWN: features +128
       const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
@@ -605,7 +621,8 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         // this lane's four rows; rows past the segment repeat the tile's first row
         // (their accumulators are never stored)
         int rr[4] = {0, 0, 0, 0};
-        if (gather && lane < BN / 4) {
+        const int n_gather = gather ? tile_n(ti.rows, BN) / 4 : 0;   // copies of 4 rows
+        if (lane < n_gather) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int m = 4 * lane + j;
@@ -619,7 +636,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
           uint8_t* st = tiles + stage * C::STAGE_BYTES;
           if (lane == 0) issue_stage(st, stage, phase, ti, P, kb, gather);
           __syncwarp();   // the stage is armed before any gathered row can land
-          if (gather && lane < BN / 4)
+          if (lane < n_gather)
             tma_gather4(st + C::TOKEN_OFF + lane * 512, &P.tmB, &full_bar[stage], kb * 64,
                         rr[0], rr[1], rr[2], rr[3]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -643,6 +660,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+        const uint32_t idesc = DIRECT ? C::IDESC : idesc_with_n(C::IDESC, tile_n(ti.rows, BN));
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
           if (WQ != WQ_BF16 &&
@@ -660,17 +678,17 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
             const uint32_t accum = (kb != ti.kb0 || kk != 0);
             if (WQ != WQ_BF16) {
               const uint32_t a_tm = tmem_base + C::A_COL0 + aslot * C::A_SLOT_COLS + kk * 8;
-              tc_mma_f16_tmem_a(d_tmem, a_tm, xd, C::IDESC, accum);
-              if (NA == 2) tc_mma_f16_tmem_a(d_tmem + BN, a_tm + 32, xd, C::IDESC, accum);
+              tc_mma_f16_tmem_a(d_tmem, a_tm, xd, idesc, accum);
+              if (NA == 2) tc_mma_f16_tmem_a(d_tmem + BN, a_tm + 32, xd, idesc, accum);
             } else if (DIRECT) {
               const uint64_t wd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
               tc_mma_f16(d_tmem, xd, wd, C::IDESC, accum);   // N = 128 * NA at once
             } else {
               const uint64_t wd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
-              tc_mma_f16(d_tmem, wd, xd, C::IDESC, accum);
+              tc_mma_f16(d_tmem, wd, xd, idesc, accum);
               if (NA == 2) {
                 const uint64_t wd2 = sw128_desc(st_addr + C::A_BYTES + kk * 2048, 8192, 1024);
-                tc_mma_f16(d_tmem + BN, wd2, xd, C::IDESC, accum);
+                tc_mma_f16(d_tmem + BN, wd2, xd, idesc, accum);
               }
             }
           }

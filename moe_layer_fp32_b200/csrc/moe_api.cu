@@ -82,31 +82,33 @@ inline bool quantised(const moe_config* c) {
          c->expert_dtype == MOE_FP8;
 }
 
-// token-tile width of the expert GEMMs from the mean rows per expert.  Quantised
-// experts keep the weights on the MMA's M side at every batch; their widest tile
-// holds 96 tokens (two accumulators of 2 x 96 columns and two slots of dequantised
-// weights fill the 512 TMEM columns).
+// Token-tile width of the expert GEMMs.  Up to 64 rows per expert on average
+// (decode), the weights sit on the MMA's M side and a tile holds up to 16, 32 or
+// 64 tokens -- as many as one expert can receive (T, or C under expert choice) --
+// while each tile's MMA covers only its own rows (rounded up to 16): lightly
+// loaded experts cost no more than before and the heavily loaded ones of a skewed
+// routing stream their weights once per 64 rows instead of once per 16.  Wider
+// (prefill) batches put 128 tokens on M; quantised experts keep the weights on M
+// at every batch, their widest tile holding 96 tokens (two accumulators of
+// 2 x 96 columns and two slots of dequantised weights fill the 512 TMEM columns).
 int pick_bn(const moe_config* c) {
   const double mean = (double)n_slots(c) / c->E;
-  if (mean <= 16) return 16;
-  if (mean <= 32) return 32;
-  if (mean <= 64) return 64;
-  return quantised(c) ? 96 : 128;
+  if (mean > 64) return quantised(c) ? 96 : 128;
+  const int most = expert_choice(c) ? ec_capacity(c) : c->T;   // rows one expert can get
+  return most <= 16 ? 16 : most <= 32 ? 32 : 64;
 }
-// Quantised experts at prefill tile widths are dequantised once to bf16 in the
-// workspace (the in-loop dequantisation would repeat for every token tile of an
-// expert); decode tiles dequantise inside the GEMM main loop.
-// Token tiles up to this width gather their rows inside the gate/up GEMM
-// (tile::gather4, four rows per copy: a few copies per stage, hidden behind the
-// weight stream); wider tiles would be bound by the copy rate, so their rows are
-// gathered once by a kernel into xp and loaded as whole tiles.
-constexpr int kGather4MaxBN = 32;
-constexpr bool kGather4Int = false;   // int8 / int4 stages hold 4x fewer weight bytes
+// Decode tiles of bf16 experts gather their rows inside the gate/up GEMM
+// (tile::gather4, four rows per copy, only the tile's own rows: a few copies per
+// stage, hidden behind the weight stream); prefill tiles would be bound by the
+// copy rate, so their rows are gathered once by a kernel into xp and loaded as
+// whole tiles.
+constexpr int kGather4MaxBN = 64;
+constexpr bool kGather4Int = false;   // int8 / int4 / fp8 stages hold 2-4x fewer weight bytes
 inline bool gather_in_gemm(const moe_config* c) {
   return pick_bn(c) <= kGather4MaxBN && (kGather4Int || c->expert_dtype == MOE_BF16);
 }
-// Split-K of narrow (decode) tiles when the expert tiles fill at most half the SMs;
-// the GEMM decides per launch from the actual tile count.
+// Split-K of decode tiles when the expert tiles fill at most half the SMs; the
+// GEMM decides per launch from the actual tile count.
 constexpr bool kSplitBf16 = false;   // int experts only: bf16 tiles stream faster whole
 inline bool split_k(const moe_config* c) {
   return tc_experts(c) && pick_bn(c) <= kGather4MaxBN &&
