@@ -454,3 +454,46 @@ def test_single_launch_decode_layer_equals_the_kernel_chain(name):
     assert res.max_margin_mismatch < ROUTE_MARGIN
     assert res.err_ratio <= TOL[sh.expert], res.err_ratio
     print(f"{name}: err/rms(out) {res.err_ratio:.3e}, err/rms(delta) {res.err_ratio_delta:.3e}")
+
+
+def test_precision_of_bf16_rows_against_fp32_rows():
+    """The layer forward keeps the gated routed rows in bf16 between the down GEMM
+    and the combine; the grouped-FFN + combine entry points keep them in FP32.
+    Both are measured against the oracle on the MoE delta (out - x), the stricter
+    denominator: the bf16 rows may add at most their own rounding (relative 2^-9
+    per row, summed over k rows) to the error the FP32 rows have, which comes from
+    h rounded to bf16 before the down GEMM."""
+    sh, T = LayerShape("prec", d=1024, E=32, k=8, f=512, seed=61), 512
+    li, x, dli, dx = inputs_on_device(sh, T)
+    layer = M.MoELayer(dli, T, out_dtype="f32")
+    idx = torch.empty(T, sh.k, dtype=torch.int32, device="cuda")
+    fused = layer.forward(dx, topk_idx=idx).cpu().numpy()
+    cfg, w = layer.cfg, layer.w
+    ws = M.alloc_workspace(cfg)
+    xn = torch.empty(T, sh.d, dtype=torch.bfloat16, device="cuda")
+    logits = torch.empty(T, sh.E, dtype=torch.float32, device="cuda")
+    M.moe_rmsnorm_router(cfg, w, dx, xn, logits, ws)
+    tidx = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T * sh.k, dtype=torch.float32, device="cuda")
+    M.moe_route(cfg, logits, dli.router_bias, tidx, gate)
+    counts = torch.empty(sh.E, dtype=torch.int32, device="cuda")
+    offs = torch.empty(sh.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    slot = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    drop = torch.empty(1, dtype=torch.int32, device="cuda")
+    M.moe_permute(cfg, tidx, counts, offs, perm, slot, drop, ws)
+    y = torch.empty(T * sh.k, sh.d, dtype=torch.float32, device="cuda")
+    M.moe_grouped_ffn(cfg, w, xn, offs, perm, gate, y, None, ws)
+    chain = torch.empty(T, sh.d, dtype=torch.float32, device="cuda")
+    M.moe_combine(cfg, y, slot, None, dx, chain)
+    chain = chain.cpu().numpy()
+    rep = O.layer_from_inputs(li, x, forced_idx=idx.cpu().numpy())
+    delta = rep["out"] - x.float().numpy().astype(np.float64)
+    rd = float(np.sqrt(np.mean(delta ** 2)))
+    e_fused = float(np.max(np.abs(fused - rep["out"]))) / rd
+    e_chain = float(np.max(np.abs(chain - rep["out"]))) / rd
+    print(f"err/rms(delta): bf16 rows {e_fused:.3e}, FP32 rows {e_chain:.3e}")
+    assert e_chain <= DELTA_GUARD["bf16"] and e_fused <= DELTA_GUARD["bf16"]
+    # the bf16 rows' own rounding: |y_a| 2^-9 summed over the k rows of a token
+    bound = sh.k * 2.0 ** -9 * float(np.max(np.abs(y.cpu().numpy()))) / rd
+    assert e_fused <= e_chain + bound
