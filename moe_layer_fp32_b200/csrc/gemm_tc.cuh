@@ -97,6 +97,11 @@ struct TcParams {
   // at out + s * split_out_stride (the routing kernel adds the parts in order)
   int k_splits;
   size_t split_out_stride;
+  // problem 0 (routed, with offsets): interleave the tiles of light experts (one
+  // token tile) evenly between the token tiles of the heavy ones, so that tiles
+  // bound by streaming a light expert's weights run beside tiles bound by the
+  // tensor cores instead of all at once
+  int interleave;
 };
 
 constexpr int kMaxSplit = 4;
@@ -172,7 +177,9 @@ struct TcConfig {
                                                     : idesc_bf16(128, BN, false, false);
   // barriers + bookkeeping after the tiles
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * 2) + 16 + 4 * STAGES;
-  static constexpr uint32_t PREFIX_BYTES = 2 * (kMaxGroups + 1) * 4;
+  // tile prefixes of the two problems, then the heavy / light class prefixes of
+  // problem 0 (interleaved order)
+  static constexpr uint32_t PREFIX_BYTES = 4 * (kMaxGroups + 1) * 4;
   // swapped epilogue: per-tile output row and scale of each token, one copy per warp;
   // direct DOWN epilogue: a 32-row x 16-column FP32 staging tile per warp (rows
   // padded to 20 floats) through which rows are stored transposed
@@ -209,9 +216,28 @@ MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int TN, i
   const int mt = tile / nt;
   ti.prob = pi;
   ti.n0 = (tile % nt) * TN;
-  const int g = find_group(pre, P.G, mt);
+  int g;
+  if (pi == 0 && p.interleave) {
+    // position mt of the interleaved sequence: light tile number floor(mt L / N)
+    // when that count steps up at mt, else heavy tile number mt - that count
+    const int* hpre = prefix + 2 * (kMaxGroups + 1);
+    const int* lpre = prefix + 3 * (kMaxGroups + 1);
+    const int L = lpre[P.G], N = pre[P.G];
+    const int lb = (int)((long long)mt * L / N);
+    const int la = (int)((long long)(mt + 1) * L / N);
+    if (la > lb) {
+      g = find_group(lpre, P.G, lb);
+      ti.m0 = 0;
+    } else {
+      const int h = mt - lb;
+      g = find_group(hpre, P.G, h);
+      ti.m0 = (h - hpre[g]) * BN;
+    }
+  } else {
+    g = find_group(pre, P.G, mt);
+    ti.m0 = (mt - pre[g]) * BN;
+  }
   ti.g = g;
-  ti.m0 = (mt - pre[g]) * BN;
   int seg_start, seg_rows;
   if (P.offsets) {
     seg_start = P.offsets[g];
@@ -490,7 +516,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
       reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
   // epilogue scratch, 16-byte aligned (float4 staging in the direct DOWN epilogue)
   int* epi_row = reinterpret_cast<int*>(
-      (reinterpret_cast<uintptr_t>(prefix + 2 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(prefix + 4 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
   float* epi_scale = reinterpret_cast<float*>(epi_row + kEpiWarps * 128);  // [8 warps][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -531,6 +557,9 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
     const TcProblem& P = p.prob[warp - 2];
     group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1));
   }
+  if (warp == 4 && p.interleave)
+    group_class_prefix(p.prob[0].offsets, p.prob[0].G, BN, prefix + 2 * (kMaxGroups + 1),
+                       prefix + 3 * (kMaxGroups + 1));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

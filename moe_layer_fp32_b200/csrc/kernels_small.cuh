@@ -46,6 +46,29 @@ MOE_DEV void group_tile_prefix(const int32_t* off, int G, int uniform, int BM, i
     carry += __shfl_sync(0xffffffffu, v, 31);
   }
 }
+// Tile prefixes of the two classes of groups of a grouped problem with offsets:
+// light groups (1..BM rows, one tile) and heavy groups (more rows).  hpre[g] =
+// tiles of heavy groups < g, lpre[g] = light groups < g.  One warp.
+MOE_DEV void group_class_prefix(const int32_t* off, int G, int BM, int* hpre, int* lpre) {
+  const int lane = threadIdx.x & 31;
+  int ch = 0, cl = 0;
+  if (lane == 0) { hpre[0] = 0; lpre[0] = 0; }
+  for (int c = 0; c < G; c += 32) {
+    const int g = c + lane;
+    const int rows = g < G ? off[g + 1] - off[g] : 0;
+    const int t = (rows + BM - 1) / BM;
+    int h = t > 1 ? t : 0, l = t == 1 ? 1 : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yh = __shfl_up_sync(0xffffffffu, h, o);
+      const int yl = __shfl_up_sync(0xffffffffu, l, o);
+      if (lane >= o) { h += yh; l += yl; }
+    }
+    if (g < G) { hpre[g + 1] = ch + h; lpre[g + 1] = cl + l; }
+    ch += __shfl_sync(0xffffffffu, h, 31);
+    cl += __shfl_sync(0xffffffffu, l, 31);
+  }
+}
 // group of tile-row `mt`: largest g with prefix[g] <= mt
 MOE_DEV int find_group(const int* prefix, int G, int mt) {
   int lo = 0, hi = G - 1;

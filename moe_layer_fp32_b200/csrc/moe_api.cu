@@ -115,6 +115,12 @@ inline bool split_k(const moe_config* c) {
          (kSplitBf16 || c->expert_dtype != MOE_BF16);
 }
 inline int split_counters() { return num_sms() * 8; }
+// Prefill tiles of bf16 experts take the interleaved tile order (light experts'
+// tiles spread between the heavy ones'); it changes nothing when every expert
+// fills more than one tile.
+inline bool interleave_tiles(const moe_config* c) {
+  return c->expert_dtype == MOE_BF16 && pick_bn(c) == 128;
+}
 // Inside the layer forward the gated routed rows of tensor-core experts are kept
 // in bf16 (half the bytes the down GEMM writes and the combine reads); the
 // grouped-FFN and combine entry points exchange them in FP32.
@@ -687,6 +693,7 @@ moe_status gateup_params(const moe_config* c, const moe_weights* w, const moe_we
   p.wait_cycles = wait_cycles(c);
   p.split_part = split_part;
   p.split_cnt = split_cnt;
+  p.interleave = interleave_tiles(c);
   return MOE_OK;
 }
 
@@ -747,6 +754,7 @@ moe_status down_params(const moe_config* c, const moe_weights* w, const moe_weig
   p.wait_cycles = wait_cycles(c);
   p.split_part = split_part;
   p.split_cnt = split_cnt;
+  p.interleave = interleave_tiles(c);
   return MOE_OK;
 }
 
