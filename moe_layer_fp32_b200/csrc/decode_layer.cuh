@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ int s_ok;
-  __shared__ double red[kDecodeThreads / 32];
+  __shared__ double red[8];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -194,8 +194,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   bool ok = true;
   // 1. RMSNorm
   for (int t = blockIdx.x; t < p.T; t += nb)
-    rmsnorm_row_bf16v<kDecodeThreads, MAXV>(p.x + (size_t)t * p.d, p.gamma,
-                                            p.xn + (size_t)t * p.d, p.d, p.eps, red);
+    rmsnorm_row_bf16v<256, MAXV>(p.x + (size_t)t * p.d, p.gamma, p.xn + (size_t)t * p.d, p.d,
+                                 p.eps, red);   // the chain's partition: identical bits
   ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
   // 2. router partial logits: work item (token group of 8, K-slice)
   if (ok) {

@@ -127,16 +127,18 @@ MOE_DEV void unpack8(const uint4& u, float (&f)[8]) {
   for (int i = 0; i < 4; ++i) { f[2 * i] = __low2float(h[i]); f[2 * i + 1] = __high2float(h[i]); }
 }
 
-// One token row, vectorised: thread i of the NT calling threads keeps up to MAXV
-// 16-byte vectors of the row in registers between the sum of squares and the
-// scaling pass (d up to NT * MAXV * 8).  `red` is a shared scratch of NT / 32
-// doubles.  Same arithmetic as k_rmsnorm; all NT threads call it.
+// One token row, vectorised: thread i < NT keeps up to MAXV 16-byte vectors of the
+// row in registers between the sum of squares and the scaling pass (d up to
+// NT * MAXV * 8).  `red` is a shared scratch of NT / 32 doubles.  Same arithmetic
+// as k_rmsnorm.  Every thread of the CTA calls it (the CTA may have more than NT
+// threads; the others only join its barriers), and the partition of the row over
+// the NT threads -- hence the order of the double sum -- depends on NT alone.
 template <int NT, int MAXV>
 MOE_DEV void rmsnorm_row_bf16v(const __nv_bfloat16* __restrict__ xrow,
                                const float* __restrict__ gamma,
                                __nv_bfloat16* __restrict__ xnrow, int d, double eps,
                                double* red) {
-  const int nv = d / 8;
+  const int nv = threadIdx.x < NT ? d / 8 : 0;
   const uint4* xr = reinterpret_cast<const uint4*>(xrow);
   uint4* outr = reinterpret_cast<uint4*>(xnrow);
   uint4 buf[MAXV];
@@ -153,7 +155,7 @@ MOE_DEV void rmsnorm_row_bf16v(const __nv_bfloat16* __restrict__ xrow,
     }
   }
   s = warp_sum(s);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  if ((threadIdx.x & 31) == 0 && threadIdx.x < NT) red[threadIdx.x >> 5] = s;
   __syncthreads();
   double tot = 0.0;
 #pragma unroll

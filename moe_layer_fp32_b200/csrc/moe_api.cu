@@ -956,7 +956,7 @@ constexpr size_t kGridBarOff = 64;
 // experts with a bf16 router of at most 256 experts, 16-byte aligned tensors.
 bool single_launch(const moe_config* c) {
   return !expert_choice(c) && c->T <= kDecodeMaxT && c->expert_dtype == MOE_BF16 &&
-         vec_router(c) && c->E <= 256 && gather_in_gemm(c) && c->d <= kDecodeThreads * 4 * 8;
+         vec_router(c) && c->E <= 256 && gather_in_gemm(c) && c->d <= 256 * 4 * 8;
 }
 
 template <int EPL, int BN>
