@@ -40,6 +40,8 @@ struct DecodeParams {
   int32_t* slot;                  // [T * k]
   int32_t* dropped;               // [1]
   float* logits_out;              // [T, E] or nullptr
+  const uint8_t* w_down;          // [E, f, d] bf16 routed experts' down weights
+  const uint8_t* sh_down;         // [S, f, d] or nullptr
   const __nv_bfloat16* y;         // [T * k, d] gated routed rows (written by the down GEMM)
   const float* ys;                // [S, T, d]
   void* out;                      // [T, d] bf16 or fp32
@@ -220,7 +222,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
   }
-  // 4. + 5. the expert GEMMs
+  // 4. + 5. the expert GEMMs.  The CTAs that get no gate/up tile first bring the
+  // touched experts' down weights into L2, 32 KB per prefetch, spread over them,
+  // so that the down step starts on warm lines while gate/up streams its own.
+  if (ok && warp == 0) {
+    const int nt = p.dn.prob[0].K / 128;   // gate/up feature tiles per token tile (f / 128)
+    int gu_tiles = 0;
+    for (int g = lane; g < p.E; g += 32) {
+      const int rows = p.offsets[g + 1] - p.offsets[g];
+      gu_tiles += (rows + BN - 1) / BN;
+    }
+    gu_tiles = warp_sum(gu_tiles) * nt + p.S * ((p.T + BN - 1) / BN) * nt;
+    const int idle = nb - gu_tiles, me = (int)blockIdx.x - gu_tiles;
+    if (me >= 0) {
+      constexpr uint32_t kChunk = 32 * 1024;
+      const size_t per = (size_t)p.dn.prob[0].K * p.d * 2;   // one expert's W_down bytes
+      const uint32_t chunks = (uint32_t)(per / kChunk);        // f, d multiples of 128: exact
+      uint32_t c0 = 0;                                         // chunks of the experts before
+      for (int g = 0; g < p.E + p.S; ++g) {
+        const bool routed = g < p.E;
+        if (routed && p.offsets[g + 1] == p.offsets[g]) continue;
+        const uint8_t* base = routed ? p.w_down + (size_t)g * per : p.sh_down + (size_t)(g - p.E) * per;
+        // chunk j of this expert goes to idle CTA (c0 + j) % idle
+        for (uint32_t j = (uint32_t)lane; j < chunks; j += 32)
+          if ((int)((c0 + j) % (uint32_t)idle) == me) prefetch_l2_bulk(base + (size_t)j * kChunk, kChunk);
+        c0 += chunks;
+      }
+    }
+  }
   if (ok) {
     tc_gemm_run<EPI_GATEUP, BN, false, WQ_BF16>(p.gu, smem, &tmem_slot, blockIdx.x, nb, false);
     ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);

@@ -1023,6 +1023,8 @@ moe_status run_decode_layer(const moe_config* c, const moe_weights* w, const voi
   dp.slot = at<int32_t>(ws, L.slot);
   dp.dropped = at<int32_t>(ws, L.dropped);
   dp.logits_out = logits_out;
+  dp.w_down = static_cast<const uint8_t*>(w->w_down);
+  dp.sh_down = static_cast<const uint8_t*>(w->sh_down);
   dp.y = static_cast<const __nv_bfloat16*>(y);
   dp.ys = ys;
   dp.out = out;
