@@ -8,7 +8,8 @@
 // grid-wide barriers:
 //   1. RMSNorm, one token per CTA;
 //   2. the router's K-sliced partial logits, (8 tokens x 128 rows) per work item;
-//   3. routing (a warp per token) and the counting-sort permutation, in CTA 0;
+//   3. routing, one token per CTA, then -- without a barrier -- the counting-sort
+//      permutation, built by every CTA (it is small);
 //   4. the grouped gate/up GEMM over the routed rows (tcgen05, 16 or 32 token
 //      tiles, rows gathered by the GEMM's own TMA);
 //   5. the grouped down GEMM (gated bf16 rows of every assignment);
@@ -208,19 +209,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                          (w % groups) * 8, w / groups, sm_r);
     ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
   }
-  // 3. routing and the permutation (CTA 0)
+  // 3. routing: CTA t routes token t -- every thread adds one expert's partial
+  //    logits in slice order, then warp 0 selects
   if (ok) {
-    if (blockIdx.x == 0) {
-      for (int t = warp; t < p.T; t += kDecodeThreads / 32)
-        route_token<EPL>(p.part, p.ns, p.T, p.E, p.k, p.bias, p.mode, p.renorm, p.idx, p.gate,
-                         p.logits_out, t, lane);
+    float* s_lg = reinterpret_cast<float*>(smem);
+    for (int t = blockIdx.x; t < p.T; t += nb) {
+      for (int e = threadIdx.x; e < p.E; e += kDecodeThreads) {
+        const float* pe = p.part + (size_t)t * p.E + e;
+        const size_t stride = (size_t)p.T * p.E;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int sl = 0; sl < p.ns; ++sl) acc += pe[sl * stride];
+        s_lg[e] = acc;
+      }
       __syncthreads();
-      if (warp == 0)
-        permute_warp(p.idx, p.T * p.k, p.E, p.cap, p.counts, p.offsets, p.perm, p.slot,
-                     p.dropped, p.err, reinterpret_cast<int*>(smem),
-                     reinterpret_cast<int*>(smem) + p.E);
+      if (warp == 0) {
+        float lg[EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) lg[i] = lane + 32 * i < p.E ? s_lg[lane + 32 * i] : 0.f;
+        route_select<EPL>(lg, p.E, p.k, p.bias, p.mode, p.renorm, p.idx, p.gate, p.logits_out,
+                          t, lane);
+      }
+      __syncthreads();
     }
     ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
+  }
+  // the permutation of the T*k <= 1024 assignments: every CTA builds it (one warp),
+  // writing the same values to the workspace, and reads back only what it wrote
+  // itself -- so no CTA waits for another before its gate/up tiles
+  if (ok) {
+    if (warp == 0)
+      permute_warp(p.idx, p.T * p.k, p.E, p.cap, p.counts, p.offsets, p.perm, p.slot, p.dropped,
+                   blockIdx.x == 0 ? p.err : nullptr, reinterpret_cast<int*>(smem),
+                   reinterpret_cast<int*>(smem) + p.E);
+    __syncthreads();
   }
   // 4. + 5. the expert GEMMs.  The CTAs that get no gate/up tile first bring the
   // touched experts' down weights into L2, 32 KB per prefetch, spread over them,

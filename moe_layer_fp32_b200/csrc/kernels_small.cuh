@@ -367,13 +367,12 @@ MOE_DEV void router_logits_of_lane(const float* part, int ns, int T, int E, int 
   }
 }
 
-// Routes token t with the calling warp.
+// Routes token t with the calling warp, from its logits lg (lane holds experts
+// lane, lane + 32, ...).
 template <int EPL>
-MOE_DEV void route_token(const float* part, int ns, int T, int E, int k, const float* bias,
-                         int mode, int renorm, int32_t* idx, float* gate, float* logits_out,
-                         int t, int lane) {
-  float lg[EPL];
-  router_logits_of_lane<EPL>(part, ns, T, E, t, lane, lg);
+MOE_DEV void route_select(const float (&lg)[EPL], int E, int k, const float* bias, int mode,
+                          int renorm, int32_t* idx, float* gate, float* logits_out, int t,
+                          int lane) {
   float key[EPL], pin[EPL];
   float mx = -INFINITY;
 #pragma unroll
@@ -438,6 +437,17 @@ MOE_DEV void route_token(const float* part, int ns, int T, int E, int k, const f
     idx[(size_t)t * k + lane] = my_e;
     gate[(size_t)t * k + lane] = my_p;
   }
+}
+
+// Routes token t with the calling warp: the router partials added in slice order,
+// then the selection.
+template <int EPL>
+MOE_DEV void route_token(const float* part, int ns, int T, int E, int k, const float* bias,
+                         int mode, int renorm, int32_t* idx, float* gate, float* logits_out,
+                         int t, int lane) {
+  float lg[EPL];
+  router_logits_of_lane<EPL>(part, ns, T, E, t, lane, lg);
+  route_select<EPL>(lg, E, k, bias, mode, renorm, idx, gate, logits_out, t, lane);
 }
 
 template <int EPL>
