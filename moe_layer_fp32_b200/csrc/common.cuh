@@ -142,12 +142,16 @@ MOE_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and records DEV_TIMEOUT, and raises *abort) if it did not within `limit`
-// clock cycles or if another role already raised *abort.
+// clock cycles or if another role already raised *abort.  A patient wait (one
+// that usually lasts a whole tile, such as the epilogue's wait for its
+// accumulator) sleeps between polls, leaving the issue slots -- and the power --
+// to the warps on the critical path.
 MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort,
-                       long long limit) {
+                       long long limit, bool patient = false) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
+    if (patient) __nanosleep(128);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > limit) {
@@ -322,10 +326,12 @@ MOE_DEV uint32_t mapa_shared(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
-// arrive on an mbarrier of another CTA of the cluster (cluster-scope release)
+// arrive on an mbarrier of another CTA of the cluster.  Used to hand a drained
+// TMEM accumulator back to the pair's MMA issuer: the caller has completed its
+// TMEM loads (tcgen05.wait::ld) and fenced them (tcgen05.fence::before_thread_sync),
+// so the arrival needs no memory fence of its own.
 MOE_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 MOE_DEV void st_shared_remote_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");

@@ -51,19 +51,21 @@ struct PairConfig {
   static constexpr int THREADS = kTcBaseThreads;
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 4 * (kMaxGroups + 1) * 4;
-  static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 20 * 4;
+  static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 16 * 4;
   static constexpr uint32_t SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
   static_assert(SMEM_BYTES + 64 <= 227 * 1024, "shared memory per CTA (dynamic + static)");
   static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 128-byte swizzle alignment");
 };
 
-// Bounded wait of a pair kernel: on time-out it also raises the peer's abort flag.
+// Bounded wait of a pair kernel: on time-out it also raises the peer's abort flag;
+// a patient wait sleeps between polls (see mbar_wait).
 MOE_DEV bool pair_wait(uint64_t* bar, uint32_t parity, const TcParams& p, volatile int* abort,
-                       uint32_t peer_abort) {
+                       uint32_t peer_abort, bool patient = false) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
+    if (patient) __nanosleep(128);
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > p.wait_cycles) {
@@ -240,7 +242,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int half = (warp - 2) >> 2;       // which half of the columns it drains
-    float* stg = stg_all + (warp - 2) * (32 * 20);
+    float* stg = stg_all + (warp - 2) * (32 * 16);
     const uint32_t tempty_even = mapa_shared(tempty_bar, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -252,7 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       int r;
       float sc;
       direct_row<EPI>(P, ti, 128 * (int)rank + q * 32 + lane, r, sc);
-      if (!pair_wait(&tfull_bar[acc], acc_phase, p, abort_flag, peer_abort)) break;
+      if (!pair_wait(&tfull_bar[acc], acc_phase, p, abort_flag, peer_abort, true)) break;
       tc_fence_after();
       direct_store<EPI, TN>(P, ti, r, sc, t_base, half, lane, stg);
       tc_fence_before();

@@ -159,11 +159,16 @@ struct TcConfig {
   static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
   static constexpr uint32_t A_REGION = 0;
   static constexpr uint32_t ACC_COLS = NA * BN;
-  // TMEM: two accumulators, then (quantised weights) two slots of NA bf16 weight
-  // blocks, 128 lanes x 32 columns each (64 k, two per 32-bit column)
+  // TMEM: two accumulators, then (quantised weights) A_SLOTS slots of NA bf16
+  // weight blocks, 128 lanes x 32 columns each (64 k, two per 32-bit column)
   static constexpr uint32_t A_COL0 = 2 * ACC_COLS;
   static constexpr uint32_t A_SLOT_COLS = WQ == WQ_BF16 ? 0 : NA * 32;
-  static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS + 2 * A_SLOT_COLS;
+  // as many weight slots as the TMEM left by the accumulators holds, at most 4, so
+  // that the dequantisation warps run up to 4 k-blocks ahead of the MMA
+  static constexpr int A_SLOTS_FIT =
+      WQ == WQ_BF16 ? 2 : (int)((512 - 2 * ACC_COLS) / (A_SLOT_COLS ? A_SLOT_COLS : 1));
+  static constexpr int A_SLOTS = WQ == WQ_BF16 ? 2 : A_SLOTS_FIT > 4 ? 4 : A_SLOTS_FIT;
+  static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS + A_SLOTS * A_SLOT_COLS;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                         : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   // swapped: A = weights, M = 128 features, N = BN tokens (K-major), one MMA per
@@ -176,15 +181,15 @@ struct TcConfig {
                                     : WQ == WQ_BF16 ? idesc_bf16(128, BN, true, false)
                                                     : idesc_bf16(128, BN, false, false);
   // barriers + bookkeeping after the tiles
-  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * 2) + 16 + 4 * STAGES;
+  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * A_SLOTS) + 16 + 4 * STAGES;
   // tile prefixes of the two problems, then the heavy / light class prefixes of
   // problem 0 (interleaved order)
   static constexpr uint32_t PREFIX_BYTES = 4 * (kMaxGroups + 1) * 4;
   // swapped epilogue: per-tile output row and scale of each token, one copy per warp;
-  // direct DOWN epilogue: a 32-row x 16-column FP32 staging tile per warp (rows
-  // padded to 20 floats) through which rows are stored transposed
+  // direct DOWN epilogue: a 32-row x 16-column FP32 staging tile per warp through
+  // which rows are stored transposed
   static constexpr uint32_t EPI_BYTES =
-      (EPI == EPI_DOWN && DIRECT) ? kEpiWarps * 32 * 20 * 4 : kEpiWarps * 128 * 8;
+      (EPI == EPI_DOWN && DIRECT) ? kEpiWarps * 32 * 16 * 4 : kEpiWarps * 128 * 8;
   static constexpr uint32_t SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + A_REGION + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
   static_assert(SMEM_BYTES + 64 <= 227 * 1024, "shared memory per CTA (dynamic + static)");
@@ -412,11 +417,17 @@ MOE_DEV void direct_row(const TcProblem& P, const TileInfo& ti, int m, int& r, f
   }
 }
 
+// Staging tile of the direct DOWN epilogue: 32 rows x 16 floats per warp, the four
+// 16-byte pieces of row r stored in the order j ^ ((r >> 1) & 3), so that the
+// lane-per-row writes and the row-striped reads of both output types hit 32
+// distinct banks per 8 lanes.
+MOE_DEV int stg_at(int r, int j) { return r * 16 + 4 * (j ^ ((r >> 1) & 3)); }
+
 // Direct-orientation epilogue: this thread holds TMEM lane (q*32 + lane) of the
 // accumulator at t_base, i.e. one token row, whose output row is r (-1: none).
 // GATEUP: 128 features, gate in columns [0,128), up in [128,256); each half of the
 // warps takes 64 features and writes bf16 h.  DOWN: TN features, half each, scaled
-// by the gate and stored through the warp's staging tile `stg` (32 rows x 20 floats).
+// by the gate and stored through the warp's staging tile `stg` (32 rows x 16 floats).
 template <int EPI, int TN>
 MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float sc,
                           uint32_t t_base, int half, int lane, float* stg) {
@@ -447,11 +458,11 @@ MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float s
       // then several lanes store one row's contiguous bytes (FP32: 4 lanes x 16 B,
       // 8 rows per instruction; bf16: 2 lanes x 16 B, 16 rows per instruction), so
       // every store fills whole 32-byte sectors.
-      float4* srow = reinterpret_cast<float4*>(stg + lane * 20);
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        srow[j] = make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
-                              v0[4 * j + 3] * sc);
+        *reinterpret_cast<float4*>(stg + stg_at(lane, j)) =
+            make_float4(v0[4 * j] * sc, v0[4 * j + 1] * sc, v0[4 * j + 2] * sc,
+                        v0[4 * j + 3] * sc);
       __syncwarp();
       if (P.out_bf16) {
         const int hh = (lane & 1) * 8;
@@ -459,8 +470,8 @@ MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float s
         for (int i = 0; i < 2; ++i) {
           const int rr = (lane >> 1) + 16 * i;
           const int rout = __shfl_sync(0xffffffffu, r, rr);
-          const float4 a = *reinterpret_cast<const float4*>(stg + rr * 20 + hh);
-          const float4 b = *reinterpret_cast<const float4*>(stg + rr * 20 + hh + 4);
+          const float4 a = *reinterpret_cast<const float4*>(stg + stg_at(rr, 2 * (lane & 1)));
+          const float4 b = *reinterpret_cast<const float4*>(stg + stg_at(rr, 2 * (lane & 1) + 1));
           __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y);
           __nv_bfloat162 h1 = __floats2bfloat162_rn(a.z, a.w);
           __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y);
@@ -477,7 +488,7 @@ MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float s
         for (int i = 0; i < 4; ++i) {
           const int rr = (lane >> 2) + 8 * i;
           const int rout = __shfl_sync(0xffffffffu, r, rr);
-          const float4 v = *reinterpret_cast<const float4*>(stg + rr * 20 + qq);
+          const float4 v = *reinterpret_cast<const float4*>(stg + stg_at(rr, lane & 3));
           if (rout >= 0)
             *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + (size_t)rout * P.ld_out +
                                        n + qq) = v;
@@ -508,9 +519,9 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;       // [2]
   uint64_t* drain_bar = tempty_bar + 2;       // [1]
-  uint64_t* deq_bar = drain_bar + 1;          // [2] dequantised slot filled
-  uint64_t* aempty_bar = deq_bar + 2;         // [2] dequantised slot consumed
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(aempty_bar + 2) + 1;
+  uint64_t* deq_bar = drain_bar + 1;                   // [A_SLOTS] weight slot filled
+  uint64_t* aempty_bar = deq_bar + C::A_SLOTS;         // [A_SLOTS] weight slot consumed
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(aempty_bar + C::A_SLOTS) + 1;
   int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
   int* prefix = reinterpret_cast<int*>(
       reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
@@ -527,7 +538,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
       mbar_init(&empty_bar[s], 1);
       issued[s] = 0;
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < C::A_SLOTS; ++a) {
       mbar_init(&deq_bar[a], C::DEQ_WARPS);
       mbar_init(&aempty_bar[a], 1);
     }
@@ -725,7 +736,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
           if (WQ != WQ_BF16) {
             tc_commit(&aempty_bar[aslot]);
-            if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+            if (++aslot == C::A_SLOTS) { aslot = 0; aphase ^= 1; }
           }
         }
         if (!ok) break;
@@ -773,7 +784,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
           __syncwarp();
           if (lane == 0) mbar_arrive(&deq_bar[aslot]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
-          if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+          if (++aslot == C::A_SLOTS) { aslot = 0; aphase ^= 1; }
         }
       }
     }
@@ -796,10 +807,10 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         int r;
         float sc;
         direct_row<EPI>(P, ti, q * 32 + lane, r, sc);
-        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles)) break;
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles, true)) break;
         tc_fence_after();
         direct_store<EPI, TN>(P, ti, r, sc, t_base, half, lane,
-                              reinterpret_cast<float*>(epi_row) + (warp - 2) * (32 * 20));
+                              reinterpret_cast<float*>(epi_row) + (warp - 2) * (32 * 16));
       } else {
         // swapped: this thread owns feature n; the tile's token rows and scales are
         // staged in this warp's shared-memory slice (warp-private: __syncwarp only)
@@ -819,7 +830,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
           s_scale[m] = sc;
         }
         __syncwarp();
-        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles)) break;
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles, true)) break;
         tc_fence_after();
         const int n = ti.n0 + q * 32 + lane;
         const bool n_ok = n < P.n_valid;
