@@ -35,7 +35,7 @@ class MoeConfig(ctypes.Structure):
                 ("act_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
                 ("router_dtype", ctypes.c_int32), ("expert_dtype", ctypes.c_int32),
                 ("group_size", ctypes.c_int32), ("wait_kcycles", ctypes.c_int32),
-                ("routing", ctypes.c_int32)]
+                ("routing", ctypes.c_int32), ("prefill_tiles", ctypes.c_int32)]
 
 
 class MoeWeights(ctypes.Structure):

@@ -30,8 +30,8 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, defines=()) -> str:
-    """Compile the library; ``defines`` are extra NAME=VALUE build options (for
-    example MOE_PAIR_TILES=0 selects the single-CTA prefill GEMM)."""
+    """Compile the library; ``defines`` are extra NAME=VALUE preprocessor options
+    passed to nvcc as -D flags (a rebuild is forced when any are given)."""
     if not force and not defines and up_to_date():
         return OUT
     nvcc = os.environ.get("NVCC", "nvcc")

@@ -149,6 +149,7 @@ moe_status validate(const moe_config* c) {
   if (c->wait_kcycles < 0) return MOE_ERR_INVALID;
   if (c->routing != MOE_ROUTE_TOPK && c->routing != MOE_ROUTE_EXPERT_CHOICE)
     return MOE_ERR_INVALID;
+  if (c->prefill_tiles != 0 && c->prefill_tiles != 1) return MOE_ERR_INVALID;
   if (c->routing == MOE_ROUTE_EXPERT_CHOICE) {
     // the expert picks rank tokens by their gate probability: a selection-only bias
     // has no meaning there; the FP32 (CUDA-core) experts take the top-k path only
@@ -369,13 +370,6 @@ moe_status launch_tc(const TcParams& p, cudaStream_t st) {
   return check_launch();
 }
 
-// Prefill tiles of bf16 experts run on CTA pairs (256 tokens per tile, one
-// cta_group::2 MMA per k-step) unless the library is built with MOE_PAIR_TILES=0.
-#ifndef MOE_PAIR_TILES
-#define MOE_PAIR_TILES 1
-#endif
-constexpr bool kPairTiles = MOE_PAIR_TILES != 0;
-
 // CTA pairs that can be resident at once.  A cluster's two CTAs must sit in one
 // GPC, so a GPC with an odd number of free SMs leaves one idle: the persistent
 // grid must not ask for more pairs than fit, or the last ones would run as a
@@ -412,15 +406,17 @@ moe_status launch_pair(const TcParams& p, cudaStream_t st) {
   return check_launch();
 }
 
+// Prefill tiles of bf16 experts run on CTA pairs (256 tokens per tile, one
+// cta_group::2 MMA per k-step) unless moe_config.prefill_tiles asks for single CTAs.
 template <int EPI, int WQ>
-moe_status launch_tc_bn_q(int bn, const TcParams& p, cudaStream_t st) {
+moe_status launch_tc_bn_q(int bn, bool pair, const TcParams& p, cudaStream_t st) {
   switch (bn) {
     case 16: return launch_tc<EPI, 16, false, WQ>(p, st);
     case 32: return launch_tc<EPI, 32, false, WQ>(p, st);
     case 64: return launch_tc<EPI, 64, false, WQ>(p, st);
     default:   // prefill tiles
       if constexpr (WQ == WQ_BF16) {   // tokens on MMA-M
-        if (kPairTiles) return launch_pair<EPI>(p, st);
+        if (pair) return launch_pair<EPI>(p, st);
         return launch_tc<EPI, 128, true, WQ>(p, st);
       } else {                         // quantised: weights on M, 96 tokens on N
         return launch_tc<EPI, 96, false, WQ>(p, st);
@@ -429,11 +425,11 @@ moe_status launch_tc_bn_q(int bn, const TcParams& p, cudaStream_t st) {
 }
 
 template <int EPI>
-moe_status launch_tc_bn(int bn, int wq, const TcParams& p, cudaStream_t st) {
-  if (wq == WQ_INT8) return launch_tc_bn_q<EPI, WQ_INT8>(bn, p, st);
-  if (wq == WQ_INT4) return launch_tc_bn_q<EPI, WQ_INT4>(bn, p, st);
-  if (wq == WQ_FP8) return launch_tc_bn_q<EPI, WQ_FP8>(bn, p, st);
-  return launch_tc_bn_q<EPI, WQ_BF16>(bn, p, st);
+moe_status launch_tc_bn(int bn, int wq, bool pair, const TcParams& p, cudaStream_t st) {
+  if (wq == WQ_INT8) return launch_tc_bn_q<EPI, WQ_INT8>(bn, pair, p, st);
+  if (wq == WQ_INT4) return launch_tc_bn_q<EPI, WQ_INT4>(bn, pair, p, st);
+  if (wq == WQ_FP8) return launch_tc_bn_q<EPI, WQ_FP8>(bn, pair, p, st);
+  return launch_tc_bn_q<EPI, WQ_BF16>(bn, pair, p, st);
 }
 
 
@@ -840,7 +836,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     if ((s = gateup_params(c, w, wl, wq, xn, xp, offsets, rr, h, split_part, split_cnt, err, p)) !=
         MOE_OK)
       return s;
-    s = launch_tc_bn<EPI_GATEUP>(bn, wq, p, st);
+    s = launch_tc_bn<EPI_GATEUP>(bn, wq, c->prefill_tiles == 0, p, st);
     if (s != MOE_OK) return s;
     mk->mark(st);
   }
@@ -849,7 +845,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     if ((s = down_params(c, w, wl, wq, offsets, rr, gate, h, y, rows_bf16, ys, split_part,
                          split_cnt, err, p)) != MOE_OK)
       return s;
-    s = launch_tc_bn<EPI_DOWN>(bn, wq, p, st);
+    s = launch_tc_bn<EPI_DOWN>(bn, wq, c->prefill_tiles == 0, p, st);
     mk->mark(st);
   }
   return s;

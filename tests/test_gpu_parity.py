@@ -456,6 +456,38 @@ def test_single_launch_decode_layer_equals_the_kernel_chain(name):
     print(f"{name}: err/rms(out) {res.err_ratio:.3e}, err/rms(delta) {res.err_ratio_delta:.3e}")
 
 
+PREFILL_TILES = {
+    "bf16_prefill_tiles": (SMALL["bf16_prefill_tiles"], 1000),
+    "bf16_prefill_skew": (SMALL["bf16_prefill_skew"], 700),
+    # several full tiles per expert and a ragged last one on each (1500 x 4 / 8 =
+    # 750 mean rows: 2 pair tiles + 238, 5 single tiles + 110), capacity-cut
+    "bf16_many_tiles": (LayerShape("bf16_many_tiles", d=256, E=8, k=4, f=256, n_shared=1,
+                                   capacity_factor=1.1, seed=24), 1500),
+}
+
+
+@pytest.mark.parametrize("name", list(PREFILL_TILES))
+def test_prefill_pair_and_single_tiles_give_the_same_bits(name):
+    """moe_config.prefill_tiles picks 256-token tiles on CTA pairs (0) or 128-token
+    tiles on single CTAs (1) for bf16 prefill batches.  Each output element is one
+    FP32 dot product accumulated in the same k order either way, so the layer
+    outputs agree bit for bit; the pair result is checked against the oracle."""
+    sh, T = PREFILL_TILES[name]
+    data = inputs_on_device(sh, T)
+    li, x, dli, dx = data
+    layer = M.MoELayer(dli, T, out_dtype="f32")
+    assert layer.cfg.prefill_tiles == 0
+    pair = layer.forward(dx).clone()
+    assert M.moe_get_device_status(layer.ws) == 0
+    layer.cfg.prefill_tiles = 1
+    single = layer.forward(dx).clone()
+    assert M.moe_get_device_status(layer.ws) == 0
+    assert torch.equal(pair, single)
+    res = run_layer(sh, T, tokens=sample_rows(T), data=data)
+    assert res.max_margin_mismatch < ROUTE_MARGIN
+    assert res.err_ratio <= TOL[sh.expert], res.err_ratio
+
+
 def test_precision_of_bf16_rows_against_fp32_rows():
     """The layer forward keeps the gated routed rows in bf16 between the down GEMM
     and the combine; the grouped-FFN + combine entry points keep them in FP32.
