@@ -117,10 +117,13 @@ typedef struct moe_config {
                               half a second).  A wait that runs out sets device error 2
                               and the kernel returns early (moe_get_device_status)      */
   int32_t routing;         /* moe_routing (0 = top-k)                                    */
-  int32_t prefill_tiles;   /* bf16/f32 experts, expert groups of more than 64 rows: 0 = tiles
-                              of 256 tokens on a pair of CTAs (one cta_group::2 MMA per
-                              k-step; the default), 1 = tiles of 128 tokens on single CTAs.
-                              Both give the same bits; other values are rejected        */
+  int32_t prefill_tiles;   /* bf16 experts at prefill (more than 64 rows per expert on
+                              average): 1 = tiles of 128 tokens on single CTAs, 2 = tiles
+                              of 256 tokens on pairs of CTAs (one cta_group::2 MMA per
+                              k-step), 0 = automatic: pairs when the batch averages at
+                              least 512 rows per routed expert (a pair tile half empty
+                              costs twice a single one), else single CTAs.  All give the
+                              same bits; other values are rejected                      */
 } moe_config;
 
 /* Layer weights (device pointers, caller-owned).

@@ -11,7 +11,8 @@
 //   3. routing, one token per CTA, then -- without a barrier -- the counting-sort
 //      permutation, built by every CTA (it is small);
 //   4. the grouped gate/up GEMM over the routed rows (tcgen05, 16 or 32 token
-//      tiles, rows gathered by the GEMM's own TMA);
+//      tiles, rows gathered by the GEMM's own TMA; split along K when the tiles
+//      fill at most half the SMs);
 //   5. the grouped down GEMM (gated bf16 rows of every assignment);
 //   6. the combine, element groups spread over all CTAs.
 // The TMEM is allocated once for both GEMMs.  Every barrier wait is bounded: a
@@ -53,6 +54,7 @@ struct DecodeParams {
   double eps;
   int T, d, E, k, S, mode, renorm, cap;
   int ns, rows;                   // router: ns K-slices of `rows` rows
+  int n_split_cnt;                // split-K tile counters (gu.split_cnt == dn.split_cnt)
 };
 
 constexpr int kDecodeThreads = kTcBaseThreads;
@@ -195,7 +197,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     tmem_relinquish();
   }
   bool ok = true;
-  // 1. RMSNorm
+  // 1. RMSNorm (and the split-K tile counters zeroed, in case a call was cut short)
+  if (p.gu.split_cnt)
+    for (int i = blockIdx.x * kDecodeThreads + threadIdx.x; i < p.n_split_cnt;
+         i += nb * kDecodeThreads)
+      p.gu.split_cnt[i] = 0;
   for (int t = blockIdx.x; t < p.T; t += nb)
     rmsnorm_row_bf16v<256, MAXV>(p.x + (size_t)t * p.d, p.gamma, p.xn + (size_t)t * p.d, p.d,
                                  p.eps, red);   // the chain's partition: identical bits
@@ -255,7 +261,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       gu_tiles += (rows + BN - 1) / BN;
     }
     gu_tiles = warp_sum(gu_tiles) * nt + p.S * ((p.T + BN - 1) / BN) * nt;
-    const int idle = nb - gu_tiles, me = (int)blockIdx.x - gu_tiles;
+    const int items = gu_tiles * split_parts(p.gu, gu_tiles, nb);   // the GEMM's work items
+    const int idle = nb - items, me = (int)blockIdx.x - items;
     if (me >= 0) {
       constexpr uint32_t kChunk = 32 * 1024;
       const size_t per = (size_t)p.dn.prob[0].K * p.d * 2;   // one expert's W_down bytes

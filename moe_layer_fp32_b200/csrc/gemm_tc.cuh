@@ -268,6 +268,19 @@ MOE_DEV void decode_work(const TcParams& p, const int* prefix, int BN, int TN, i
   ti.kb0 = ti.ks * kbl / S;
   ti.kb1 = (ti.ks + 1) * kbl / S;
 }
+// K-parts of each output tile of a split-K launch (1 when the params hold no
+// partial-sum buffer): as many as fit the grid, at most kMaxSplit, and at least
+// two k-blocks per part.
+MOE_DEV int split_parts(const TcParams& p, int out_tiles, int ncta) {
+  if (p.split_part == nullptr || out_tiles <= 0) return 1;
+  int kbmin = p.prob[0].K / 64;
+  if (p.n_prob > 1 && p.prob[1].K / 64 < kbmin) kbmin = p.prob[1].K / 64;
+  int S = ncta / out_tiles;
+  if (S > kMaxSplit) S = kMaxSplit;
+  if (S > kbmin / 2) S = kbmin / 2;
+  return S < 1 ? 1 : S;
+}
+
 MOE_DEV int total_tiles(const TcParams& p, const int* prefix, int TN) {
   int tot = 0;
   for (int pi = 0; pi < p.n_prob; ++pi) {
@@ -581,14 +594,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   constexpr bool kCanSplit = !DIRECT && EPI != EPI_ROUTER && BN <= 64;
   int S = 1;
   if (EPI == EPI_ROUTER && p.k_splits > 1) S = p.k_splits;
-  if (kCanSplit && p.split_part != nullptr && out_tiles > 0) {
-    int kbmin = p.prob[0].K / 64;
-    if (p.n_prob > 1 && p.prob[1].K / 64 < kbmin) kbmin = p.prob[1].K / 64;
-    S = ncta / out_tiles;
-    if (S > kMaxSplit) S = kMaxSplit;
-    if (S > kbmin / 2) S = kbmin / 2;
-    if (S < 1) S = 1;
-  }
+  if (kCanSplit) S = split_parts(p, out_tiles, ncta);
   const int total = out_tiles * S;
 
   if (warp == 0) {

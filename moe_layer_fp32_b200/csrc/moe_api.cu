@@ -121,6 +121,16 @@ inline int split_counters() { return num_sms() * 8; }
 inline bool interleave_tiles(const moe_config* c) {
   return c->expert_dtype == MOE_BF16 && pick_bn(c) == 128;
 }
+// Pair tiles of 256 tokens halve each SM's operand traffic per MMA, but an
+// expert's last tile is on average half empty, and a half-empty pair tile costs
+// what two single tiles do.  Measured on B200 (same bits either way): pairs are
+// 2-12% faster from 512 rows per expert up (OLMoE-shaped T=4096, 16384,
+// V2-Lite-shaped T=8192) and 7% slower at 295 (DeepSeek-V3-shaped T=9440).
+constexpr double kPairMinRowsPerExpert = 512.0;
+inline bool pair_tiles(const moe_config* c) {
+  if (c->prefill_tiles != 0) return c->prefill_tiles == 2;
+  return (double)n_slots(c) / c->E >= kPairMinRowsPerExpert;
+}
 // Inside the layer forward the gated routed rows of tensor-core experts are kept
 // in bf16 (half the bytes the down GEMM writes and the combine reads); the
 // grouped-FFN and combine entry points exchange them in FP32.
@@ -149,7 +159,7 @@ moe_status validate(const moe_config* c) {
   if (c->wait_kcycles < 0) return MOE_ERR_INVALID;
   if (c->routing != MOE_ROUTE_TOPK && c->routing != MOE_ROUTE_EXPERT_CHOICE)
     return MOE_ERR_INVALID;
-  if (c->prefill_tiles != 0 && c->prefill_tiles != 1) return MOE_ERR_INVALID;
+  if (c->prefill_tiles < 0 || c->prefill_tiles > 2) return MOE_ERR_INVALID;
   if (c->routing == MOE_ROUTE_EXPERT_CHOICE) {
     // the expert picks rank tokens by their gate probability: a selection-only bias
     // has no meaning there; the FP32 (CUDA-core) experts take the top-k path only
@@ -407,7 +417,8 @@ moe_status launch_pair(const TcParams& p, cudaStream_t st) {
 }
 
 // Prefill tiles of bf16 experts run on CTA pairs (256 tokens per tile, one
-// cta_group::2 MMA per k-step) unless moe_config.prefill_tiles asks for single CTAs.
+// cta_group::2 MMA per k-step) or on single CTAs (128 tokens), as
+// moe_config.prefill_tiles and pair_tiles() decide.
 template <int EPI, int WQ>
 moe_status launch_tc_bn_q(int bn, bool pair, const TcParams& p, cudaStream_t st) {
   switch (bn) {
@@ -836,7 +847,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     if ((s = gateup_params(c, w, wl, wq, xn, xp, offsets, rr, h, split_part, split_cnt, err, p)) !=
         MOE_OK)
       return s;
-    s = launch_tc_bn<EPI_GATEUP>(bn, wq, c->prefill_tiles == 0, p, st);
+    s = launch_tc_bn<EPI_GATEUP>(bn, wq, pair_tiles(c), p, st);
     if (s != MOE_OK) return s;
     mk->mark(st);
   }
@@ -845,7 +856,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     if ((s = down_params(c, w, wl, wq, offsets, rr, gate, h, y, rows_bf16, ys, split_part,
                          split_cnt, err, p)) != MOE_OK)
       return s;
-    s = launch_tc_bn<EPI_DOWN>(bn, wq, c->prefill_tiles == 0, p, st);
+    s = launch_tc_bn<EPI_DOWN>(bn, wq, pair_tiles(c), p, st);
     mk->mark(st);
   }
   return s;
@@ -998,13 +1009,16 @@ moe_status run_decode_layer(const moe_config* c, const moe_weights* w, const voi
   void* y = at<void>(ws, L.y);
   float* ys = c->n_shared ? at<float>(ws, L.ys) : nullptr;
   const RoutedRows rr{perm, c->k, perm};
+  float* split_part = split_k(c) ? at<float>(ws, L.split) : nullptr;
+  int32_t* split_cnt = split_k(c) ? at<int32_t>(ws, L.splitcnt) : nullptr;
   moe_status s;
-  if ((s = gateup_params(c, w, *w, WQ_BF16, xn, nullptr, offsets, rr, h, nullptr, nullptr, err,
-                         dp.gu)) != MOE_OK)
+  if ((s = gateup_params(c, w, *w, WQ_BF16, xn, nullptr, offsets, rr, h, split_part, split_cnt,
+                         err, dp.gu)) != MOE_OK)
     return s;
-  if ((s = down_params(c, w, *w, WQ_BF16, offsets, rr, gate, h, y, true, ys, nullptr, nullptr,
-                       err, dp.dn)) != MOE_OK)
+  if ((s = down_params(c, w, *w, WQ_BF16, offsets, rr, gate, h, y, true, ys, split_part,
+                       split_cnt, err, dp.dn)) != MOE_OK)
     return s;
+  dp.n_split_cnt = split_cnt ? split_counters() : 0;
   dp.x = static_cast<const __nv_bfloat16*>(x);
   dp.gamma = static_cast<const float*>(w->rms_gamma);
   dp.w_router = static_cast<const __nv_bfloat16*>(w->w_router);

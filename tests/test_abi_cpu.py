@@ -74,7 +74,7 @@ def test_workspace_size_for_presets(lib, preset):
 def test_invalid_configs_are_rejected_on_the_host(lib):
     sh = moe_synth.PRESETS["olmoe"]
     bad = [dict(k=65), dict(k=0), dict(T=0), dict(E=0), dict(d=100), dict(n_shared=9),
-           dict(prefill_tiles=2), dict(prefill_tiles=-1), dict(wait_kcycles=-1)]
+           dict(prefill_tiles=3), dict(prefill_tiles=-1), dict(wait_kcycles=-1)]
     for b in bad:
         cfg = M.make_config(sh, 16)
         for kk, v in b.items():

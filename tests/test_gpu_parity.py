@@ -468,21 +468,26 @@ PREFILL_TILES = {
 
 @pytest.mark.parametrize("name", list(PREFILL_TILES))
 def test_prefill_pair_and_single_tiles_give_the_same_bits(name):
-    """moe_config.prefill_tiles picks 256-token tiles on CTA pairs (0) or 128-token
-    tiles on single CTAs (1) for bf16 prefill batches.  Each output element is one
-    FP32 dot product accumulated in the same k order either way, so the layer
-    outputs agree bit for bit; the pair result is checked against the oracle."""
+    """moe_config.prefill_tiles picks 256-token tiles on CTA pairs (2) or 128-token
+    tiles on single CTAs (1) for bf16 prefill batches (0: chosen by the rows per
+    expert).  Each output element is one FP32 dot product accumulated in the same
+    k order either way, so the layer outputs agree bit for bit; the result is
+    checked against the oracle."""
     sh, T = PREFILL_TILES[name]
     data = inputs_on_device(sh, T)
     li, x, dli, dx = data
     layer = M.MoELayer(dli, T, out_dtype="f32")
     assert layer.cfg.prefill_tiles == 0
+    auto = layer.forward(dx).clone()
+    assert M.moe_get_device_status(layer.ws) == 0
+    layer.cfg.prefill_tiles = 2
     pair = layer.forward(dx).clone()
     assert M.moe_get_device_status(layer.ws) == 0
     layer.cfg.prefill_tiles = 1
     single = layer.forward(dx).clone()
     assert M.moe_get_device_status(layer.ws) == 0
     assert torch.equal(pair, single)
+    assert torch.equal(auto, single)
     res = run_layer(sh, T, tokens=sample_rows(T), data=data)
     assert res.max_margin_mismatch < ROUTE_MARGIN
     assert res.err_ratio <= TOL[sh.expert], res.err_ratio
