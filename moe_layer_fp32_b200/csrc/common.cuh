@@ -32,6 +32,13 @@ MOE_DEV unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
                : "memory");
   return old;
 }
+MOE_DEV void st_relaxed_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// fire-and-forget add that releases this thread's earlier memory operations
+MOE_DEV void red_release_add_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 MOE_DEV unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -17,9 +17,9 @@
 //   6. the combine, element groups spread over all CTAs.
 // The TMEM is allocated once for both GEMMs.  Every barrier wait is bounded: a
 // CTA that gives up sets device error 2 and skips the remaining steps, so every
-// CTA finishes.  The grid barrier's two words live in the workspace; they are
-// left at zero by a completed call and cleared by moe_clear_device_status after
-// an error.
+// CTA finishes.  The grid barrier's two words live in the workspace: the count is
+// left at zero by a completed call, the generation only advances; both are
+// cleared by moe_clear_device_status after an error.
 #pragma once
 #include "gemm_tc.cuh"
 
@@ -61,41 +61,55 @@ constexpr int kDecodeThreads = kTcBaseThreads;
 constexpr int kDecodeMaxT = 32;
 
 // Bounded grid-wide barrier of a cooperative launch.  Thread 0 of every CTA
-// arrives on bar[0]; the last arrival resets it and advances the generation in
-// bar[1], which the others wait for.  Returns false (and sets device error 2) if
-// the wait ran out, and also when some CTA has recorded a time-out before
-// arriving: the caller then takes no further step and arrives at no further
-// barrier, so no CTA is ever released from a barrier that another has not
-// reached.  All threads of the CTA return the same value.
+// arrives on bar[0] (adding 1, plus kBarErr if this CTA's step ran out of time);
+// the last arrival resets the count and publishes the next generation in bar[1]
+// (with its top bit set if any CTA reported a time-out), which the others wait
+// for.  Thread 0 keeps the generation it expects in `gen`, read once when the
+// kernel starts, so that an arrival costs one atomic and the release one store
+// and one reduction, with no other round trip to L2.  Returns false (and sets
+// device error 2) if the wait ran out, and when some CTA reported a time-out:
+// the caller then takes no further step and arrives at no further barrier, so
+// no CTA is ever released from a barrier that another has not reached.  All
+// threads of the CTA return the same value.
 // Data that one step writes with ordinary stores and a later step reads through
 // the TMA (the normalised rows, h) crosses from the generic to the async proxy:
 // every thread fences its own stores before the barrier and its later copies
 // after it.
-MOE_DEV bool grid_barrier(unsigned* bar, int nblocks, long long limit, int32_t* err, int* s_ok) {
+constexpr unsigned kBarErr = 1u << 16;
+constexpr unsigned kGenErr = 1u << 31;
+MOE_DEV bool grid_barrier(unsigned* bar, int nblocks, unsigned& gen, bool mine_ok,
+                          long long limit, int32_t* err, int* s_ok) {
   fence_proxy_async_global();
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    const unsigned g = ld_acquire_gpu(bar + 1);
-    // the arrival releases this CTA's writes (ordered after the CTA barrier by the
-    // fence); the last one acquires everyone's, resets the count and publishes the
-    // new generation, which every waiter acquires
+    // the fence orders the CTA's writes (made visible to this thread by the CTA
+    // barrier) before the arrival; the last arrival fences again, so that its
+    // release of the new generation carries every CTA's writes to the waiters
     __threadfence();
-    if (atom_add_acq_rel_gpu(bar, 1u) == (unsigned)nblocks - 1) {
-      atomicExch(bar, 0u);
-      atom_add_acq_rel_gpu(bar + 1, 1u);
+    const unsigned add = mine_ok ? 1u : 1u + kBarErr;
+    const unsigned now = atomicAdd(bar, add) + add;
+    const unsigned prev = gen;
+    if ((now & (kBarErr - 1)) == (unsigned)nblocks) {
+      __threadfence();
+      st_relaxed_gpu(bar, 0u);
+      const unsigned inc = (now >= kBarErr) ? 1u + kGenErr : 1u;
+      red_release_add_gpu(bar + 1, inc);
+      gen = prev + inc;
     } else {
       const long long t0 = clock64();
-      while (ld_acquire_gpu(bar + 1) == g) {
-        __nanosleep(32);
+      unsigned g;
+      while ((g = ld_acquire_gpu(bar + 1)) == prev) {
+        __nanosleep(20);
         if (clock64() - t0 > limit) {
           set_error(err, DEV_TIMEOUT);
           ok = 0;
           break;
         }
       }
+      gen = g;
     }
-    if (*reinterpret_cast<volatile int32_t*>(err) == DEV_TIMEOUT) ok = 0;
+    if ((gen - prev) != 1u) ok = 0;   // a CTA reported a time-out
     *s_ok = ok;
   }
   __syncthreads();
@@ -196,6 +210,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     tmem_alloc(&tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
+  unsigned gen = 0;   // thread 0: the grid barrier's current generation
+  if (threadIdx.x == 0) gen = ld_acquire_gpu(p.grid_bar + 1);
   bool ok = true;
   // 1. RMSNorm (and the split-K tile counters zeroed, in case a call was cut short)
   if (p.gu.split_cnt)
@@ -205,7 +221,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   for (int t = blockIdx.x; t < p.T; t += nb)
     rmsnorm_row_bf16v<256, MAXV>(p.x + (size_t)t * p.d, p.gamma, p.xn + (size_t)t * p.d, p.d,
                                  p.eps, red);   // the chain's partition: identical bits
-  ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
+  ok = grid_barrier(p.grid_bar, nb, gen, true, p.wait_cycles, p.err, &s_ok);
   // 2. router partial logits: work item (token group of 8, K-slice)
   if (ok) {
     float* sm_r = reinterpret_cast<float*>(smem);
@@ -213,7 +229,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     for (int w = blockIdx.x; w < groups * p.ns; w += nb)
       router_vec_tile<8, kDecodeThreads>(p.xn, p.w_router, p.part, p.T, p.d, p.E, p.rows,
                                          (w % groups) * 8, w / groups, sm_r);
-    ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
+    ok = grid_barrier(p.grid_bar, nb, gen, true, p.wait_cycles, p.err, &s_ok);
   }
   // 3. routing: CTA t routes token t -- every thread adds one expert's partial
   //    logits in slice order, then warp 0 selects
@@ -238,7 +254,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       __syncthreads();
     }
-    ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
+    ok = grid_barrier(p.grid_bar, nb, gen, true, p.wait_cycles, p.err, &s_ok);
   }
   // the permutation of the T*k <= 1024 assignments: every CTA builds it (one warp),
   // writing the same values to the workspace, and reads back only what it wrote
@@ -280,12 +296,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   }
   if (ok) {
-    tc_gemm_run<EPI_GATEUP, BN, false, WQ_BF16>(p.gu, smem, &tmem_slot, blockIdx.x, nb, false);
-    ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
+    const bool mine = tc_gemm_run<EPI_GATEUP, BN, false, WQ_BF16>(p.gu, smem, &tmem_slot,
+                                                                 blockIdx.x, nb, false);
+    ok = grid_barrier(p.grid_bar, nb, gen, mine, p.wait_cycles, p.err, &s_ok);
   }
   if (ok) {
-    tc_gemm_run<EPI_DOWN, BN, false, WQ_BF16>(p.dn, smem, &tmem_slot, blockIdx.x, nb, false);
-    ok = grid_barrier(p.grid_bar, nb, p.wait_cycles, p.err, &s_ok);
+    const bool mine = tc_gemm_run<EPI_DOWN, BN, false, WQ_BF16>(p.dn, smem, &tmem_slot,
+                                                               blockIdx.x, nb, false);
+    ok = grid_barrier(p.grid_bar, nb, gen, mine, p.wait_cycles, p.err, &s_ok);
   }
   // 6. combine (4 columns per thread; every tensor is 16-byte aligned here)
   if (ok) {

@@ -519,9 +519,10 @@ MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float s
 // is at *tmem_slot once the CTA has synchronised.  with_pdl: wait for the previous
 // kernel of the stream (programmatic dependent launch) before reading global
 // memory.  All threads of the CTA call it; it returns after a __syncthreads, with
-// every MMA it issued complete and every barrier idle.
+// every MMA it issued complete and every barrier idle, true unless one of this
+// CTA's waits ran out (device error 2 is then set).
 template <int EPI, int BN, bool DIRECT, int WQ>
-MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_slot, int cta,
+MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_slot, int cta,
                          int ncta, bool with_pdl) {
   using C = TcConfig<EPI, BN, DIRECT, WQ>;
   constexpr int NA = C::NA;
@@ -946,6 +947,7 @@ MOE_DEV void tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   }
   tc_fence_before();
   __syncthreads();
+  return *abort_flag == 0;
 }
 
 template <int EPI, int BN, bool DIRECT, int WQ>
