@@ -1167,7 +1167,10 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
       return s;
   }
   mk->mark(st);
-  if (fused_combine(cfg)) {
+  // the fused combine reads x and writes out two elements at a time
+  const bool comb_aligned = reinterpret_cast<uintptr_t>(x) % 4 == 0 &&
+                            reinterpret_cast<uintptr_t>(out) % (cfg->out_dtype == MOE_F32 ? 8 : 4) == 0;
+  if (fused_combine(cfg) && comb_aligned) {
     // the combine runs in the down GEMM's epilogue; its step is empty in the profile
     const CombParams cb = comb_params(cfg, ws, L, x, out);
     if ((s = run_ffn(cfg, w, xn, offsets, RoutedRows{perm, cfg->k, perm}, gate, y, ys, ws, st,
