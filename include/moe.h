@@ -324,11 +324,7 @@ moe_status moe_combine(const moe_config* cfg, const float* y_assign, const int32
  * Between the down GEMM and the combine the gated routed rows of tensor-core
  * experts are kept in bf16 (the round-to-nearest-even of the FP32 rows that
  * moe_grouped_ffn returns), so the result equals moe_combine applied to those
- * rounded rows, bit for bit.  With top-k routing, tensor-core experts, x 4-byte
- * and out 4-byte (bf16) or 8-byte (FP32) aligned, the combine runs inside the
- * down GEMM's epilogue: per token and cell of output features, the epilogue warp
- * whose rows complete the token's count adds them in the same fixed order (no
- * separate launch; same bits). */
+ * rounded rows, bit for bit. */
 moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const void* x,
                              void* out, void* ws, size_t ws_bytes, float* logits_out,
                              int32_t* topk_idx_out, int32_t* counts_out, void* stream);

@@ -13,9 +13,8 @@
 //   4. the grouped gate/up GEMM over the routed rows (tcgen05, 16 or 32 token
 //      tiles, rows gathered by the GEMM's own TMA; split along K when the tiles
 //      fill at most half the SMs);
-//   5. the grouped down GEMM (gated bf16 rows of every assignment), whose
-//      epilogue also runs the combine: the arrival that completes a token's rows
-//      for a cell of 32 features adds them in the combine's fixed order.
+//   5. the grouped down GEMM (gated bf16 rows of every assignment);
+//   6. the combine, element groups spread over all CTAs.
 // The TMEM is allocated once for both GEMMs.  Every barrier wait is bounded: a
 // CTA that gives up sets device error 2 and skips the remaining steps, so every
 // CTA finishes.  The grid barrier's two words live in the workspace: the count is
@@ -45,14 +44,17 @@ struct DecodeParams {
   float* logits_out;              // [T, E] or nullptr
   const uint8_t* w_down;          // [E, f, d] bf16 routed experts' down weights
   const uint8_t* sh_down;         // [S, f, d] or nullptr
+  const __nv_bfloat16* y;         // [T * k, d] gated routed rows (written by the down GEMM)
+  const float* ys;                // [S, T, d]
+  void* out;                      // [T, d] bf16 or fp32
+  int out_f32;
   int32_t* err;
   unsigned* grid_bar;             // [2]: arrivals, generation
   long long wait_cycles;
   double eps;
   int T, d, E, k, S, mode, renorm, cap;
   int ns, rows;                   // router: ns K-slices of `rows` rows
-  int32_t* zero;                  // the GEMMs' split-K and combine counters, zeroed in step 1
-  int nzero;
+  int n_split_cnt;                // split-K tile counters (gu.split_cnt == dn.split_cnt)
 };
 
 constexpr int kDecodeThreads = kTcBaseThreads;
@@ -211,9 +213,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   unsigned gen = 0;   // thread 0: the grid barrier's current generation
   if (threadIdx.x == 0) gen = ld_acquire_gpu(p.grid_bar + 1);
   bool ok = true;
-  // 1. RMSNorm (and the GEMMs' split-K and combine counters zeroed)
-  for (int i = blockIdx.x * kDecodeThreads + threadIdx.x; i < p.nzero; i += nb * kDecodeThreads)
-    p.zero[i] = 0;
+  // 1. RMSNorm (and the split-K tile counters zeroed, in case a call was cut short)
+  if (p.gu.split_cnt)
+    for (int i = blockIdx.x * kDecodeThreads + threadIdx.x; i < p.n_split_cnt;
+         i += nb * kDecodeThreads)
+      p.gu.split_cnt[i] = 0;
   for (int t = blockIdx.x; t < p.T; t += nb)
     rmsnorm_row_bf16v<256, MAXV>(p.x + (size_t)t * p.d, p.gamma, p.xn + (size_t)t * p.d, p.d,
                                  p.eps, red);   // the chain's partition: identical bits
@@ -296,10 +300,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                                                  blockIdx.x, nb, false);
     ok = grid_barrier(p.grid_bar, nb, gen, mine, p.wait_cycles, p.err, &s_ok);
   }
-  // 5. + 6. the down GEMM, whose epilogue also runs the combine (each output cell
-  // summed by the arrival that completes its token's rows)
-  if (ok)
-    tc_gemm_run<EPI_DOWN, BN, false, WQ_BF16>(p.dn, smem, &tmem_slot, blockIdx.x, nb, false);
+  if (ok) {
+    const bool mine = tc_gemm_run<EPI_DOWN, BN, false, WQ_BF16>(p.dn, smem, &tmem_slot,
+                                                               blockIdx.x, nb, false);
+    ok = grid_barrier(p.grid_bar, nb, gen, mine, p.wait_cycles, p.err, &s_ok);
+  }
+  // 6. combine (4 columns per thread; every tensor is 16-byte aligned here)
+  if (ok) {
+    const size_t n = (size_t)p.T * (p.d / 4);
+    for (size_t i = (size_t)blockIdx.x * kDecodeThreads + threadIdx.x; i < n;
+         i += (size_t)nb * kDecodeThreads) {
+      if (p.out_f32)
+        combine_elems<__nv_bfloat16, float, __nv_bfloat16, 4>(
+            p.y, p.slot, p.ys, p.S, p.x, static_cast<float*>(p.out), p.T, p.d, p.k, i);
+      else
+        combine_elems<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16, 4>(
+            p.y, p.slot, p.ys, p.S, p.x, static_cast<__nv_bfloat16*>(p.out), p.T, p.d, p.k, i);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -244,8 +244,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
     const int half = (warp - 2) >> 2;       // which half of the columns it drains
     float* stg = stg_all + (warp - 2) * (32 * 16);
     const uint32_t tempty_even = mapa_shared(tempty_bar, 0);
-    if (EPI == EPI_DOWN && p.comb.cnt)
-      comb_empty_tokens(p.comb, blockIdx.x * kEpiWarps + (warp - 2), gridDim.x * kEpiWarps, lane);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < total; tile += npairs) {
@@ -256,19 +254,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       int r;
       float sc;
       direct_row<EPI>(P, ti, 128 * (int)rank + q * 32 + lane, r, sc);
-      int ct = -1;           // fused combine: the row's token and its kept rows
-      uint32_t ckept = 0;
-      if (EPI == EPI_DOWN && p.comb.cnt && r >= 0) {
-        ct = comb_token(P, p.comb, r);
-        ckept = comb_kept(p.comb, ct);
-      }
       if (!pair_wait(&tfull_bar[acc], acc_phase, p, abort_flag, peer_abort, true)) break;
       tc_fence_after();
       direct_store<EPI, TN>(P, ti, r, sc, t_base, half, lane, stg);
-      if (EPI == EPI_DOWN && p.comb.cnt) {
-        const int n0 = ti.n0 + half * (TN / 2);   // this warp's cell
-        if (n0 < P.n_valid) comb_cell(p.comb, ct, ckept, n0, TN / 2, lane);
-      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(tempty_even + acc * 8);

@@ -80,26 +80,6 @@ struct TcProblem {
   CUtensorMap tmS2;
 };
 
-// The combine of the layer forward, fused into the DOWN epilogue (top-k routing,
-// bf16 routed rows; cnt == nullptr: off).  After an epilogue warp has stored its
-// rows of a cell of features (the features it drains of one output tile), each
-// row is counted on cnt[t * (d / 32) + n / 32] (t: the row's token, n: the cell's
-// first feature).  The arrival that completes a token's rows for the cell -- its
-// kept routed rows and its shared experts' rows -- adds them in the combine's
-// fixed order (residual, shared experts s = 0..S-1, routed rows j = 0..k-1) and
-// writes that cell of out[t]: the same sums, bit for bit, as the separate combine,
-// with no floating-point atomics and no waiting.
-struct CombParams {
-  int32_t* cnt;               // [T][d/32] arrival counters, zero when the GEMM starts
-  const int32_t* slot;        // slot_of [T*k]: assignment t*k+j has a row iff >= 0
-  const __nv_bfloat16* y;     // gated routed rows [T*k][d] bf16 (by assignment)
-  const float* ys;            // shared experts' rows [S][T][d] FP32, or nullptr
-  const __nv_bfloat16* res;   // residual x [T][d]
-  void* out;                  // [T][d] bf16, or FP32 with out_f32
-  int out_f32;
-  int T, k, S, d;
-};
-
 struct TcParams {
   TcProblem prob[2];
   int n_prob;
@@ -122,7 +102,6 @@ struct TcParams {
   // bound by streaming a light expert's weights run beside tiles bound by the
   // tensor cores instead of all at once
   int interleave;
-  CombParams comb;            // DOWN: the fused combine (comb.cnt == nullptr: off)
 };
 
 constexpr int kMaxSplit = 4;
@@ -533,97 +512,6 @@ MOE_DEV void direct_store(const TcProblem& P, const TileInfo& ti, int r, float s
   }
 }
 
-// ---------------------------------------------------------------- fused combine
-// Token of output row r: routed rows are stored by assignment (t*k + j), the
-// shared experts' rows at s*T + t.
-MOE_DEV int comb_token(const TcProblem& P, const CombParams& cb, int r) {
-  return P.perm_assign ? r / cb.k : r % cb.T;
-}
-// Bit j set: assignment t*k + j of token t has a row.
-MOE_DEV uint32_t comb_kept(const CombParams& cb, int t) {
-  uint32_t m = 0;
-  const int32_t* sl = cb.slot + (size_t)t * cb.k;
-  for (int j = 0; j < cb.k; ++j) m |= (sl[j] >= 0 ? 1u : 0u) << j;
-  return m;
-}
-MOE_DEV float2 ldcg_bf16x2(const __nv_bfloat16* p) {
-  const unsigned u = __ldcg(reinterpret_cast<const unsigned*>(p));
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
-}
-// Two features e, e+1 of token t, summed in the combine's order.
-MOE_DEV void comb_pair(const CombParams& cb, int t, uint32_t kept, int e) {
-  const float2 r = __bfloat1622float2(
-      *reinterpret_cast<const __nv_bfloat162*>(cb.res + (size_t)t * cb.d + e));
-  float a0 = r.x, a1 = r.y;
-  for (int s = 0; s < cb.S; ++s) {
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(cb.ys + ((size_t)s * cb.T + t) * cb.d + e));
-    a0 += v.x;
-    a1 += v.y;
-  }
-  for (int j = 0; j < cb.k; ++j) {
-    if (!((kept >> j) & 1u)) continue;
-    const float2 v = ldcg_bf16x2(cb.y + ((size_t)t * cb.k + j) * cb.d + e);
-    a0 += v.x;
-    a1 += v.y;
-  }
-  if (cb.out_f32)
-    *reinterpret_cast<float2*>(static_cast<float*>(cb.out) + (size_t)t * cb.d + e) = make_float2(a0, a1);
-  else
-    *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(cb.out) + (size_t)t * cb.d + e) =
-        __floats2bfloat162_rn(a0, a1);
-}
-// One feature e of token t.
-MOE_DEV void comb_one(const CombParams& cb, int t, uint32_t kept, int e) {
-  float a = __bfloat162float(cb.res[(size_t)t * cb.d + e]);
-  for (int s = 0; s < cb.S; ++s) a += __ldcg(cb.ys + ((size_t)s * cb.T + t) * cb.d + e);
-  for (int j = 0; j < cb.k; ++j) {
-    if (!((kept >> j) & 1u)) continue;
-    const unsigned short u =
-        __ldcg(reinterpret_cast<const unsigned short*>(cb.y + ((size_t)t * cb.k + j) * cb.d + e));
-    a += __bfloat162float(__ushort_as_bfloat16(u));
-  }
-  if (cb.out_f32)
-    static_cast<float*>(cb.out)[(size_t)t * cb.d + e] = a;
-  else
-    static_cast<__nv_bfloat16*>(cb.out)[(size_t)t * cb.d + e] = __float2bfloat16_rn(a);
-}
-// Whole warp, after its stores of the cell [n0, n0 + w) (w = 32 or a multiple of
-// 64): lane's row belongs to token t (-1: none) whose kept mask is `kept`.  Counts
-// each row; every token whose rows this warp completes is combined over the cell.
-MOE_DEV void comb_cell(const CombParams& cb, int t, uint32_t kept, int n0, int w, int lane) {
-  __syncwarp();
-  __threadfence();   // the warp's stores of the cell, before its counts
-  bool last = false;
-  if (t >= 0) {
-    const int need = __popc(kept) + cb.S;
-    last = atomicAdd(cb.cnt + (size_t)t * (cb.d >> 5) + (n0 >> 5), 1) == need - 1;
-  }
-  uint32_t m = __ballot_sync(0xffffffffu, last);
-  if (!m) return;
-  __threadfence();   // every other row of those tokens, before reading them
-  while (m) {
-    const int src = __ffs(m) - 1;
-    m &= m - 1;
-    const int tt = __shfl_sync(0xffffffffu, t, src);
-    const uint32_t kk = __shfl_sync(0xffffffffu, kept, src);
-    if (w == 32)
-      comb_one(cb, tt, kk, n0 + lane);
-    else
-      for (int e = n0 + 2 * lane; e < n0 + w; e += 64) comb_pair(cb, tt, kk, e);
-  }
-}
-// Tokens with no row at all (no shared experts, every assignment dropped): out is
-// the residual.  Warp `wid` of `nw` takes tokens wid, wid + nw, ...
-MOE_DEV void comb_empty_tokens(const CombParams& cb, int wid, int nw, int lane) {
-  if (cb.S != 0) return;
-  for (int t = wid; t < cb.T; t += nw) {
-    bool any = false;
-    for (int j = lane; j < cb.k; j += 32) any = any || cb.slot[(size_t)t * cb.k + j] >= 0;
-    if (__any_sync(0xffffffffu, any)) continue;
-    for (int e = 2 * lane; e < cb.d; e += 64) comb_pair(cb, t, 0u, e);
-  }
-}
-
 // The grouped GEMM of one CTA over the work items cta, cta + ncta, ...: barrier
 // set-up in its shared memory (`smem`, 1024-byte aligned, C::SMEM_BYTES - 1024
 // bytes), the warp roles, and after an abort the drain of this CTA's copies still
@@ -913,8 +801,6 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
     const int half = (warp - 2) >> 2;       // which half of the columns it drains
     int* s_row = epi_row + (warp - 2) * 128;
     float* s_scale = epi_scale + (warp - 2) * 128;
-    if (EPI == EPI_DOWN && p.comb.cnt)
-      comb_empty_tokens(p.comb, cta * kEpiWarps + (warp - 2), ncta * kEpiWarps, lane);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cta; tile < total; tile += ncta) {
@@ -928,20 +814,10 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         int r;
         float sc;
         direct_row<EPI>(P, ti, q * 32 + lane, r, sc);
-        int ct = -1;           // fused combine: the row's token and its kept rows
-        uint32_t ckept = 0;
-        if (EPI == EPI_DOWN && p.comb.cnt && r >= 0) {
-          ct = comb_token(P, p.comb, r);
-          ckept = comb_kept(p.comb, ct);
-        }
         if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles, true)) break;
         tc_fence_after();
         direct_store<EPI, TN>(P, ti, r, sc, t_base, half, lane,
                               reinterpret_cast<float*>(epi_row) + (warp - 2) * (32 * 16));
-        if (EPI == EPI_DOWN && p.comb.cnt) {
-          const int n0 = ti.n0 + half * (TN / 2);   // this warp's cell
-          if (n0 < P.n_valid) comb_cell(p.comb, ct, ckept, n0, TN / 2, lane);
-        }
       } else {
         // swapped: this thread owns feature n; the tile's token rows and scales are
         // staged in this warp's shared-memory slice (warp-private: __syncwarp only)
@@ -1046,17 +922,6 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
               const int r = s_row[c * 16 + j];
               if (r >= 0 && n_ok) Y[(size_t)r * P.ld_out + n] = v0[j] * s_scale[c * 16 + j];
             }
-          }
-        }
-        if (EPI == EPI_DOWN && p.comb.cnt && finish && ti.n0 + q * 32 < P.n_valid) {
-          // fused combine: lane i counts the warp's i-th token column (columns
-          // c*16 + j of c = half, half + 2, ...), cell = this warp's 32 features
-          for (int i0 = 0; i0 < BN / 2; i0 += 32) {
-            const int i = i0 + lane;
-            const int m = (half + 2 * (i >> 4)) * 16 + (i & 15);
-            const int r = (m < BN && m < ti.rows) ? s_row[m] : -1;
-            const int t = r >= 0 ? comb_token(P, p.comb, r) : -1;
-            comb_cell(p.comb, t, t >= 0 ? comb_kept(p.comb, t) : 0u, ti.n0 + q * 32, 32, lane);
           }
         }
       }

@@ -87,9 +87,8 @@ MOE_DEV int find_group(const int* prefix, int G, int mt) {
 MOE_DEV void store_act(__nv_bfloat16* p, double v) { *p = bf16_from_double(v); }
 MOE_DEV void store_act(float* p, double v) { *p = (float)v; }
 
-// Both RMSNorm kernels also zero `nzero` ints at `zero` (spread over the CTAs):
-// the split-K and fused-combine counters of the expert GEMMs that follow later in
-// the same layer.
+// Both RMSNorm kernels also zero `nzero` ints at `zero` (CTA 0): the split-K
+// counters of the expert GEMMs that follow later in the same layer.
 template <typename TA>
 __global__ void __launch_bounds__(256) k_rmsnorm(const TA* __restrict__ x,
                                                  const float* __restrict__ gamma,
@@ -97,7 +96,8 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const TA* __restrict__ x,
                                                  int32_t* __restrict__ zero, int nzero) {
   pdl_wait();
   pdl_trigger();
-  for (int i = blockIdx.x * 256 + threadIdx.x; i < nzero; i += gridDim.x * 256) zero[i] = 0;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
   __shared__ double red[8];
   const size_t row = (size_t)blockIdx.x * d;
   double s = 0.0;
@@ -188,7 +188,8 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bf16v(const __nv_bfloat16* __re
                                                        int nzero) {
   pdl_wait();
   pdl_trigger();
-  for (int i = blockIdx.x * 256 + threadIdx.x; i < nzero; i += gridDim.x * 256) zero[i] = 0;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
   __shared__ double red[8];
   rmsnorm_row_bf16v<256, MAXV>(x + (size_t)blockIdx.x * d, gamma, xn + (size_t)blockIdx.x * d, d,
                                eps, red);

@@ -135,19 +135,11 @@ inline bool pair_tiles(const moe_config* c) {
 // in bf16 (half the bytes the down GEMM writes and the combine reads); the
 // grouped-FFN and combine entry points exchange them in FP32.
 inline bool y_bf16(const moe_config* c) { return tc_experts(c); }
-// The layer forward's combine runs inside the down GEMM's epilogue (top-k routing,
-// tensor-core experts): each output cell is summed by the arrival that completes
-// its token's rows, in the combine's fixed order, so the separate combine launch
-// and its pass over the routed rows go away.
-constexpr bool kFuseCombine = true;
-inline bool fused_combine(const moe_config* c) {
-  return kFuseCombine && tc_experts(c) && c->routing == MOE_ROUTE_TOPK && y_bf16(c);
-}
 
 
 struct Layout {
   size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, split,
-      splitcnt, combcnt, combcnt_end, h, y, ys, sct,
+      splitcnt, h, y, ys, sct,
       total;
   int ns;
 };
@@ -222,10 +214,6 @@ Layout layout(const moe_config* c) {
   L.xp = o;       o = align_up(o + (tc_experts(c) && !gather_in_gemm(c) ? R * d * act : 0));
   L.split = o;    o = align_up(o + (split_k(c) ? (size_t)num_sms() * 2 * pick_bn(c) * 128 * 4 : 0));
   L.splitcnt = o; o = align_up(o + (split_k(c) ? (size_t)split_counters() * 4 : 0));
-  // right after the split-K counters, so that one range zeroes both
-  L.combcnt = o;  o = o + (fused_combine(c) ? T * (d / 32) * 4 : 0);
-  L.combcnt_end = o;
-  o = align_up(o);
   L.h = o;        o = align_up(o + (R + S * T) * f * hb);
   L.y = o;        o = align_up(o + R * d * (y_bf16(c) ? 2 : 4));
   L.ys = o;       o = align_up(o + S * T * d * 4);
@@ -718,28 +706,10 @@ moe_status gateup_params(const moe_config* c, const moe_weights* w, const moe_we
 
 // Parameters of the grouped down GEMM: routed rows of h to rows rr.dst of y scaled
 // by their gate, and the shared experts' rows of h to ys.
-// The fused combine's parameters for a layer forward over workspace `ws`.
-CombParams comb_params(const moe_config* c, void* ws, const Layout& L, const void* x, void* out) {
-  CombParams cb{};
-  cb.cnt = at<int32_t>(ws, L.combcnt);
-  cb.slot = at<int32_t>(ws, L.slot);
-  cb.y = at<__nv_bfloat16>(ws, L.y);
-  cb.ys = c->n_shared ? at<float>(ws, L.ys) : nullptr;
-  cb.res = static_cast<const __nv_bfloat16*>(x);
-  cb.out = out;
-  cb.out_f32 = c->out_dtype == MOE_F32 ? 1 : 0;
-  cb.T = c->T;
-  cb.k = c->k;
-  cb.S = c->n_shared;
-  cb.d = c->d;
-  return cb;
-}
-
 moe_status down_params(const moe_config* c, const moe_weights* w, const moe_weights& wl, int wq,
                        const int32_t* offsets, RoutedRows rr, const float* gate,
                        const __nv_bfloat16* h, void* y, bool rows_bf16, float* ys,
-                       float* split_part, int32_t* split_cnt, int32_t* err, TcParams& p,
-                       const CombParams* comb = nullptr) {
+                       float* split_part, int32_t* split_cnt, int32_t* err, TcParams& p) {
   const int T = c->T, S = c->n_shared, bn = pick_bn(c), R = (int)n_slots(c);
   const int32_t* perm = rr.dst;
   p = TcParams{};
@@ -792,15 +762,13 @@ moe_status down_params(const moe_config* c, const moe_weights* w, const moe_weig
   p.split_part = split_part;
   p.split_cnt = split_cnt;
   p.interleave = interleave_tiles(c);
-  if (comb) p.comb = *comb;
   return MOE_OK;
 }
 
 moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
                    const int32_t* offsets, RoutedRows rr, const float* gate, void* y,
                    float* ys, void* ws, cudaStream_t st, Marks* mk = nullptr,
-                   bool counters_zeroed = false, bool rows_bf16 = false,
-                   const CombParams* comb = nullptr) {
+                   bool counters_zeroed = false, bool rows_bf16 = false) {
   Marks none;
   if (!mk) mk = &none;
   const Layout L = layout(c);
@@ -886,7 +854,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   {
     TcParams p;
     if ((s = down_params(c, w, wl, wq, offsets, rr, gate, h, y, rows_bf16, ys, split_part,
-                         split_cnt, err, p, comb)) != MOE_OK)
+                         split_cnt, err, p)) != MOE_OK)
       return s;
     s = launch_tc_bn<EPI_DOWN>(bn, wq, pair_tiles(c), p, st);
     mk->mark(st);
@@ -994,7 +962,7 @@ constexpr size_t kGridBarOff = 64;
 // The whole layer in one cooperative launch: decode batches (T <= 32) of bf16
 // experts with a bf16 router of at most 256 experts, 16-byte aligned tensors.
 bool single_launch(const moe_config* c) {
-  return fused_combine(c) && c->T <= kDecodeMaxT && c->expert_dtype == MOE_BF16 &&
+  return !expert_choice(c) && c->T <= kDecodeMaxT && c->expert_dtype == MOE_BF16 &&
          vec_router(c) && c->E <= 256 && gather_in_gemm(c) && c->d <= 256 * 4 * 8;
 }
 
@@ -1047,12 +1015,10 @@ moe_status run_decode_layer(const moe_config* c, const moe_weights* w, const voi
   if ((s = gateup_params(c, w, *w, WQ_BF16, xn, nullptr, offsets, rr, h, split_part, split_cnt,
                          err, dp.gu)) != MOE_OK)
     return s;
-  const CombParams cb = comb_params(c, ws, L, x, out);
   if ((s = down_params(c, w, *w, WQ_BF16, offsets, rr, gate, h, y, true, ys, split_part,
-                       split_cnt, err, dp.dn, &cb)) != MOE_OK)
+                       split_cnt, err, dp.dn)) != MOE_OK)
     return s;
-  dp.zero = at<int32_t>(ws, L.splitcnt);
-  dp.nzero = (int)((L.combcnt_end - L.splitcnt) / 4);
+  dp.n_split_cnt = split_cnt ? split_counters() : 0;
   dp.x = static_cast<const __nv_bfloat16*>(x);
   dp.gamma = static_cast<const float*>(w->rms_gamma);
   dp.w_router = static_cast<const __nv_bfloat16*>(w->w_router);
@@ -1069,6 +1035,10 @@ moe_status run_decode_layer(const moe_config* c, const moe_weights* w, const voi
   dp.logits_out = logits_out;
   dp.w_down = static_cast<const uint8_t*>(w->w_down);
   dp.sh_down = static_cast<const uint8_t*>(w->sh_down);
+  dp.y = static_cast<const __nv_bfloat16*>(y);
+  dp.ys = ys;
+  dp.out = out;
+  dp.out_f32 = c->out_dtype == MOE_F32 ? 1 : 0;
   dp.err = err;
   dp.grid_bar = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kGridBarOff);
   dp.wait_cycles = wait_cycles(c);
@@ -1123,10 +1093,9 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
     if (aligned) return run_decode_layer(cfg, w, x, out, ws, logits_out, idx, counts, st);
   }
   mk->mark(st);
-  // the split-K and fused-combine counters of the expert GEMMs, zeroed by the RMSNorm
-  const int nzero = (int)((L.combcnt_end - L.splitcnt) / 4);
-  if ((s = run_rmsnorm(cfg, w, x, xn, st, nzero ? at<int32_t>(ws, L.splitcnt) : nullptr,
-                       nzero)) != MOE_OK)
+  int32_t* split_cnt = split_k(cfg) ? at<int32_t>(ws, L.splitcnt) : nullptr;
+  if ((s = run_rmsnorm(cfg, w, x, xn, st, split_cnt, split_cnt ? split_counters() : 0)) !=
+      MOE_OK)
     return s;
   mk->mark(st);
   if ((s = run_router(cfg, w, xn, part, L.ns, err, st)) != MOE_OK) return s;
@@ -1167,18 +1136,6 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
       return s;
   }
   mk->mark(st);
-  // the fused combine reads x and writes out two elements at a time
-  const bool comb_aligned = reinterpret_cast<uintptr_t>(x) % 4 == 0 &&
-                            reinterpret_cast<uintptr_t>(out) % (cfg->out_dtype == MOE_F32 ? 8 : 4) == 0;
-  if (fused_combine(cfg) && comb_aligned) {
-    // the combine runs in the down GEMM's epilogue; its step is empty in the profile
-    const CombParams cb = comb_params(cfg, ws, L, x, out);
-    if ((s = run_ffn(cfg, w, xn, offsets, RoutedRows{perm, cfg->k, perm}, gate, y, ys, ws, st,
-                     mk, true, true, &cb)) != MOE_OK)
-      return s;
-    mk->mark(st);
-    return MOE_OK;
-  }
   if ((s = run_ffn(cfg, w, xn, offsets, RoutedRows{perm, cfg->k, perm}, gate, y, ys, ws, st, mk,
                    true, y_bf16(cfg))) != MOE_OK)
     return s;
@@ -1393,23 +1350,21 @@ const char* moe_status_string(moe_status s) {
 int32_t moe_layer_step_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
   // expert choice: rmsnorm, router, scores, picks, [gather], gate/up, down, combine
-  // rmsnorm, router, route, permute, [gather], gate/up, down, combine (empty when
-  // the down GEMM runs the combine)
+  // rmsnorm, router, route, permute, [dequantise + gather], gate/up, down, combine
   return tc_experts(cfg) ? 8 : 7;
 }
 
 int32_t moe_layer_launch_count(const moe_config* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
   if (single_launch(cfg)) return 1;   // with 16-byte aligned tensors
-  // rmsnorm, router, route, gate/up, down and (unless the down GEMM runs it) the
-  // combine, plus the permutation (its own launch, three for large batches, or none
-  // when it shares the routing launch), and for tensor-core experts at wide tiles
-  // the row gather
+  // rmsnorm, router, route, gate/up, down and combine, plus the permutation (its
+  // own launch, three for large batches, or none when it shares the routing
+  // launch), and for tensor-core experts at wide tiles the row gather
   const int gather = tc_experts(cfg) && !gather_in_gemm(cfg) ? 1 : 0;
   if (expert_choice(cfg))   // rmsnorm, router, scores, picks, gate/up, down, combine
     return 7 + gather;
   const int perm = fused_route_permute(cfg) ? 0 : cfg->T * cfg->k > kPermSingleMax ? 3 : 1;
-  return (fused_combine(cfg) ? 5 : 6) + perm + gather;
+  return 6 + perm + gather;
 }
 
 }  // extern "C"

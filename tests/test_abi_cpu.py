@@ -133,18 +133,17 @@ def test_make_weights_maps_every_layer_tensor():
 
 
 # (preset, T) -> kernel launches per layer call.  Decode batches (T <= 32) of bf16
-# experts run as one cooperative launch.  Otherwise five always run (RMSNorm,
-# router, route, gate/up, down) and FP32 experts add the combine (tensor-core
-# experts run it inside the down GEMM's epilogue); the permutation adds 0 (it
-# shares the routing launch up to 32 tokens), 1 (one CTA, T*k <= 4096) or 3
-# (count / scan / rank); tensor-core experts add the row gather unless bf16
-# decode tiles (<= 64 rows per expert on average) gather inside the GEMM
-# (quantised weights are expanded inside the GEMM at every batch).
-LAUNCHES = [("tiny", 64, 7), ("olmoe", 1, 1), ("olmoe", 16, 1), ("olmoe", 64, 6),
-            ("olmoe", 4096, 9), ("v2lite", 32, 1), ("v2lite", 8192, 9),
-            ("qwen3_int4", 1, 6), ("qwen3_int4", 64, 7), ("qwen3_int4", 16384, 9),
-            ("qwen3_int8", 16384, 9), ("qwen3_fp8", 64, 7), ("qwen3_fp8", 16384, 9),
-            ("v3", 32, 1), ("v3", 256, 6), ("v3", 9440, 9)]
+# experts run as one cooperative launch.  Otherwise six always run (RMSNorm,
+# router, route, gate/up, down, combine); the permutation adds 0 (it shares the
+# routing launch up to 32 tokens), 1 (one CTA, T*k <= 4096) or 3 (count / scan /
+# rank); tensor-core experts add the row gather unless bf16 decode tiles (<= 32
+# rows per expert on average) gather inside the GEMM (quantised weights are
+# expanded inside the GEMM at every batch).
+LAUNCHES = [("tiny", 64, 7), ("olmoe", 1, 1), ("olmoe", 16, 1), ("olmoe", 64, 7),
+            ("olmoe", 4096, 10), ("v2lite", 32, 1), ("v2lite", 8192, 10),
+            ("qwen3_int4", 1, 7), ("qwen3_int4", 64, 8), ("qwen3_int4", 16384, 10),
+            ("qwen3_int8", 16384, 10), ("qwen3_fp8", 64, 8), ("qwen3_fp8", 16384, 10),
+            ("v3", 32, 1), ("v3", 256, 7), ("v3", 9440, 10)]
 
 
 @pytest.mark.parametrize("preset,T,n", LAUNCHES)

@@ -296,53 +296,53 @@ def test_layer_is_deterministic_and_replayable():
 
 
 @pytest.mark.parametrize("T", [16, 100, 700])
-def test_fused_combine_with_dropped_tokens(T):
-    """The layer forward runs the combine in the down GEMM's epilogue: the arrival
-    that completes a token's rows sums them.  With no shared expert, k = 1 and a
-    capacity of half the mean load, many tokens keep no row at all; their output
-    must be the residual exactly, and every other token the oracle's value.  T = 16
-    is the single-launch layer (decode tiles), 100 the kernel chain with decode
-    tiles, 700 the chain with prefill tiles.  The separate combine entry point fed
-    the same routed rows gives the same bits."""
-    sh = LayerShape("drop_no_shared", d=256, E=8, k=1, f=256, capacity_factor=0.5, seed=25)
+def test_dropped_tokens_and_combine(T):
+    """With no shared expert, k = 2 and a capacity of half the mean load, half the
+    assignments are dropped and many tokens keep no row at all; their output must
+    be the residual exactly, and every token the oracle's value.  T = 16 is the
+    single-launch layer (decode tiles), 100 the kernel chain with decode tiles,
+    700 the chain with prefill tiles.  The combine entry point fed the layer's
+    routed rows (rounded to bf16 as the layer keeps them) gives the same bits."""
+    sh = LayerShape("drop_no_shared", d=256, E=8, k=2, f=256, capacity_factor=0.5, seed=25)
     li, x, dli, dx = inputs_on_device(sh, T)
     layer = M.MoELayer(dli, T, out_dtype="f32")
-    # one launch; or RMSNorm, router, route, permutation, [row gather], gate/up, down
-    assert M.moe_layer_launch_count(layer.cfg) == {16: 1, 100: 6, 700: 7}[T]
-    slot = torch.empty(T, dtype=torch.int32, device="cuda")
+    # one launch; or RMSNorm, router, route, permutation, [row gather], gate/up, down,
+    # combine
+    assert M.moe_layer_launch_count(layer.cfg) == {16: 1, 100: 7, 700: 8}[T]
     out = layer.forward(dx).clone()
     assert M.moe_get_device_status(layer.ws) == 0
     res = run_layer(sh, T, data=(li, x, dli, dx))
     assert res.max_margin_mismatch < ROUTE_MARGIN
     assert res.err_ratio <= TOL[sh.expert], res.err_ratio
     # tokens without a kept row: out == residual, bit for bit
-    cap = int(np.ceil(0.5 * T * 1 / 8))
-    counts = np.bincount(res.idx[:, 0], minlength=8)
-    assert (counts > cap).any(), "the capacity must drop some tokens"
-    idx = res.idx[:, 0]
-    rank = np.zeros(T, dtype=np.int64)
-    seen = np.zeros(8, dtype=np.int64)
-    for t in range(T):
-        rank[t] = seen[idx[t]]
-        seen[idx[t]] += 1
-    dropped = rank >= cap
+    cap = int(np.ceil(0.5 * T * sh.k / sh.E))
+    flat = res.idx.reshape(-1)                       # assignment a = t*k + j
+    rank = np.zeros(flat.size, dtype=np.int64)
+    seen = np.zeros(sh.E, dtype=np.int64)
+    for a, e in enumerate(flat):
+        rank[a] = seen[e]
+        seen[e] += 1
+    kept = (rank < cap).reshape(T, sh.k)
+    empty = ~kept.any(axis=1)
+    assert empty.any(), "the capacity must leave some tokens without a row"
     xf = dx.float().cpu().numpy()
-    np.testing.assert_array_equal(out.cpu().numpy()[dropped], xf[dropped])
+    np.testing.assert_array_equal(out.cpu().numpy()[empty], xf[empty])
     # the separate combine over the layer's own routed rows gives the same bits
     cfg, w = layer.cfg, layer.w
     ws = M.alloc_workspace(cfg)
     xn = torch.empty(T, sh.d, dtype=torch.bfloat16, device="cuda")
     logits = torch.empty(T, sh.E, dtype=torch.float32, device="cuda")
     M.moe_rmsnorm_router(cfg, w, dx, xn, logits, ws)
-    idx_d = torch.empty(T, dtype=torch.int32, device="cuda")
-    gate = torch.empty(T, dtype=torch.float32, device="cuda")
+    idx_d = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T * sh.k, dtype=torch.float32, device="cuda")
     M.moe_route(cfg, logits, dli.router_bias, idx_d, gate)
     counts_d = torch.empty(sh.E, dtype=torch.int32, device="cuda")
     offs = torch.empty(sh.E + 1, dtype=torch.int32, device="cuda")
-    perm = torch.empty(T, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
+    slot = torch.empty(T * sh.k, dtype=torch.int32, device="cuda")
     drop = torch.empty(1, dtype=torch.int32, device="cuda")
     M.moe_permute(cfg, idx_d, counts_d, offs, perm, slot, drop, ws)
-    y = torch.empty(T, sh.d, dtype=torch.float32, device="cuda")
+    y = torch.empty(T * sh.k, sh.d, dtype=torch.float32, device="cuda")
     M.moe_grouped_ffn(cfg, w, xn, offs, perm, gate, y, None, ws)
     o2 = torch.empty(T, sh.d, dtype=torch.float32, device="cuda")
     M.moe_combine(cfg, y.to(torch.bfloat16).to(torch.float32), slot, None, dx, o2)
