@@ -50,7 +50,7 @@ struct PairConfig {
   static constexpr uint32_t IDESC = idesc_bf16(256, 256, false, true);
   static constexpr int THREADS = kTcBaseThreads;
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
-  static constexpr uint32_t PREFIX_BYTES = 4 * (kMaxGroups + 1) * 4;
+  static constexpr uint32_t PREFIX_BYTES = 5 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 16 * 4;
   static constexpr uint32_t SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
@@ -98,7 +98,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
   int* issued = const_cast<int*>(abort_flag) + 2;   // [STAGES] last issued parity + 1
   int* prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
   float* stg_all = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(prefix + 4 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(prefix + 5 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();   // 0: the CTA that issues the pair's MMAs
@@ -141,7 +141,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
   pdl_trigger();
   if (warp >= 2 && warp - 2 < p.n_prob) {
     const TcProblem& P = p.prob[warp - 2];
-    group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1));
+    group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1),
+                      warp == 2 && P.offsets ? prefix + 4 * (kMaxGroups + 1) : nullptr);
   }
   if (warp == 4 && p.interleave)
     group_class_prefix(p.prob[0].offsets, p.prob[0].G, BN, prefix + 2 * (kMaxGroups + 1),

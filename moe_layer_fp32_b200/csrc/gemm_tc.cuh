@@ -182,9 +182,9 @@ struct TcConfig {
                                                     : idesc_bf16(128, BN, false, false);
   // barriers + bookkeeping after the tiles
   static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * A_SLOTS) + 16 + 4 * STAGES;
-  // tile prefixes of the two problems, then the heavy / light class prefixes of
-  // problem 0 (interleaved order)
-  static constexpr uint32_t PREFIX_BYTES = 4 * (kMaxGroups + 1) * 4;
+  // tile prefixes of the two problems, the heavy / light class prefixes of
+  // problem 0 (interleaved order), and problem 0's group offsets
+  static constexpr uint32_t PREFIX_BYTES = 5 * (kMaxGroups + 1) * 4;
   // swapped epilogue: per-tile output row and scale of each token, one copy per warp;
   // direct DOWN epilogue: a 32-row x 16-column FP32 staging tile per warp through
   // which rows are stored transposed
@@ -245,8 +245,10 @@ MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int TN, i
   ti.g = g;
   int seg_start, seg_rows;
   if (P.offsets) {
-    seg_start = P.offsets[g];
-    seg_rows = P.offsets[g + 1] - seg_start;
+    // problem 0's offsets were copied to shared memory with its tile prefix
+    const int* so = pi == 0 ? prefix + 4 * (kMaxGroups + 1) : P.offsets;
+    seg_start = so[g];
+    seg_rows = so[g + 1] - seg_start;
     ti.b_row = seg_start + ti.m0;
   } else {
     seg_start = g * P.uniform_rows;
@@ -541,7 +543,7 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
       reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
   // epilogue scratch, 16-byte aligned (float4 staging in the direct DOWN epilogue)
   int* epi_row = reinterpret_cast<int*>(
-      (reinterpret_cast<uintptr_t>(prefix + 4 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(prefix + 5 * (kMaxGroups + 1)) + 15) & ~uintptr_t(15));
   float* epi_scale = reinterpret_cast<float*>(epi_row + kEpiWarps * 128);  // [8 warps][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -580,7 +582,8 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   }
   if (warp >= 2 && warp - 2 < p.n_prob) {
     const TcProblem& P = p.prob[warp - 2];
-    group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1));
+    group_tile_prefix(P.offsets, P.G, P.uniform_rows, BN, prefix + (warp - 2) * (kMaxGroups + 1),
+                      warp == 2 && P.offsets ? prefix + 4 * (kMaxGroups + 1) : nullptr);
   }
   if (warp == 4 && p.interleave)
     group_class_prefix(p.prob[0].offsets, p.prob[0].G, BN, prefix + 2 * (kMaxGroups + 1),

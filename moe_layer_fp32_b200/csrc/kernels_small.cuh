@@ -28,14 +28,20 @@ MOE_DEV float warp_max(float v) {
 // Tile prefix over the groups of a grouped problem: prefix[g] = number of
 // BM-row tiles of groups < g.  rows(g) = off[g+1] - off[g], or `uniform` rows
 // when off == nullptr.  Called by one warp; s_off is a shared scratch of G+1.
-MOE_DEV void group_tile_prefix(const int32_t* off, int G, int uniform, int BM, int* prefix) {
+MOE_DEV void group_tile_prefix(const int32_t* off, int G, int uniform, int BM, int* prefix,
+                               int* off_copy = nullptr) {
   const int lane = threadIdx.x & 31;
   int carry = 0;
   if (lane == 0) prefix[0] = 0;
+  if (off_copy && lane == 0) off_copy[0] = off[0];
   for (int c = 0; c < G; c += 32) {
     int g = c + lane;
     int rows = 0;
-    if (g < G) rows = off ? (off[g + 1] - off[g]) : uniform;
+    if (g < G) {
+      const int o1 = off ? off[g + 1] : 0;
+      rows = off ? (o1 - off[g]) : uniform;
+      if (off_copy) off_copy[g + 1] = o1;
+    }
     int v = (rows + BM - 1) / BM;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
