@@ -107,6 +107,9 @@ MOE_DEV void fence_proxy_async_smem() {
 MOE_DEV void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
+MOE_DEV void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 // ---------------------------------------------------------------------------
 // mbarrier

@@ -139,9 +139,10 @@ struct TcConfig {
   // bf16 weights: one ring of TMA stages [weights NA x 16 KB | tokens].
   // int8 / int4 / fp8 weights: a deep ring of TMA stages [tokens | raw weights |
   // scales in a 1 KB slot] (so that enough weight bytes are in flight to cover
-  // HBM latency); the dequantisation warps expand each block into one of two TMEM
-  // slots of bf16 weights, from which the MMA takes its A operand.  Every stage
-  // is 1024-byte aligned.
+  // HBM latency); the dequantisation warps expand each block into a slot of bf16
+  // weights: in TMEM for swapped tiles (the MMA's A operand), in shared memory for
+  // direct tiles (the B operand, K-major, 128-byte swizzle, NA x 128 rows of 128 B
+  // per slot).  Every stage is 1024-byte aligned.
   static constexpr uint32_t STAGE_BYTES =
       WQ == WQ_BF16 ? NA * A_BYTES + B_BYTES : B_BYTES + NA * RAW_BYTES + 1024;
   static constexpr uint32_t TOKEN_OFF = WQ == WQ_BF16 ? NA * A_BYTES : 0;
@@ -150,34 +151,40 @@ struct TcConfig {
   // bytes the TMA delivers per stage
   static constexpr uint32_t TX_BYTES =
       WQ == WQ_BF16 ? STAGE_BYTES : B_BYTES + NA * (RAW_BYTES + SCALE_BYTES);
-  // one dequantisation thread per feature of each weight block: 4 warps per block,
-  // each warp on the TMEM lane quadrant its warp index allows
-  static constexpr int DEQ_WARPS = WQ == WQ_BF16 ? 0 : 4 * NA;
+  // one dequantisation thread per feature of each weight block (4 warps per block,
+  // each warp on the TMEM lane quadrant its warp index allows); direct tiles, whose
+  // expanded weights go to shared memory, two threads per feature (8 warps per
+  // block), each for half of the k-block
+  static constexpr int DEQ_WARPS = WQ == WQ_BF16 ? 0 : (DIRECT ? 8 : 4) * NA;
   static constexpr int THREADS = kTcBaseThreads + 32 * DEQ_WARPS;
-  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  // direct tiles of quantised weights: two shared-memory slots of expanded weights
+  static constexpr bool SMEM_W = DIRECT && WQ != WQ_BF16;
+  static constexpr uint32_t W_SLOT_BYTES = SMEM_W ? NA * 128 * 128 : 0;
+  static constexpr uint32_t A_REGION = 2 * W_SLOT_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024 - A_REGION) / STAGE_BYTES;
   static constexpr int STAGE_CAP = WQ == WQ_BF16 ? 8 : 16;
   static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
-  static constexpr uint32_t A_REGION = 0;
   static constexpr uint32_t ACC_COLS = NA * BN;
   // TMEM: two accumulators, then (quantised weights) A_SLOTS slots of NA bf16
   // weight blocks, 128 lanes x 32 columns each (64 k, two per 32-bit column)
   static constexpr uint32_t A_COL0 = 2 * ACC_COLS;
-  static constexpr uint32_t A_SLOT_COLS = WQ == WQ_BF16 ? 0 : NA * 32;
+  static constexpr uint32_t A_SLOT_COLS = (WQ == WQ_BF16 || SMEM_W) ? 0 : NA * 32;
   // as many weight slots as the TMEM left by the accumulators holds, at most 4, so
   // that the dequantisation warps run up to 4 k-blocks ahead of the MMA
   static constexpr int A_SLOTS_FIT =
       WQ == WQ_BF16 ? 2 : (int)((512 - 2 * ACC_COLS) / (A_SLOT_COLS ? A_SLOT_COLS : 1));
-  static constexpr int A_SLOTS = WQ == WQ_BF16 ? 2 : A_SLOTS_FIT > 4 ? 4 : A_SLOTS_FIT;
+  static constexpr int A_SLOTS = (WQ == WQ_BF16 || SMEM_W) ? 2 : A_SLOTS_FIT > 4 ? 4 : A_SLOTS_FIT;
   static constexpr uint32_t TMEM_NEED = 2 * ACC_COLS + A_SLOTS * A_SLOT_COLS;
   static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                         : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   // swapped: A = weights, M = 128 features, N = BN tokens (K-major), one MMA per
   //          weight block; bf16 weights come from shared memory (MN-major), the
   //          dequantised ones from TMEM (K-major);
-  // direct:  A = tokens (K-major), B = all NA weight blocks at once (MN-major, the
-  //          blocks 16 KB apart = two 64-feature boxes each at the 8 KB leading
-  //          offset), M = 128 tokens, N = 128 * NA
-  static constexpr uint32_t IDESC = DIRECT            ? idesc_bf16(128, 128 * NA, false, true)
+  // direct:  A = tokens (K-major), B = all NA weight blocks at once (bf16: MN-major,
+  //          the blocks 16 KB apart = two 64-feature boxes each at the 8 KB
+  //          leading offset; expanded quantised weights: K-major, one 128-byte row
+  //          per feature), M = 128 tokens, N = 128 * NA
+  static constexpr uint32_t IDESC = DIRECT            ? idesc_bf16(128, 128 * NA, false, !SMEM_W)
                                     : WQ == WQ_BF16 ? idesc_bf16(128, BN, true, false)
                                                     : idesc_bf16(128, BN, false, false);
   // barriers + bookkeeping after the tiles
@@ -195,7 +202,6 @@ struct TcConfig {
   static_assert(SMEM_BYTES + 64 <= 227 * 1024, "shared memory per CTA (dynamic + static)");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0");
   static_assert(!DIRECT || BN == 128, "direct tiles hold 128 tokens");
-  static_assert(WQ == WQ_BF16 || !DIRECT, "quantised weights take the swapped tiles");
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 128-byte swizzle alignment");
   static_assert(NA * SCALE_BYTES <= 1024, "scale slot");
   static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
@@ -344,60 +350,63 @@ MOE_DEV void int4x8_to_bf16(uint32_t v, const uint32_t (&s2)[4], uint32_t (&o)[4
   }
 }
 
-// One feature's 64 codes of a k-block (stored K-contiguous in shared memory: int4
-// 32 bytes, int8 / fp8 64 bytes) to 32 bf16x2 words, k = 2c in the low half of
-// word c, each value bf16(q * s): the exact product rounded once.  The 16-byte
-// pieces are read in a lane-rotated order so that the 8 lanes of each quarter-warp
-// cover all 32 banks.
-template <int WQ>
-MOE_DEV void dequant_row(const uint8_t* row, __nv_bfloat16 s, int lane, uint32_t (&o)[32]) {
-  if (WQ == WQ_INT4) {
-    // load j reads piece (j + r) & 1; swap back when r = 1
-    const int r = (lane >> 2) & 1;
-    uint4 v[2];
+// NC consecutive codes of one feature (64: a whole k-block, 32: half of it;
+// stored K-contiguous in shared memory: int4 NC/2 bytes, int8 / fp8 NC bytes) to
+// NC/2 bf16x2 words, code 2c in the low half of word c, each value bf16(q * s):
+// the exact product rounded once.  The 16-byte pieces are read in a lane-rotated
+// order so that the lanes of each quarter-warp spread over the banks.
+template <int WQ, int NC = 64>
+MOE_DEV void dequant_row(const uint8_t* row, __nv_bfloat16 s, int lane, uint32_t (&o)[NC / 2]) {
+  constexpr int P = (WQ == WQ_INT4 ? NC / 2 : NC) / 16;   // 16-byte pieces of the codes
+  // load j reads piece (j + r) % P, r depending on the lane; rotated back below
+  const int r = P == 1 ? 0 : (lane >> (P == 2 ? 2 : 1)) & (P - 1);
+  uint4 v[P];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) v[j] = *reinterpret_cast<const uint4*>(row + 16 * ((j + r) & 1));
-    if (r) {
-      const uint4 t = v[0];
-      v[0] = v[1];
-      v[1] = t;
+  for (int j = 0; j < P; ++j) v[j] = *reinterpret_cast<const uint4*>(row + 16 * ((j + r) & (P - 1)));
+  if (P == 2 && r) {
+    const uint4 t = v[0];
+    v[0] = v[P - 1];
+    v[P - 1] = t;
+  }
+  if (P == 4) {
+    if (r & 1) {
+      const uint4 t = v[3 % P];
+      v[3 % P] = v[2 % P];
+      v[2 % P] = v[1 % P];
+      v[1 % P] = v[0];
+      v[0] = t;
     }
+    if (r & 2) {
+      uint4 t = v[0];
+      v[0] = v[2 % P];
+      v[2 % P] = t;
+      t = v[1 % P];
+      v[1 % P] = v[3 % P];
+      v[3 % P] = t;
+    }
+  }
+  uint32_t wd[4 * P];
+#pragma unroll
+  for (int j = 0; j < P; ++j) {
+    wd[4 * j] = v[j].x;
+    wd[4 * j + 1] = v[j].y;
+    wd[4 * j + 2] = v[j].z;
+    wd[4 * j + 3] = v[j].w;
+  }
+  if (WQ == WQ_INT4) {
     const uint32_t s2 = (uint32_t)__bfloat16_as_ushort(s) * 0x10001u;
     const uint32_t sp[4] = {s2, s2, s2, s2};
-    const uint32_t wd[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4 * P; ++i) {
       uint32_t q4[4];
       int4x8_to_bf16(wd[i], sp, q4);
 #pragma unroll
       for (int j = 0; j < 4; ++j) o[4 * i + j] = q4[j];
     }
   } else {
-    // load j reads piece (j + r) & 3; rotate back by r (two conditional rotations)
-    const int r = (lane >> 1) & 3;
-    uint4 v[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(row + 16 * ((j + r) & 3));
-    if (r & 1) {
-      const uint4 t = v[3];
-      v[3] = v[2];
-      v[2] = v[1];
-      v[1] = v[0];
-      v[0] = t;
-    }
-    if (r & 2) {
-      uint4 t = v[0];
-      v[0] = v[2];
-      v[2] = t;
-      t = v[1];
-      v[1] = v[3];
-      v[3] = t;
-    }
     const float sf = __bfloat162float(s);
-    const uint32_t wd[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
-                             v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < 4 * P; ++i) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float q0, q1;
@@ -406,11 +415,15 @@ MOE_DEV void dequant_row(const uint8_t* row, __nv_bfloat16 s, int lane, uint32_t
           q0 = q.x;
           q1 = q.y;
         } else {
-          q0 = (float)(int8_t)((wd[i] >> (16 * h)) & 0xff);
-          q1 = (float)(int8_t)((wd[i] >> (16 * h + 8)) & 0xff);
+          // offset binary u = q + 128 placed in the mantissa of 2^23: the float
+          // 2^23 + u, minus 2^23 + 128, is q exactly (full-rate byte permute and
+          // add instead of the quarter-rate integer-to-float conversion)
+          const uint32_t u = wd[i] ^ 0x80808080u;
+          q0 = __uint_as_float(__byte_perm(u, 0x4B000000u, h ? 0x7542 : 0x7540)) - 8388736.f;
+          q1 = __uint_as_float(__byte_perm(u, 0x4B000000u, h ? 0x7543 : 0x7541)) - 8388736.f;
         }
-        __nv_bfloat162 r = __floats2bfloat162_rn(q0 * sf, q1 * sf);
-        o[2 * i + h] = *reinterpret_cast<uint32_t*>(&r);
+        __nv_bfloat162 rr = __floats2bfloat162_rn(q0 * sf, q1 * sf);
+        o[2 * i + h] = *reinterpret_cast<uint32_t*>(&rr);
       }
     }
   }
@@ -530,7 +543,8 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   constexpr int NA = C::NA;
   constexpr int STAGES = C::STAGES;
   uint8_t* tiles = smem;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
+  uint8_t* wslots = tiles + STAGES * C::STAGE_BYTES;   // direct quantised: expanded weights
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(wslots + C::A_REGION);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;       // [2]
@@ -726,7 +740,11 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
             //    Dequantised weights: TMEM, 8 columns (16 k) per step.
             const uint64_t xd = sw128_desc(b_addr + kk * 32, 16, 1024);
             const uint32_t accum = (kb != ti.kb0 || kk != 0);
-            if (WQ != WQ_BF16) {
+            if (C::SMEM_W) {
+              const uint64_t wd =
+                  sw128_desc(smem_u32(wslots + aslot * C::W_SLOT_BYTES) + kk * 32, 16, 1024);
+              tc_mma_f16(d_tmem, xd, wd, C::IDESC, accum);   // N = 128 * NA at once
+            } else if (WQ != WQ_BF16) {
               const uint32_t a_tm = tmem_base + C::A_COL0 + aslot * C::A_SLOT_COLS + kk * 8;
               tc_mma_f16_tmem_a(d_tmem, a_tm, xd, idesc, accum);
               if (NA == 2) tc_mma_f16_tmem_a(d_tmem + BN, a_tm + 32, xd, idesc, accum);
@@ -763,9 +781,13 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   } else if (warp >= 2 + kEpiWarps) {
     // ------------------------------------------------------------ dequantisation
     if (WQ != WQ_BF16) {
-      // warp w expands weight block (w - 10) / 4 for the 32 features of its TMEM lane
-      // quadrant w % 4: one thread per feature, its 64 codes of the k-block
-      const int blk = (warp - 2 - kEpiWarps) >> 2;
+      // swapped tiles: warp w expands weight block (w - 10) / 4 for the 32 features
+      // of its TMEM lane quadrant w % 4, one thread per feature, its 64 codes of the
+      // k-block; direct tiles: warp w, block (w - 10) / 8, codes [32 sub, 32 sub + 32)
+      // with sub = ((w - 10) / 4) % 2, of the features of quadrant w % 4
+      const int dw = warp - 2 - kEpiWarps;
+      const int blk = C::SMEM_W ? dw >> 3 : dw >> 2;
+      const int sub = C::SMEM_W ? (dw >> 2) & 1 : 0;
       const int qd = warp & 3;
       const int feat = qd * 32 + lane;
       int stage = 0;
@@ -784,12 +806,25 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
           const uint8_t* row = st + C::RAW_OFF + blk * C::RAW_BYTES + feat * C::RAW_ROW;
           const __nv_bfloat16 sc =
               reinterpret_cast<const __nv_bfloat16*>(st + C::SCALE_OFF)[128 * blk + feat];
-          uint32_t w[32];
-          dequant_row<WQ>(row, sc, lane, w);
-          tmem_st32(tmem_base + ((uint32_t)(qd * 32) << 16) + C::A_COL0 +
-                        aslot * C::A_SLOT_COLS + blk * 32,
-                    w);
-          tmem_wait_st();
+          if (C::SMEM_W) {
+            uint32_t w[16];
+            dequant_row<WQ, 32>(row + sub * (C::RAW_ROW / 2), sc, lane, w);
+            // row (blk*128 + feat) of the slot, 16-byte chunk c at c ^ (row & 7)
+            const int wr = blk * 128 + feat;
+            uint8_t* dst = wslots + aslot * C::W_SLOT_BYTES + wr * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(dst + 16 * ((4 * sub + c) ^ (wr & 7))) =
+                  make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+            fence_proxy_async_shared();   // the tensor core reads them through the async proxy
+          } else {
+            uint32_t w[32];
+            dequant_row<WQ>(row, sc, lane, w);
+            tmem_st32(tmem_base + ((uint32_t)(qd * 32) << 16) + C::A_COL0 +
+                          aslot * C::A_SLOT_COLS + blk * 32,
+                      w);
+            tmem_wait_st();
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&deq_bar[aslot]);

@@ -88,12 +88,12 @@ inline bool quantised(const moe_config* c) {
 // while each tile's MMA covers only its own rows (rounded up to 16): lightly
 // loaded experts cost no more than before and the heavily loaded ones of a skewed
 // routing stream their weights once per 64 rows instead of once per 16.  Wider
-// (prefill) batches put 128 tokens on M; quantised experts keep the weights on M
-// at every batch, their widest tile holding 96 tokens (two accumulators of
-// 2 x 96 columns and two slots of dequantised weights fill the 512 TMEM columns).
+// (prefill) batches put 128 tokens on M and N = 256 features on the B side; the
+// B operand of quantised experts is expanded by the dequantisation warps into
+// shared memory (one expansion per 128 tokens, four MMAs per k-block).
 int pick_bn(const moe_config* c) {
   const double mean = (double)n_slots(c) / c->E;
-  if (mean > 64) return quantised(c) ? 96 : 128;
+  if (mean > 64) return 128;
   const int most = expert_choice(c) ? ec_capacity(c) : c->T;   // rows one expert can get
   return most <= 16 ? 16 : most <= 32 ? 32 : 64;
 }
@@ -429,8 +429,8 @@ moe_status launch_tc_bn_q(int bn, bool pair, const TcParams& p, cudaStream_t st)
       if constexpr (WQ == WQ_BF16) {   // tokens on MMA-M
         if (pair) return launch_pair<EPI>(p, st);
         return launch_tc<EPI, 128, true, WQ>(p, st);
-      } else {                         // quantised: weights on M, 96 tokens on N
-        return launch_tc<EPI, 96, false, WQ>(p, st);
+      } else {                         // quantised: tokens on M, expanded weights in smem
+        return launch_tc<EPI, 128, true, WQ>(p, st);
       }
   }
 }
