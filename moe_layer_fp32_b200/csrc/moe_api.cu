@@ -107,11 +107,25 @@ constexpr bool kGather4Int = false;   // int8 / int4 / fp8 stages hold 2-4x fewe
 inline bool gather_in_gemm(const moe_config* c) {
   return pick_bn(c) <= kGather4MaxBN && (kGather4Int || c->expert_dtype == MOE_BF16);
 }
+// Quantised decode batches whose expert tiles (estimated from the experts they
+// can touch) fill the SMs take the direct orientation of the prefill tiles too:
+// per k-block four N = 256 MMAs instead of eight N <= 64 ones, the expanded
+// weights in shared memory.  The 128 token rows of such a tile are mostly padding,
+// but the tensor cores are idle at decode while the issue cost of each MMA and the
+// weight expansion bound the swapped tiles.  Smaller batches keep the swapped
+// tiles, split along K.
+inline bool direct_quant_decode(const moe_config* c) {
+  if (!quantised(c) || pick_bn(c) > 64) return false;
+  const double touched = std::min<double>((double)c->E, (double)n_slots(c));
+  return touched * ((c->f + 127) / 128) >= num_sms();
+}
+// Token-tile width the expert GEMMs launch with.
+inline int tile_bn(const moe_config* c) { return direct_quant_decode(c) ? 128 : pick_bn(c); }
 // Split-K of decode tiles when the expert tiles fill at most half the SMs; the
 // GEMM decides per launch from the actual tile count.
 constexpr bool kSplitBf16 = false;   // int experts only: bf16 tiles stream faster whole
 inline bool split_k(const moe_config* c) {
-  return tc_experts(c) && pick_bn(c) <= kGather4MaxBN &&
+  return tc_experts(c) && tile_bn(c) <= kGather4MaxBN &&
          (kSplitBf16 || c->expert_dtype != MOE_BF16);
 }
 inline int split_counters() { return num_sms() * 8; }
@@ -649,7 +663,7 @@ moe_status gateup_params(const moe_config* c, const moe_weights* w, const moe_we
                          const void* xn, const void* xp, const int32_t* offsets, RoutedRows rr,
                          __nv_bfloat16* h, float* split_part, int32_t* split_cnt, int32_t* err,
                          TcParams& p) {
-  const int T = c->T, S = c->n_shared, bn = pick_bn(c), R = (int)n_slots(c);
+  const int T = c->T, S = c->n_shared, bn = tile_bn(c), R = (int)n_slots(c);
   const bool g4 = gather_in_gemm(c);
   p = TcParams{};
   TcProblem& P = p.prob[0];
@@ -710,7 +724,7 @@ moe_status down_params(const moe_config* c, const moe_weights* w, const moe_weig
                        const int32_t* offsets, RoutedRows rr, const float* gate,
                        const __nv_bfloat16* h, void* y, bool rows_bf16, float* ys,
                        float* split_part, int32_t* split_cnt, int32_t* err, TcParams& p) {
-  const int T = c->T, S = c->n_shared, bn = pick_bn(c), R = (int)n_slots(c);
+  const int T = c->T, S = c->n_shared, bn = tile_bn(c), R = (int)n_slots(c);
   const int32_t* perm = rr.dst;
   p = TcParams{};
   TcProblem& P = p.prob[0];
@@ -822,7 +836,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
       if (!a16(o)) return MOE_ERR_INVALID;
   }
   __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
-  const int bn = pick_bn(c);
+  const int bn = tile_bn(c);
   const int R = (int)n_slots(c);
   const int wq = wq_of(c);
   const moe_weights& wl = *w;

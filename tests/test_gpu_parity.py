@@ -44,6 +44,12 @@ SMALL = {
                              bias_mode="logit", seed=22),
     "fp8_prefill": LayerShape("fp8_prefill", d=512, E=8, k=2, f=384, expert="fp8",
                               capacity_factor=1.25, seed=23),
+    # quantised decode tiles that fill the SMs (64 experts x 3 feature tiles): the
+    # direct orientation with 128-token tiles, expanded weights in shared memory
+    "int4_decode_direct": LayerShape("int4_decode_direct", d=256, E=64, k=8, f=384, n_shared=1,
+                                     expert="int4", seed=26),
+    "int8_decode_direct": LayerShape("int8_decode_direct", d=256, E=64, k=6, f=384,
+                                     expert="int8", bias_mode="logit", seed=27),
     # FP32 experts with f not a multiple of 4 (scalar weight columns in gate/up)
     "f32_odd_f": LayerShape("f32_odd_f", d=136, E=6, k=2, f=130, n_shared=1, act="f32",
                             router="f32", expert="f32", capacity_factor=1.5,
@@ -53,7 +59,7 @@ SMALL_T = {"bf16_plain": 100, "bf16_shared_cap": 77, "bf16_select_tc_router": 20
            "bf16_prefill_tiles": 1000, "f32_tiny": 64, "int4_decode": 20, "int8_decode": 50,
            "int4_prefill": 900, "int8_prefill": 700, "f32_odd_f": 37,
            "bf16_tc_router_split": 300, "bf16_prefill_skew": 700, "fp8_decode": 40,
-           "fp8_prefill": 800}
+           "fp8_prefill": 800, "int4_decode_direct": 40, "int8_decode_direct": 61}
 
 
 @pytest.fixture(autouse=True)
@@ -167,7 +173,8 @@ def test_permute_flags_out_of_range_expert():
 # --------------------------------------------------------------------- a6 + a7
 @pytest.mark.parametrize("name", ["bf16_plain", "bf16_shared_cap", "bf16_prefill_tiles", "f32_tiny",
                                   "int4_decode", "int8_decode", "int4_prefill", "int8_prefill",
-                                  "bf16_prefill_skew", "fp8_decode", "fp8_prefill"])
+                                  "bf16_prefill_skew", "fp8_decode", "fp8_prefill",
+                                  "int4_decode_direct", "int8_decode_direct"])
 def test_grouped_ffn_matches_oracle_per_assignment(name):
     sh, T = SMALL[name], SMALL_T[name]
     li, x, dli, dx = inputs_on_device(sh, T)
