@@ -56,6 +56,9 @@ def parse_args():
                    help="skip the other configurations (decode and prefill batches)")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-parity", action="store_true")
+    p.add_argument("--prefill-tiles", choices=["auto", "single", "pair"], default="auto",
+                   help="bf16 prefill tiles: chosen by rows per expert (auto), 128-token tiles "
+                        "on single CTAs, or 256-token tiles on CTA pairs")
     return p.parse_args()
 
 
@@ -215,6 +218,7 @@ def run_ours(args):
     x_host = moe_synth.make_x(sh, T, stream=T + 7919 * rank)
     x = x_host.to(dev)
     layer = M.MoELayer(li, T)            # output in the activation dtype (bf16)
+    layer.cfg.prefill_tiles = {"auto": 0, "single": 1, "pair": 2}[args.prefill_tiles]
     cfg = layer.cfg
     L = M.moe_layer_launch_count(cfg)
     n_steps = M.moe_layer_step_count(cfg)
@@ -300,7 +304,8 @@ def run_ours(args):
            "steps": K, "warmup": W, "ms_per_step": round(ms_max / K, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic (seeded N(0,1) tokens, fan-in-scaled random expert weights)",
-           "config": config_dict(sh, T, world), "roofline": roof, "layer_roofline": layer_roof,
+           "config": dict(config_dict(sh, T, world), prefill_tiles=args.prefill_tiles),
+           "roofline": roof, "layer_roofline": layer_roof,
            "e2e": e2e, "gpu_launches": L * K, "launches_per_step": L, "clocks": clk,
            "kernels_avg_us": {k: round(v * 1e3, 2) for k, v in per_kernel.items()}}
     if rank == 0 and world == 1 and not args.no_parity:
