@@ -8,7 +8,8 @@
 // grid-wide barriers:
 //   1. RMSNorm, one token per CTA;
 //   2. the router's K-sliced partial logits, (8 tokens x 128 rows) per work item;
-//   3. routing, one token per CTA, then -- without a barrier -- the counting-sort
+//   3. routing (one token per CTA and a barrier; or, for small problems, every
+//      token by every CTA), then -- without a barrier -- the counting-sort
 //      permutation, built by every CTA (it is small);
 //   4. the grouped gate/up GEMM over the routed rows (tcgen05, 16 or 32 token
 //      tiles, rows gathered by the GEMM's own TMA; split along K when the tiles
@@ -54,6 +55,7 @@ struct DecodeParams {
   double eps;
   int T, d, E, k, S, mode, renorm, cap;
   int ns, rows;                   // router: ns K-slices of `rows` rows
+  int route_all;                  // every CTA routes every token (no barrier before permuting)
   int n_split_cnt;                // split-K tile counters (gu.split_cnt == dn.split_cnt)
 };
 
@@ -231,30 +233,54 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                          (w % groups) * 8, w / groups, sm_r);
     ok = grid_barrier(p.grid_bar, nb, gen, true, p.wait_cycles, p.err, &s_ok);
   }
-  // 3. routing: CTA t routes token t -- every thread adds one expert's partial
-  //    logits in slice order, then warp 0 selects
+  // 3. routing.  Small problems (T * ns * E partial sums, at most 32K): every CTA
+  //    routes every token itself -- all threads add the partial logits of
+  //    (token, expert) pairs in slice order, then warp w selects for tokens w,
+  //    w + 10, ... -- writing the same routes to the workspace, so that no grid
+  //    barrier is needed before the permutation.  Otherwise CTA t routes token t
+  //    and a barrier follows.
   if (ok) {
     float* s_lg = reinterpret_cast<float*>(smem);
-    for (int t = blockIdx.x; t < p.T; t += nb) {
-      for (int e = threadIdx.x; e < p.E; e += kDecodeThreads) {
-        const float* pe = p.part + (size_t)t * p.E + e;
-        const size_t stride = (size_t)p.T * p.E;
+    const size_t stride = (size_t)p.T * p.E;
+    if (p.route_all) {
+      for (int i = threadIdx.x; i < p.T * p.E; i += kDecodeThreads) {
+        const float* pe = p.part + i;   // [slice][t][e], i = t * E + e
         float acc = 0.f;
 #pragma unroll 8
         for (int sl = 0; sl < p.ns; ++sl) acc += pe[sl * stride];
-        s_lg[e] = acc;
+        s_lg[i] = acc;
       }
       __syncthreads();
-      if (warp == 0) {
+      for (int t = warp; t < p.T; t += kDecodeThreads / 32) {
         float lg[EPL];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) lg[i] = lane + 32 * i < p.E ? s_lg[lane + 32 * i] : 0.f;
+        for (int i = 0; i < EPL; ++i)
+          lg[i] = lane + 32 * i < p.E ? s_lg[t * p.E + lane + 32 * i] : 0.f;
         route_select<EPL>(lg, p.E, p.k, p.bias, p.mode, p.renorm, p.idx, p.gate, p.logits_out,
                           t, lane);
       }
-      __syncthreads();
+      __syncthreads();   // this CTA's routes, written above, are what its permutation reads
+    } else {
+      for (int t = blockIdx.x; t < p.T; t += nb) {
+        for (int e = threadIdx.x; e < p.E; e += kDecodeThreads) {
+          const float* pe = p.part + (size_t)t * p.E + e;
+          float acc = 0.f;
+#pragma unroll 8
+          for (int sl = 0; sl < p.ns; ++sl) acc += pe[sl * stride];
+          s_lg[e] = acc;
+        }
+        __syncthreads();
+        if (warp == 0) {
+          float lg[EPL];
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) lg[i] = lane + 32 * i < p.E ? s_lg[lane + 32 * i] : 0.f;
+          route_select<EPL>(lg, p.E, p.k, p.bias, p.mode, p.renorm, p.idx, p.gate, p.logits_out,
+                            t, lane);
+        }
+        __syncthreads();
+      }
+      ok = grid_barrier(p.grid_bar, nb, gen, true, p.wait_cycles, p.err, &s_ok);
     }
-    ok = grid_barrier(p.grid_bar, nb, gen, true, p.wait_cycles, p.err, &s_ok);
   }
   // the permutation of the T*k <= 1024 assignments: every CTA builds it (one warp),
   // writing the same values to the workspace, and reads back only what it wrote

@@ -1067,6 +1067,7 @@ moe_status run_decode_layer(const moe_config* c, const moe_weights* w, const voi
   dp.cap = capacity_rows(c);
   dp.ns = L.ns;
   dp.rows = kRouterSlice;
+  dp.route_all = (long long)c->T * L.ns * c->E <= 32768 ? 1 : 0;
   const int bn = pick_bn(c);
 #define MOE_DECODE(EPL)                                                        \
   return bn == 16 ? launch_decode<EPL, 16>(dp, st) : launch_decode<EPL, 32>(dp, st)
