@@ -313,22 +313,16 @@ MOE_DEV uint32_t idesc_with_n(uint32_t idesc, int n) {
   return (idesc & ~(0x3Fu << 17)) | ((uint32_t)(n >> 3) << 17);
 }
 
-// Dequantise one raw weight block (128 features x 64 k of tile (g, n, kb)) into the
-// bf16 MN-major layout with the 128-byte swizzle that a TMA load would have
-// produced: 16-byte chunk cc (8 features) of k-row k of 64-feature half h sits at
-// h * 8192 + k * 128 + ((cc ^ (k & 7)) << 4).  Value = bf16(q * s), the exact
-// product rounded once; the block's 128 scales were loaded by the TMA with it.
-// Features at or beyond N were zero-filled by the TMA (q = 0, s = 0).
-// Eight int4 values (two's complement nibbles, nibble j = feature j) to bf16 q*s,
-// packed as four bf16x2 pairs of consecutive features.  XOR 8 turns each nibble
+// Eight int4 values (two's complement nibbles, nibble j = code j of the row) to
+// bf16 q*s, packed as four bf16x2 pairs of consecutive codes.  XOR 8 turns each nibble
 // into the offset value q + 8 in [0, 15]; OR-ing it into the low mantissa bits of
 // bf16 128.0 (0x4300) gives exactly 136 + q; subtracting 136.0 (0x4308) leaves q
-// exactly; byte permutes restore feature order and one bf16x2 multiply by the
+// exactly; byte permutes restore the code order and one bf16x2 multiply by the
 // scale pair yields the exact product q*s rounded once (round to nearest even).
 MOE_DEV void int4x8_to_bf16(uint32_t v, const uint32_t (&s2)[4], uint32_t (&o)[4]) {
   v ^= 0x88888888u;
   const uint32_t magic = 0x43004300u;
-  uint32_t a = (v & 0x000F000Fu) | magic;           // features (0, 4)
+  uint32_t a = (v & 0x000F000Fu) | magic;           // codes (0, 4)
   uint32_t b = ((v >> 4) & 0x000F000Fu) | magic;    // (1, 5)
   uint32_t c = ((v >> 8) & 0x000F000Fu) | magic;    // (2, 6)
   uint32_t d = ((v >> 12) & 0x000F000Fu) | magic;   // (3, 7)
