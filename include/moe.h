@@ -139,8 +139,10 @@ typedef struct moe_config {
  *   s_down      INT8, FP8: bf16 [E, d]; INT4: bf16 [E, f/128, d]; otherwise NULL
  *   sh_*        the same for the n_shared shared experts ([S, ...]); NULL if S == 0
  * int8 weights are symmetric with one scale per output column; int4 weights are
- * symmetric signed 4-bit, two per byte along the contiguous (reduction) dim, low
- * nibble = even k, with one scale per 128 rows of K and output column; fp8
+ * symmetric signed 4-bit (two's complement), two per byte along the contiguous
+ * (reduction) dim, eight per 4-byte word: nibble j of the little-endian word holds
+ * k = 8w + (0, 2, 4, 6, 1, 3, 5, 7)[j] (even k in the low nibbles of the word's bytes,
+ * odd k in the high ones), with one scale per 128 rows of K and output column; fp8
  * weights are E4M3 codes (no infinities, largest finite 448) with one scale per
  * output column.  In every case the weight the layer uses is bf16(q * s): the
  * exact product rounded once, formed inside the expert GEMM's main loop. */

@@ -313,34 +313,25 @@ MOE_DEV uint32_t idesc_with_n(uint32_t idesc, int n) {
   return (idesc & ~(0x3Fu << 17)) | ((uint32_t)(n >> 3) << 17);
 }
 
-// Eight int4 values (two's complement nibbles, nibble j = code j of the row) to
-// bf16 q*s, packed as four bf16x2 pairs of consecutive codes.  XOR 8 turns each nibble
-// into the offset value q + 8 in [0, 15]; OR-ing it into the low mantissa bits of
-// bf16 128.0 (0x4300) gives exactly 136 + q; subtracting 136.0 (0x4308) leaves q
-// exactly; byte permutes restore the code order and one bf16x2 multiply by the
-// scale pair yields the exact product q*s rounded once (round to nearest even).
+// Eight int4 codes of one 4-byte word (two's complement nibbles; nibble j of the
+// little-endian word holds code (0, 2, 4, 6, 1, 3, 5, 7)[j] of the eight, the storage
+// order of the layer's int4 weights) to bf16 q*s, packed as four bf16x2 pairs of
+// consecutive codes.  XOR 8 turns each nibble into the offset value q + 8 in
+// [0, 15]; masking nibbles j and j + 4 -- codes 2j and 2j+1 -- into the low mantissa
+// bits of the two halves of bf16 128.0 (0x4300) gives exactly 136 + q; subtracting
+// 136.0 (0x4308) leaves q exactly; one bf16x2 multiply by the scale pair yields the
+// exact product q*s rounded once (round to nearest even).
 MOE_DEV void int4x8_to_bf16(uint32_t v, const uint32_t (&s2)[4], uint32_t (&o)[4]) {
   v ^= 0x88888888u;
   const uint32_t magic = 0x43004300u;
-  uint32_t a = (v & 0x000F000Fu) | magic;           // codes (0, 4)
-  uint32_t b = ((v >> 4) & 0x000F000Fu) | magic;    // (1, 5)
-  uint32_t c = ((v >> 8) & 0x000F000Fu) | magic;    // (2, 6)
-  uint32_t d = ((v >> 12) & 0x000F000Fu) | magic;   // (3, 7)
   const __nv_bfloat162 k136 = __halves2bfloat162(__ushort_as_bfloat16(0x4308),
                                                  __ushort_as_bfloat16(0x4308));
-  __nv_bfloat162 qa = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), k136);
-  __nv_bfloat162 qb = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&b), k136);
-  __nv_bfloat162 qc = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&c), k136);
-  __nv_bfloat162 qd = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&d), k136);
-  const uint32_t ua = *reinterpret_cast<uint32_t*>(&qa), ub = *reinterpret_cast<uint32_t*>(&qb);
-  const uint32_t uc = *reinterpret_cast<uint32_t*>(&qc), ud = *reinterpret_cast<uint32_t*>(&qd);
-  uint32_t p[4] = {__byte_perm(ua, ub, 0x5410), __byte_perm(uc, ud, 0x5410),
-                   __byte_perm(ua, ub, 0x7632), __byte_perm(uc, ud, 0x7632)};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&p[i]),
-                               *reinterpret_cast<const __nv_bfloat162*>(&s2[i]));
-    o[i] = *reinterpret_cast<uint32_t*>(&r);
+    uint32_t a = ((v >> (4 * i)) & 0x000F000Fu) | magic;   // codes (2i, 2i + 1)
+    const __nv_bfloat162 q = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), k136);
+    const __nv_bfloat162 r = __hmul2(q, *reinterpret_cast<const __nv_bfloat162*>(&s2[i]));
+    o[i] = *reinterpret_cast<const uint32_t*>(&r);
   }
 }
 

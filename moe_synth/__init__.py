@@ -29,7 +29,8 @@ Recipe (every tensor draws from its own PCG64 stream,
   ``s = bf16(max|w| / 448)``, ``q = e4m3(w / s)`` (round to nearest even).
 * int4 weights: symmetric, groups of ``group_size`` along the reduction (K) dim,
   ``s = bf16(max|w| / 7)``, ``q = clamp(rint(w / s), -8, 7)``; two values per byte
-  along the contiguous (K) dim, low nibble first.
+  along the contiguous (K) dim, eight per 4-byte word: nibble j of the
+  little-endian word holds code 8w + (0, 2, 4, 6, 1, 3, 5, 7)[j].
 
 Weight layouts follow the layer's statement of the problem: ``W_r[d, E]``,
 ``W_gate/W_up[E, d, f]``, ``W_down[E, f, d]``; shared experts ``[S, d, f]`` and
@@ -193,8 +194,9 @@ def quantize_int4(w: torch.Tensor, group: int) -> Tuple[torch.Tensor, torch.Tens
     """w[K, N] fp32 -> (packed uint8 [N, K/2], s bf16 [K/group, N]).
 
     Groups of ``group`` rows along K share a scale per column.  The codes are
-    stored with K contiguous (the transpose of w): byte j of row n holds k = 2j in
-    its low nibble and k = 2j+1 in its high nibble.
+    stored with K contiguous (the transpose of w), eight codes per 4-byte word:
+    nibble j of the little-endian word holds code 8w + (0, 2, 4, 6, 1, 3, 5, 7)[j]
+    (the even codes in the low nibbles of its bytes, the odd ones in the high).
     """
     K, N = w.shape
     wg = w.view(K // group, group, N)
@@ -202,9 +204,10 @@ def quantize_int4(w: torch.Tensor, group: int) -> Tuple[torch.Tensor, torch.Tens
     s = (amax / 7.0).to(torch.bfloat16)
     s = torch.where(s.float() > 0, s, torch.ones_like(s))
     q = torch.round(wg / s.float().unsqueeze(1)).clamp_(-8, 7).to(torch.int16).view(K, N)
-    qt = q.t()
-    lo = (qt[:, 0::2] & 0xF)
-    hi = (qt[:, 1::2] & 0xF) << 4
+    qt = q.t().contiguous().view(N, K // 8, 8)
+    nib = qt[:, :, [0, 2, 4, 6, 1, 3, 5, 7]].reshape(N, K) & 0xF   # nibble j of each word
+    lo = nib[:, 0::2]
+    hi = nib[:, 1::2] << 4
     return (lo | hi).to(torch.uint8).contiguous(), s
 
 

@@ -308,14 +308,25 @@ def permute(idx, E: int, capacity_factor: float = 0.0) -> Dict[str, np.ndarray]:
 # ---------------------------------------------------------------------------
 # expert weights as the layer sees them
 # ---------------------------------------------------------------------------
+# Nibble j of each little-endian 4-byte word of int4 codes holds code 8w + INT4_ORDER[j]
+# of that word's eight: the even codes in the low nibbles of the four bytes, the odd
+# ones in the high nibbles (byte 0: codes 0 and 2, byte 1: 4 and 6, byte 2: 1 and 3,
+# byte 3: 5 and 7).
+INT4_ORDER = (0, 2, 4, 6, 1, 3, 5, 7)
+
+
 def unpack_int4(packed) -> np.ndarray:
-    """uint8 [R, C/2] -> int [R, C]; low nibble = even column, two's complement."""
+    """uint8 [R, C/2] -> int [R, C] (C a multiple of 8), two's complement nibbles
+    in the word order INT4_ORDER."""
     p = np.asarray(packed, dtype=np.uint8).astype(np.int64)
-    lo = p & 0xF
-    hi = (p >> 4) & 0xF
-    q = np.empty((p.shape[0], p.shape[1] * 2), dtype=np.int64)
-    q[:, 0::2] = lo
-    q[:, 1::2] = hi
+    R, nb = p.shape
+    nib = np.empty((R, nb * 2), dtype=np.int64)
+    nib[:, 0::2] = p & 0xF            # nibble 2b of the stream: low half of byte b
+    nib[:, 1::2] = (p >> 4) & 0xF
+    nib = nib.reshape(R, nb // 4, 8)
+    q = np.empty_like(nib)
+    q[:, :, list(INT4_ORDER)] = nib   # nibble j -> code INT4_ORDER[j]
+    q = q.reshape(R, nb * 2)
     return np.where(q >= 8, q - 16, q)
 
 
