@@ -117,7 +117,7 @@ typedef struct moe_config {
                               half a second).  A wait that runs out sets device error 2
                               and the kernel returns early (moe_get_device_status)      */
   int32_t routing;         /* moe_routing (0 = top-k)                                    */
-  int32_t prefill_tiles;   /* bf16 experts at prefill (more than 64 rows per expert on
+  int32_t prefill_tiles;   /* tensor-core experts at prefill (more than 64 rows per expert on
                               average): 1 = tiles of 128 tokens on single CTAs, 2 = tiles
                               of 256 tokens on pairs of CTAs (one cta_group::2 MMA per
                               k-step), 0 = automatic: pairs when the batch averages at

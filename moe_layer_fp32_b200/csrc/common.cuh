@@ -343,6 +343,12 @@ MOE_DEV uint32_t mapa_shared(const void* p, uint32_t rank) {
 MOE_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// arrive that releases the caller's earlier writes at cluster scope (shared-memory
+// data that the pair's MMA, issued by the other CTA, is about to read)
+MOE_DEV void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
 MOE_DEV void st_shared_remote_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }

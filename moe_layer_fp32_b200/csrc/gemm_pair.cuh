@@ -35,25 +35,44 @@
 
 namespace moe {
 
-template <int EPI>
+template <int EPI, int WQ = WQ_BF16>
 struct PairConfig {
+  static constexpr bool QUANT = WQ != WQ_BF16;
   static constexpr int BN = 256;                                   // tokens per pair tile
   static constexpr int TILE_N = EPI == EPI_GATEUP ? 128 : 256;     // features per tile
   static constexpr uint32_t B_HALF = 128 * 64 * 2;   // 128 weight columns x 64 k
   static constexpr uint32_t A_BYTES = 128 * 64 * 2;  // 128 token rows x 64 k
-  static constexpr uint32_t STAGE_BYTES = B_HALF + A_BYTES;
-  static constexpr uint32_t TOKEN_OFF = B_HALF;
-  static constexpr int STAGES = 6;
+  // quantised weights: this CTA's 128 features x 64 codes, K-contiguous rows, and
+  // their 128 bf16 scales in a 1 KB slot
+  static constexpr uint32_t RAW_ROW = ByteWeights<WQ>::value ? 64 : WQ == WQ_INT4 ? 32 : 0;
+  static constexpr uint32_t RAW_BYTES = 128 * RAW_ROW;
+  static constexpr uint32_t SCALE_BYTES = QUANT ? 256 : 0;
+  // bf16 stage: [weights | tokens]; quantised stage: [tokens | codes | scales]
+  static constexpr uint32_t STAGE_BYTES = QUANT ? A_BYTES + RAW_BYTES + 1024 : B_HALF + A_BYTES;
+  static constexpr uint32_t TOKEN_OFF = QUANT ? 0 : B_HALF;
+  static constexpr uint32_t RAW_OFF = A_BYTES;
+  static constexpr uint32_t SCALE_OFF = A_BYTES + RAW_BYTES;
+  // quantised: two shared-memory slots of this CTA's expanded weights (the MMA's B
+  // half), 128 rows of 128 B, K-major with the 128-byte swizzle
+  static constexpr uint32_t W_SLOT_BYTES = QUANT ? 128 * 128 : 0;
+  static constexpr uint32_t W_REGION = 2 * W_SLOT_BYTES;
+  static constexpr int STAGES_RAW = (184 * 1024 - W_REGION) / STAGE_BYTES;
+  static constexpr int STAGES = QUANT ? (STAGES_RAW > 8 ? 8 : STAGES_RAW) : 6;
   static constexpr uint32_t ACC_COLS = 256;
   static constexpr uint32_t TMEM_COLS = 512;
-  // A = tokens (K-major), B = weights (MN-major); M = 256 tokens, N = 256 columns
-  static constexpr uint32_t IDESC = idesc_bf16(256, 256, false, true);
-  static constexpr int THREADS = kTcBaseThreads;
-  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16 + 4 * STAGES;
+  // A = tokens (K-major); B = weights, bf16 MN-major as loaded, expanded K-major;
+  // M = 256 tokens, N = 256 columns
+  static constexpr uint32_t IDESC = idesc_bf16(256, 256, false, !QUANT);
+  // two dequantisation threads per feature of this CTA's half, each for 32 codes
+  static constexpr int DEQ_WARPS = QUANT ? 8 : 0;
+  static constexpr int THREADS = kTcBaseThreads + 32 * DEQ_WARPS;
+  // full, empty, [raw full] per stage; tfull, tempty, drain; [deq, wempty] x 2
+  static constexpr uint32_t BAR_BYTES =
+      8 * (2 * STAGES + 5 + (QUANT ? STAGES + 4 : 0)) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 5 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 16 * 4;
   static constexpr uint32_t SMEM_BYTES =
-      1024 + STAGES * STAGE_BYTES + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
+      1024 + STAGES * STAGE_BYTES + W_REGION + BAR_BYTES + PREFIX_BYTES + 16 + EPI_BYTES;
   static_assert(SMEM_BYTES + 64 <= 227 * 1024, "shared memory per CTA (dynamic + static)");
   static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 128-byte swizzle alignment");
 };
@@ -77,10 +96,10 @@ MOE_DEV bool pair_wait(uint64_t* bar, uint32_t parity, const TcParams& p, volati
   }
 }
 
-template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
+template <int EPI, int WQ = WQ_BF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>::THREADS, 1)
     k_tc_gemm_pair(const __grid_constant__ TcParams p) {
-  using C = PairConfig<EPI>;
+  using C = PairConfig<EPI, WQ>;
   constexpr int STAGES = C::STAGES;
   constexpr int BN = C::BN;
   constexpr int TN = C::TILE_N;
@@ -88,12 +107,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
+  uint8_t* wslots = tiles + STAGES * C::STAGE_BYTES;   // quantised: expanded weights
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(wslots + C::W_REGION);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;       // [2]
   uint64_t* drain_bar = tempty_bar + 2;       // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  // quantised: this CTA's codes landed [STAGES] (local); both CTAs' weight slot a
+  // expanded [2] (the even CTA's, counted by both CTAs' dequantisation warps); this
+  // CTA's slot a read by the MMAs [2] (local)
+  uint64_t* rawfull_bar = drain_bar + 1;
+  uint64_t* deq_bar = rawfull_bar + (C::QUANT ? STAGES : 0);
+  uint64_t* wempty_bar = deq_bar + (C::QUANT ? 2 : 0);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty_bar + (C::QUANT ? 2 : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* issued = const_cast<int*>(abort_flag) + 2;   // [STAGES] last issued parity + 1
   int* prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
@@ -116,6 +142,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       mbar_init(&tempty_bar[a], 2 * kEpiWarps);
     }
     mbar_init(drain_bar, 1);
+    if (C::QUANT) {
+      for (int s = 0; s < STAGES; ++s) mbar_init(&rawfull_bar[s], 1);
+      for (int a = 0; a < 2; ++a) {
+        mbar_init(&deq_bar[a], 2 * C::DEQ_WARPS);
+        mbar_init(&wempty_bar[a], 1);
+      }
+    }
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -129,6 +162,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       tma_prefetch_desc(&p.prob[pi].tmA);
       if (EPI == EPI_GATEUP) tma_prefetch_desc(&p.prob[pi].tmA2);
       tma_prefetch_desc(&p.prob[pi].tmB);
+      if (C::QUANT) {
+        tma_prefetch_desc(&p.prob[pi].tmS);
+        if (EPI == EPI_GATEUP) tma_prefetch_desc(&p.prob[pi].tmS2);
+      }
     }
   }
   // both CTAs' barriers are initialised (and the TMEM allocated) before either
@@ -177,12 +214,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
             break;
           }
           uint8_t* st = tiles + stage * C::STAGE_BYTES;
-          // the even CTA arms the stage for both CTAs' bytes
-          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE_BYTES);
           issued[stage] = (int)phase + 1;
           const uint32_t fb = full_even + stage * 8;
-          tma_load_3d_pair(st, wmap, fb, wn, kb * 64, ti.g);
-          tma_load_3d_pair(st + 8192, wmap, fb, wn + 64, kb * 64, ti.g);
+          if (!C::QUANT) {
+            // the even CTA arms the stage for both CTAs' bytes
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE_BYTES);
+            tma_load_3d_pair(st, wmap, fb, wn, kb * 64, ti.g);
+            tma_load_3d_pair(st + 8192, wmap, fb, wn + 64, kb * 64, ti.g);
+          } else {
+            // tokens of both CTAs complete on the even CTA's barrier; this CTA's
+            // codes and scales on its own, where its dequantisation warps wait.
+            // Codes stored K-contiguous [G][N][K bytes] (x: the k-block's byte
+            // offset in a feature's row, y: the first feature); scales int8 / fp8
+            // [G][N], int4 [G][K/128][N]
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::A_BYTES);
+            mbar_arrive_expect_tx(&rawfull_bar[stage], C::RAW_BYTES + C::SCALE_BYTES);
+            const void* smap = (EPI == EPI_GATEUP && rank == 1) ? (const void*)&P.tmS2
+                                                                 : (const void*)&P.tmS;
+            tma_load_3d(st + C::RAW_OFF, wmap, &rawfull_bar[stage], kb * (int)C::RAW_ROW, wn, ti.g);
+            if (WQ != WQ_INT4)
+              tma_load_3d(st + C::SCALE_OFF, smap, &rawfull_bar[stage], wn, ti.g, 0);
+            else
+              tma_load_3d(st + C::SCALE_OFF, smap, &rawfull_bar[stage], wn, kb / 2, ti.g);
+          }
           tma_load_2d_pair(st + C::TOKEN_OFF, &P.tmB, fb, kb * 64, brow);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -194,8 +248,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       // -------------------------------------------------- MMA issuer (even CTA)
       const uint32_t empty_peer = mapa_shared(empty_bar, peer);
       const uint32_t tfull_peer = mapa_shared(tfull_bar, peer);
+      const uint32_t wempty_peer = mapa_shared(wempty_bar, peer);
       int stage = 0;
       uint32_t phase = 0;
+      int aslot = 0;
+      uint32_t aphase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -211,21 +268,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
             ok = false;
             break;
           }
+          if (C::QUANT && !pair_wait(&deq_bar[aslot], aphase, p, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t st_addr = smem_u32(tiles + stage * C::STAGE_BYTES);
+          const uint32_t w_addr = smem_u32(wslots + aslot * C::W_SLOT_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             // tokens: K-major SW128, 16 k = 32 B per step, 8-row groups 1 KB apart;
-            // weights: MN-major SW128, 16 k-rows of 128 B per step, the two
-            // 64-column halves 8 KB apart, 8-row groups 1 KB apart
+            // bf16 weights: MN-major SW128, 16 k-rows of 128 B per step, the two
+            // 64-column halves 8 KB apart, 8-row groups 1 KB apart; expanded
+            // weights: K-major SW128 like the tokens (each CTA's slot at the same
+            // offset holds its 128 of the 256 columns)
             const uint64_t ad = sw128_desc(st_addr + C::TOKEN_OFF + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
+            const uint64_t bd = C::QUANT ? sw128_desc(w_addr + kk * 32, 16, 1024)
+                                         : sw128_desc(st_addr + kk * 2048, 8192, 1024);
             tc2_mma_f16(d_tmem, ad, bd, C::IDESC, (kb != 0 || kk != 0) ? 1u : 0u);
           }
-          // stage s of both CTAs is free once these MMAs have read it
+          // stage s (and weight slot a) of both CTAs are free once these MMAs have
+          // read them
           tc2_commit(smem_u32(&empty_bar[stage]));
           tc2_commit(empty_peer + stage * 8);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (C::QUANT) {
+            tc2_commit(smem_u32(&wempty_bar[aslot]));
+            tc2_commit(wempty_peer + aslot * 8);
+            if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+          }
         }
         if (!ok) break;
         tc2_commit(smem_u32(&tfull_bar[acc]));
@@ -239,6 +310,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kWaitCycles) {}
     }
     __syncwarp();
+  } else if (warp >= 2 + kEpiWarps) {
+    if (C::QUANT) {
+      // -------------------------------------------------- dequantisation
+      // warp w (10..17) expands codes [32 sub, 32 sub + 32) of the k-block, sub =
+      // ((w - 10) / 4) % 2, for the 32 features of quadrant w % 4 of this CTA's 128,
+      // into row `feature` of the weight slot (16-byte chunk c at c ^ (row & 7)),
+      // then counts on the even CTA's expansion barrier with a cluster-scope release
+      const int dw = warp - 2 - kEpiWarps;
+      const int sub = (dw >> 2) & 1;
+      const int feat = (warp & 3) * 32 + lane;
+      const uint32_t deq_even = mapa_shared(deq_bar, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int aslot = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, TN, tile, ti);
+        const int kbl = p.prob[ti.prob].K / 64;
+        for (int kb = 0; kb < kbl; ++kb) {
+          if (!pair_wait(&rawfull_bar[stage], phase, p, abort_flag, peer_abort) ||
+              !pair_wait(&wempty_bar[aslot], aphase ^ 1, p, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* st = tiles + stage * C::STAGE_BYTES;
+          const __nv_bfloat16 sc = reinterpret_cast<const __nv_bfloat16*>(st + C::SCALE_OFF)[feat];
+          uint32_t w[16];
+          dequant_row<WQ, 32>(st + C::RAW_OFF + feat * C::RAW_ROW + sub * (C::RAW_ROW / 2), sc,
+                              lane, w);
+          uint8_t* dst = wslots + aslot * C::W_SLOT_BYTES + feat * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(dst + 16 * ((4 * sub + c) ^ (feat & 7))) =
+                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          fence_proxy_async_shared();   // the tensor core reads them through the async proxy
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_release_cluster(deq_even + aslot * 8);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
@@ -284,6 +401,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcBaseThreads, 1)
       // flight a fixed, generous time to land
       const long long t0 = clock64();
       while (clock64() - t0 < (1ll << 21)) {}
+    }
+    // quantised: this CTA's codes and scales complete on its own barriers
+    if (C::QUANT) {
+      for (int s = 0; s < STAGES; ++s) {
+        if (issued[s]) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&rawfull_bar[s], (uint32_t)(issued[s] - 1)) &&
+                 clock64() - t0 < kWaitCycles) {}
+        }
+      }
     }
   }
   // neither CTA leaves while the pair's MMAs may still read its memory or write its

@@ -398,33 +398,34 @@ moe_status launch_tc(const TcParams& p, cudaStream_t st) {
 // GPC, so a GPC with an odd number of free SMs leaves one idle: the persistent
 // grid must not ask for more pairs than fit, or the last ones would run as a
 // second wave after the others have finished their share of the tiles.
-template <int EPI>
+template <int EPI, int WQ>
 int resident_pairs() {
-  static int cached[8] = {};   // per device, on first use
+  static int cached[8] = {};   // per device and kernel, on first use
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (dev < 8 && cached[dev] > 0) return cached[dev];
-  using C = PairConfig<EPI>;
+  using C = PairConfig<EPI, WQ>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms() / 2 * 2);
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, (void*)k_tc_gemm_pair<EPI>, &cfg) != cudaSuccess || n < 1)
+  if (cudaOccupancyMaxActiveClusters(&n, (void*)k_tc_gemm_pair<EPI, WQ>, &cfg) != cudaSuccess ||
+      n < 1)
     n = 0;
   if (n > num_sms() / 2) n = num_sms() / 2;
   if (dev < 8 && n > 0) cached[dev] = n;
   return n;
 }
 
-template <int EPI>
+template <int EPI, int WQ>
 moe_status launch_pair(const TcParams& p, cudaStream_t st) {
-  using C = PairConfig<EPI>;
-  auto kern = k_tc_gemm_pair<EPI>;
+  using C = PairConfig<EPI, WQ>;
+  auto kern = k_tc_gemm_pair<EPI, WQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  const int pairs = resident_pairs<EPI>();
+  const int pairs = resident_pairs<EPI, WQ>();
   if (pairs < 1) return MOE_ERR_CUDA;
   MOE_LAUNCH((kern), 2 * pairs, C::THREADS, C::SMEM_BYTES, st, p);
   return check_launch();
@@ -440,12 +441,9 @@ moe_status launch_tc_bn_q(int bn, bool pair, const TcParams& p, cudaStream_t st)
     case 32: return launch_tc<EPI, 32, false, WQ>(p, st);
     case 64: return launch_tc<EPI, 64, false, WQ>(p, st);
     default:   // prefill tiles
-      if constexpr (WQ == WQ_BF16) {   // tokens on MMA-M
-        if (pair) return launch_pair<EPI>(p, st);
-        return launch_tc<EPI, 128, true, WQ>(p, st);
-      } else {                         // quantised: tokens on M, expanded weights in smem
-        return launch_tc<EPI, 128, true, WQ>(p, st);
-      }
+      // tokens on M (quantised weights expanded into shared memory)
+      if (pair) return launch_pair<EPI, WQ>(p, st);
+      return launch_tc<EPI, 128, true, WQ>(p, st);
   }
 }
 

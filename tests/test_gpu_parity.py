@@ -525,14 +525,22 @@ PREFILL_TILES = {
     # 750 mean rows: 2 pair tiles + 238, 5 single tiles + 110), capacity-cut
     "bf16_many_tiles": (LayerShape("bf16_many_tiles", d=256, E=8, k=4, f=256, n_shared=1,
                                    capacity_factor=1.1, seed=24), 1500),
+    # quantised weights expanded into shared memory, on CTA pairs or single CTAs
+    # (550 / 600 / 560 rows per expert: pairs by default)
+    "int4_pairs": (LayerShape("int4_pairs", d=256, E=4, k=2, f=384, n_shared=1, expert="int4",
+                              seed=28), 1100),
+    "int8_pairs": (LayerShape("int8_pairs", d=384, E=4, k=2, f=256, expert="int8",
+                              capacity_factor=1.1, seed=29), 1200),
+    "fp8_pairs": (LayerShape("fp8_pairs", d=256, E=8, k=4, f=256, n_shared=1, expert="fp8",
+                             seed=30), 1120),
 }
 
 
 @pytest.mark.parametrize("name", list(PREFILL_TILES))
 def test_prefill_pair_and_single_tiles_give_the_same_bits(name):
     """moe_config.prefill_tiles picks 256-token tiles on CTA pairs (2) or 128-token
-    tiles on single CTAs (1) for bf16 prefill batches (0: chosen by the rows per
-    expert).  Each output element is one FP32 dot product accumulated in the same
+    tiles on single CTAs (1) for prefill batches (0: chosen by the rows per
+    expert), bf16 or quantised.  Each output element is one FP32 dot product accumulated in the same
     k order either way, so the layer outputs agree bit for bit; the result is
     checked against the oracle."""
     sh, T = PREFILL_TILES[name]
@@ -550,6 +558,7 @@ def test_prefill_pair_and_single_tiles_give_the_same_bits(name):
     assert M.moe_get_device_status(layer.ws) == 0
     assert torch.equal(pair, single)
     assert torch.equal(auto, single)
+    assert M.moe_layer_launch_count(layer.cfg) >= 8
     res = run_layer(sh, T, tokens=sample_rows(T), data=data)
     assert res.max_margin_mismatch < ROUTE_MARGIN
     assert res.err_ratio <= TOL[sh.expert], res.err_ratio
