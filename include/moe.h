@@ -120,10 +120,10 @@ typedef struct moe_config {
   int32_t prefill_tiles;   /* tensor-core experts at prefill (more than 64 rows per expert on
                               average): 1 = tiles of 128 tokens on single CTAs, 2 = tiles
                               of 256 tokens on pairs of CTAs (one cta_group::2 MMA per
-                              k-step), 0 = automatic: pairs when the batch averages at
-                              least 512 rows per routed expert (a pair tile half empty
-                              costs twice a single one), else single CTAs.  All give the
-                              same bits; other values are rejected                      */
+                              k-step), 0 = automatic: pairs for bf16 experts when the
+                              batch averages at least 512 rows per routed expert (a pair
+                              tile half empty costs twice a single one), else single
+                              CTAs.  All give the same bits; other values are rejected  */
 } moe_config;
 
 /* Layer weights (device pointers, caller-owned).

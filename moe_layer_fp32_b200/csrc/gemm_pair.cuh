@@ -52,10 +52,11 @@ struct PairConfig {
   static constexpr uint32_t TOKEN_OFF = QUANT ? 0 : B_HALF;
   static constexpr uint32_t RAW_OFF = A_BYTES;
   static constexpr uint32_t SCALE_OFF = A_BYTES + RAW_BYTES;
-  // quantised: two shared-memory slots of this CTA's expanded weights (the MMA's B
+  // quantised: shared-memory slots of this CTA's expanded weights (the MMA's B
   // half), 128 rows of 128 B, K-major with the 128-byte swizzle
   static constexpr uint32_t W_SLOT_BYTES = QUANT ? 128 * 128 : 0;
-  static constexpr uint32_t W_REGION = 2 * W_SLOT_BYTES;
+  static constexpr int W_SLOTS = 4;   // expansion runs up to four k-blocks ahead
+  static constexpr uint32_t W_REGION = W_SLOTS * W_SLOT_BYTES;
   static constexpr int STAGES_RAW = (184 * 1024 - W_REGION) / STAGE_BYTES;
   static constexpr int STAGES = QUANT ? (STAGES_RAW > 8 ? 8 : STAGES_RAW) : 6;
   static constexpr uint32_t ACC_COLS = 256;
@@ -68,7 +69,7 @@ struct PairConfig {
   static constexpr int THREADS = kTcBaseThreads + 32 * DEQ_WARPS;
   // full, empty, [raw full] per stage; tfull, tempty, drain; [deq, wempty] x 2
   static constexpr uint32_t BAR_BYTES =
-      8 * (2 * STAGES + 5 + (QUANT ? STAGES + 4 : 0)) + 16 + 4 * STAGES;
+      8 * (2 * STAGES + 5 + (QUANT ? STAGES + 2 * W_SLOTS : 0)) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 5 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 16 * 4;
   static constexpr uint32_t SMEM_BYTES =
@@ -114,12 +115,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
   uint64_t* tempty_bar = tfull_bar + 2;       // [2]
   uint64_t* drain_bar = tempty_bar + 2;       // [1]
   // quantised: this CTA's codes landed [STAGES] (local); both CTAs' weight slot a
-  // expanded [2] (the even CTA's, counted by both CTAs' dequantisation warps); this
-  // CTA's slot a read by the MMAs [2] (local)
+  // expanded [W_SLOTS] (the even CTA's, counted by both CTAs' dequantisation warps);
+  // this CTA's slot a read by the MMAs [W_SLOTS] (local)
   uint64_t* rawfull_bar = drain_bar + 1;
   uint64_t* deq_bar = rawfull_bar + (C::QUANT ? STAGES : 0);
-  uint64_t* wempty_bar = deq_bar + (C::QUANT ? 2 : 0);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty_bar + (C::QUANT ? 2 : 0));
+  uint64_t* wempty_bar = deq_bar + (C::QUANT ? C::W_SLOTS : 0);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty_bar + (C::QUANT ? C::W_SLOTS : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* issued = const_cast<int*>(abort_flag) + 2;   // [STAGES] last issued parity + 1
   int* prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
@@ -144,7 +145,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
     mbar_init(drain_bar, 1);
     if (C::QUANT) {
       for (int s = 0; s < STAGES; ++s) mbar_init(&rawfull_bar[s], 1);
-      for (int a = 0; a < 2; ++a) {
+      for (int a = 0; a < C::W_SLOTS; ++a) {
         mbar_init(&deq_bar[a], 2 * C::DEQ_WARPS);
         mbar_init(&wempty_bar[a], 1);
       }
@@ -295,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
           if (C::QUANT) {
             tc2_commit(smem_u32(&wempty_bar[aslot]));
             tc2_commit(wempty_peer + aslot * 8);
-            if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+            if (++aslot == C::W_SLOTS) { aslot = 0; aphase ^= 1; }
           }
         }
         if (!ok) break;
@@ -350,9 +351,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
           fence_proxy_async_shared();   // the tensor core reads them through the async proxy
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_release_cluster(deq_even + aslot * 8);
+          if (lane == 0) {
+            if (rank == 0) mbar_arrive(&deq_bar[aslot]);   // the issuing CTA's own barrier
+            else mbar_arrive_release_cluster(deq_even + aslot * 8);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
-          if (++aslot == 2) { aslot = 0; aphase ^= 1; }
+          if (++aslot == C::W_SLOTS) { aslot = 0; aphase ^= 1; }
         }
       }
     }

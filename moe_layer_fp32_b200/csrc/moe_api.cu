@@ -141,9 +141,12 @@ inline bool interleave_tiles(const moe_config* c) {
 // 2-12% faster from 512 rows per expert up (OLMoE-shaped T=4096, 16384,
 // V2-Lite-shaped T=8192) and 7% slower at 295 (DeepSeek-V3-shaped T=9440).
 constexpr double kPairMinRowsPerExpert = 512.0;
+// Quantised experts on pairs (each CTA expanding half of the 256 weight columns)
+// measured slower than on single CTAs (Qwen3-shaped int4 T=16384 gate/up: 1.57 ms
+// against 1.16 ms): the automatic choice keeps them on single CTAs.
 inline bool pair_tiles(const moe_config* c) {
   if (c->prefill_tiles != 0) return c->prefill_tiles == 2;
-  return (double)n_slots(c) / c->E >= kPairMinRowsPerExpert;
+  return c->expert_dtype == MOE_BF16 && (double)n_slots(c) / c->E >= kPairMinRowsPerExpert;
 }
 // Inside the layer forward the gated routed rows of tensor-core experts are kept
 // in bf16 (half the bytes the down GEMM writes and the combine reads); the

@@ -526,7 +526,7 @@ PREFILL_TILES = {
     "bf16_many_tiles": (LayerShape("bf16_many_tiles", d=256, E=8, k=4, f=256, n_shared=1,
                                    capacity_factor=1.1, seed=24), 1500),
     # quantised weights expanded into shared memory, on CTA pairs or single CTAs
-    # (550 / 600 / 560 rows per expert: pairs by default)
+    # (550 / 600 / 560 rows per expert; quantised experts take single CTAs by default)
     "int4_pairs": (LayerShape("int4_pairs", d=256, E=8, k=4, f=384, n_shared=1, expert="int4",
                               seed=28), 1100),
     "int8_pairs": (LayerShape("int8_pairs", d=384, E=8, k=4, f=256, expert="int8",
