@@ -345,8 +345,9 @@ MOE_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
 }
 // arrive that releases the caller's earlier writes at cluster scope (shared-memory
 // data that the pair's MMA, issued by the other CTA, is about to read)
-MOE_DEV void mbar_arrive_release_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+MOE_DEV void mbar_arrive_release_cluster(uint32_t cluster_addr, uint32_t count) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   cluster_addr), "r"(count)
                : "memory");
 }
 MOE_DEV void st_shared_remote_u32(uint32_t cluster_addr, uint32_t v) {

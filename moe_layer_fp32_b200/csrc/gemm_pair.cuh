@@ -69,7 +69,7 @@ struct PairConfig {
   static constexpr int THREADS = kTcBaseThreads + 32 * DEQ_WARPS;
   // full, empty, [raw full] per stage; tfull, tempty, drain; [deq, wempty] x 2
   static constexpr uint32_t BAR_BYTES =
-      8 * (2 * STAGES + 5 + (QUANT ? STAGES + 2 * W_SLOTS : 0)) + 16 + 4 * STAGES;
+      8 * (2 * STAGES + 5 + (QUANT ? STAGES + 3 * W_SLOTS : 0)) + 16 + 4 * STAGES;
   static constexpr uint32_t PREFIX_BYTES = 5 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t EPI_BYTES = kEpiWarps * 32 * 16 * 4;
   static constexpr uint32_t SMEM_BYTES =
@@ -120,7 +120,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
   uint64_t* rawfull_bar = drain_bar + 1;
   uint64_t* deq_bar = rawfull_bar + (C::QUANT ? STAGES : 0);
   uint64_t* wempty_bar = deq_bar + (C::QUANT ? C::W_SLOTS : 0);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty_bar + (C::QUANT ? C::W_SLOTS : 0));
+  // the other CTA: its slot a expanded [W_SLOTS] (local, relayed to deq_bar)
+  uint64_t* deq_local = wempty_bar + (C::QUANT ? C::W_SLOTS : 0);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(deq_local + (C::QUANT ? C::W_SLOTS : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* issued = const_cast<int*>(abort_flag) + 2;   // [STAGES] last issued parity + 1
   int* prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
@@ -146,6 +148,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
     if (C::QUANT) {
       for (int s = 0; s < STAGES; ++s) mbar_init(&rawfull_bar[s], 1);
       for (int a = 0; a < C::W_SLOTS; ++a) {
+        mbar_init(&deq_local[a], C::DEQ_WARPS);
         mbar_init(&deq_bar[a], 2 * C::DEQ_WARPS);
         mbar_init(&wempty_bar[a], 1);
       }
@@ -309,6 +312,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
       tc2_commit(smem_u32(drain_bar));
       const long long t0 = clock64();
       while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < kWaitCycles) {}
+    } else if (C::QUANT && lane == 0 && rank == 1) {
+      // ------------------------------------------ expansion relay (other CTA)
+      // once this CTA's eight dequantisation warps have filled weight slot a, count
+      // them on the issuing CTA's barrier with one cluster-scope release
+      const uint32_t deq_even = mapa_shared(deq_bar, 0);
+      int aslot = 0;
+      uint32_t aphase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        TileInfo ti;
+        decode_tile(p, prefix, BN, TN, tile, ti);
+        const int kbl = p.prob[ti.prob].K / 64;
+        for (int kb = 0; kb < kbl; ++kb) {
+          if (!pair_wait(&deq_local[aslot], aphase, p, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_release_cluster(deq_even + aslot * 8, C::DEQ_WARPS);
+          if (++aslot == C::W_SLOTS) { aslot = 0; aphase ^= 1; }
+        }
+      }
     }
     __syncwarp();
   } else if (warp >= 2 + kEpiWarps) {
@@ -321,7 +345,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
       const int dw = warp - 2 - kEpiWarps;
       const int sub = (dw >> 2) & 1;
       const int feat = (warp & 3) * 32 + lane;
-      const uint32_t deq_even = mapa_shared(deq_bar, 0);
       int stage = 0;
       uint32_t phase = 0;
       int aslot = 0;
@@ -351,10 +374,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairConfig<EPI, WQ>:
           fence_proxy_async_shared();   // the tensor core reads them through the async proxy
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            if (rank == 0) mbar_arrive(&deq_bar[aslot]);   // the issuing CTA's own barrier
-            else mbar_arrive_release_cluster(deq_even + aslot * 8);
-          }
+          // the issuing CTA's warps count on its barrier; the other CTA's on a local
+          // one, which one relay thread hands over with a single cluster-scope release
+          if (lane == 0) mbar_arrive(rank == 0 ? &deq_bar[aslot] : &deq_local[aslot]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
           if (++aslot == C::W_SLOTS) { aslot = 0; aphase ^= 1; }
         }
