@@ -832,9 +832,12 @@ __global__ void __launch_bounds__(256) k_gather_rows(const TA* __restrict__ xn,
 // ---------------------------------------------------------------------------
 template <int VEC>
 MOE_DEV void loadv(const float* p, float (&v)[VEC]) {
-  if constexpr (VEC == 4) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  if constexpr (VEC == 4 || VEC == 8) {
+#pragma unroll
+    for (int h = 0; h < VEC / 4; ++h) {
+      const float4 a = *reinterpret_cast<const float4*>(p + 4 * h);
+      v[4 * h] = a.x; v[4 * h + 1] = a.y; v[4 * h + 2] = a.z; v[4 * h + 3] = a.w;
+    }
   } else {
 #pragma unroll
     for (int u = 0; u < VEC; ++u) v[u] = p[u];
@@ -842,7 +845,15 @@ MOE_DEV void loadv(const float* p, float (&v)[VEC]) {
 }
 template <int VEC>
 MOE_DEV void loadv(const __nv_bfloat16* p, float (&v)[VEC]) {
-  if constexpr (VEC == 4) {
+  if constexpr (VEC == 8) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&w[h]);
+      v[2 * h] = __low2float(a); v[2 * h + 1] = __high2float(a);
+    }
+  } else if constexpr (VEC == 4) {
     const uint2 q = *reinterpret_cast<const uint2*>(p);
     const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&q.x);
     const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&q.y);
@@ -854,8 +865,11 @@ MOE_DEV void loadv(const __nv_bfloat16* p, float (&v)[VEC]) {
 }
 template <int VEC>
 MOE_DEV void storev(float* p, const float (&v)[VEC]) {
-  if constexpr (VEC == 4) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  if constexpr (VEC == 4 || VEC == 8) {
+#pragma unroll
+    for (int h = 0; h < VEC / 4; ++h)
+      *reinterpret_cast<float4*>(p + 4 * h) =
+          make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
   } else {
 #pragma unroll
     for (int u = 0; u < VEC; ++u) p[u] = v[u];
@@ -863,7 +877,15 @@ MOE_DEV void storev(float* p, const float (&v)[VEC]) {
 }
 template <int VEC>
 MOE_DEV void storev(__nv_bfloat16* p, const float (&v)[VEC]) {
-  if constexpr (VEC == 4) {
+  if constexpr (VEC == 8) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      __nv_bfloat162 a = __floats2bfloat162_rn(v[2 * h], v[2 * h + 1]);
+      w[h] = *reinterpret_cast<uint32_t*>(&a);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (VEC == 4) {
     __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
     __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
     *reinterpret_cast<uint2*>(p) =

@@ -913,8 +913,11 @@ moe_status launch_combine(const moe_config* c, const void* y, bool rows_bf16,
 moe_status run_combine(const moe_config* c, const void* y, bool rows_bf16, const int32_t* slot,
                        const float* ys, const void* res, void* out, cudaStream_t st) {
   auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  // eight columns per thread (16-byte bf16 loads) where the rows allow it: measured
+  // 0.78x the time of four on the V3-shaped T=9440 combine
   if (a16(y) && a16(ys) && a16(res) && a16(out))
-    return launch_combine<4>(c, y, rows_bf16, slot, ys, res, out, st);
+    return c->d % 8 == 0 ? launch_combine<8>(c, y, rows_bf16, slot, ys, res, out, st)
+                         : launch_combine<4>(c, y, rows_bf16, slot, ys, res, out, st);
   return launch_combine<1>(c, y, rows_bf16, slot, ys, res, out, st);
 }
 
@@ -941,7 +944,8 @@ moe_status run_combine_ec(const moe_config* c, const void* y, bool rows_bf16,
                           cudaStream_t st) {
   auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
   if (a16(y) && a16(ys) && a16(res) && a16(out))
-    return launch_combine_ec<4>(c, y, rows_bf16, slot_te, ys, res, out, st);
+    return c->d % 8 == 0 ? launch_combine_ec<8>(c, y, rows_bf16, slot_te, ys, res, out, st)
+                         : launch_combine_ec<4>(c, y, rows_bf16, slot_te, ys, res, out, st);
   return launch_combine_ec<1>(c, y, rows_bf16, slot_te, ys, res, out, st);
 }
 
