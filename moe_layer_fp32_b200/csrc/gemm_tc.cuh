@@ -102,6 +102,11 @@ struct TcParams {
   // bound by streaming a light expert's weights run beside tiles bound by the
   // tensor cores instead of all at once
   int interleave;
+  // Dynamic tile order (nullptr: static, tiles cta, cta + ncta, ...): each CTA takes
+  // its first tile statically and every further one from this counter (zero when
+  // the launch starts), so that tiles run in index order whatever their costs and
+  // the tiles that share an expert's weights stay close in time (L2 reuse)
+  int32_t* tile_ctr;
 };
 
 constexpr int kMaxSplit = 4;
@@ -188,7 +193,11 @@ struct TcConfig {
                                     : WQ == WQ_BF16 ? idesc_bf16(128, BN, true, false)
                                                     : idesc_bf16(128, BN, false, false);
   // barriers + bookkeeping after the tiles
-  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5 + 2 * A_SLOTS) + 16 + 4 * STAGES;
+  // tile queue from the producer to the other roles
+  static constexpr int TQ = 4;
+  static constexpr int TQ_CONSUMERS = 1 + kEpiWarps + DEQ_WARPS;
+  static constexpr uint32_t BAR_BYTES =
+      8 * (2 * STAGES + 5 + 2 * A_SLOTS + 2 * TQ) + 16 + 4 * STAGES + 4 * TQ;
   // tile prefixes of the two problems, the heavy / light class prefixes of
   // problem 0 (interleaved order), and problem 0's group offsets
   static constexpr uint32_t PREFIX_BYTES = 5 * (kMaxGroups + 1) * 4;
@@ -536,8 +545,11 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   uint64_t* drain_bar = tempty_bar + 2;       // [1]
   uint64_t* deq_bar = drain_bar + 1;                   // [A_SLOTS] weight slot filled
   uint64_t* aempty_bar = deq_bar + C::A_SLOTS;         // [A_SLOTS] weight slot consumed
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(aempty_bar + C::A_SLOTS) + 1;
+  uint64_t* tq_full = aempty_bar + C::A_SLOTS;         // [TQ] tile index written
+  uint64_t* tq_empty = tq_full + C::TQ;                // [TQ] tile index read by every role
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tq_empty + C::TQ) + 1;
   int* issued = const_cast<int*>(abort_flag) + 2;               // [STAGES] last issued parity+1
+  volatile int* tq = issued + STAGES;                           // [TQ] tile indices
   int* prefix = reinterpret_cast<int*>(
       reinterpret_cast<uint8_t*>(full_bar) + C::BAR_BYTES);
   // epilogue scratch, 16-byte aligned (float4 staging in the direct DOWN epilogue)
@@ -556,6 +568,10 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
     for (int a = 0; a < C::A_SLOTS; ++a) {
       mbar_init(&deq_bar[a], C::DEQ_WARPS);
       mbar_init(&aempty_bar[a], 1);
+    }
+    for (int q = 0; q < C::TQ; ++q) {
+      mbar_init(&tq_full[q], 1);
+      mbar_init(&tq_empty[q], C::TQ_CONSUMERS);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
@@ -599,6 +615,34 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
   if (EPI == EPI_ROUTER && p.k_splits > 1) S = p.k_splits;
   if (kCanSplit) S = split_parts(p, out_tiles, ncta);
   const int total = out_tiles * S;
+
+  // Tile queue.  The producer's lane 0 decides each tile of this CTA -- statically,
+  // or from the dynamic counter after the first -- and publishes it; the MMA thread,
+  // the epilogue warps and the dequantisation warps read the same sequence.  An
+  // index >= total ends it.
+  auto next_tile = [&](int k) -> int {
+    if (k == 0) return cta;
+    return p.tile_ctr ? ncta + atomicAdd(p.tile_ctr, 1) : cta + k * ncta;
+  };
+  int tq_slot = 0;        // this thread's position in the queue
+  uint32_t tq_phase = 0;
+  auto push_tile = [&](int t) -> bool {
+    if (!mbar_wait(&tq_empty[tq_slot], tq_phase ^ 1, p.err, abort_flag, p.wait_cycles)) return false;
+    tq[tq_slot] = t;
+    mbar_arrive(&tq_full[tq_slot]);
+    if (++tq_slot == C::TQ) { tq_slot = 0; tq_phase ^= 1; }
+    return true;
+  };
+  // one consumer: a whole warp (every lane reads, lane 0 counts) or a lone thread
+  auto pop_tile = [&](bool whole_warp, bool patient) -> int {
+    if (!mbar_wait(&tq_full[tq_slot], tq_phase, p.err, abort_flag, p.wait_cycles, patient))
+      return total;
+    const int t = tq[tq_slot];
+    if (whole_warp) __syncwarp();
+    if (!whole_warp || lane == 0) mbar_arrive(&tq_empty[tq_slot]);
+    if (++tq_slot == C::TQ) { tq_slot = 0; tq_phase ^= 1; }
+    return t;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -650,7 +694,10 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
     bool ok = true;
     if (!any_gather) {
       if (lane == 0) {
-        for (int tile = cta; tile < total && ok; tile += ncta) {
+        for (int k = 0; ok; ++k) {
+          const int tile = next_tile(k);
+          if (!push_tile(tile)) { ok = false; break; }
+          if (tile >= total) break;
           TileInfo ti;
           decode_work(p, prefix, BN, TN, S, tile, ti);
           const TcProblem& P = p.prob[ti.prob];
@@ -662,7 +709,15 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         }
       }
     } else {
-      for (int tile = cta; tile < total && ok; tile += ncta) {
+      for (int k = 0; ok; ++k) {
+        int tile = 0;
+        if (lane == 0) {
+          tile = next_tile(k);
+          if (!push_tile(tile)) tile = -1;
+        }
+        tile = __shfl_sync(0xffffffffu, tile, 0);
+        if (tile < 0) { ok = false; break; }
+        if (tile >= total) break;
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
         const TcProblem& P = p.prob[ti.prob];
@@ -703,7 +758,9 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = cta; tile < total && ok; tile += ncta) {
+      while (ok) {
+        const int tile = pop_tile(false, false);
+        if (tile >= total) break;
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag, p.wait_cycles)) break;
@@ -780,7 +837,9 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
       int aslot = 0;
       uint32_t aphase = 0;
       bool ok = true;
-      for (int tile = cta; tile < total && ok; tile += ncta) {
+      while (ok) {
+        const int tile = pop_tile(true, true);
+        if (tile >= total) break;
         TileInfo ti;
         decode_work(p, prefix, BN, TN, S, tile, ti);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
@@ -826,7 +885,9 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
     float* s_scale = epi_scale + (warp - 2) * 128;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cta; tile < total; tile += ncta) {
+    while (true) {
+      const int tile = pop_tile(true, true);
+      if (tile >= total) break;
       TileInfo ti;
       decode_work(p, prefix, BN, TN, S, tile, ti);
       const TcProblem& P = p.prob[ti.prob];

@@ -156,7 +156,7 @@ inline bool y_bf16(const moe_config* c) { return tc_experts(c); }
 
 struct Layout {
   size_t err, xn, part, idx, gate, counts, offsets, perm, slot, dropped, blk, xp, split,
-      splitcnt, h, y, ys, sct,
+      splitcnt, tilectr, h, y, ys, sct,
       total;
   int ns;
 };
@@ -231,6 +231,9 @@ Layout layout(const moe_config* c) {
   L.xp = o;       o = align_up(o + (tc_experts(c) && !gather_in_gemm(c) ? R * d * act : 0));
   L.split = o;    o = align_up(o + (split_k(c) ? (size_t)num_sms() * 2 * pick_bn(c) * 128 * 4 : 0));
   L.splitcnt = o; o = align_up(o + (split_k(c) ? (size_t)split_counters() * 4 : 0));
+  // right after the split-K counters (one range zeroes both): the dynamic tile
+  // counters of the two expert GEMMs
+  L.tilectr = o;  o = align_up(o + 2 * 4);
   L.h = o;        o = align_up(o + (R + S * T) * f * hb);
   L.y = o;        o = align_up(o + R * d * (y_bf16(c) ? 2 : 4));
   L.ys = o;       o = align_up(o + S * T * d * 4);
@@ -845,8 +848,13 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
   const bool g4 = gather_in_gemm(c);
   float* split_part = split_k(c) ? at<float>(ws, L.split) : nullptr;
   int32_t* split_cnt = split_k(c) ? at<int32_t>(ws, L.splitcnt) : nullptr;
-  if (split_cnt && !counters_zeroed &&
-      cudaMemsetAsync(split_cnt, 0, (size_t)split_counters() * 4, st) != cudaSuccess)
+  // prefill tiles take their tiles in index order from a counter (the tiles that
+  // share an expert's weights stay close in time)
+  int32_t* tile_ctr = bn == 128 ? at<int32_t>(ws, L.tilectr) : nullptr;
+  // the split-K and dynamic tile counters (zeroed by the layer's RMSNorm otherwise)
+  if (!counters_zeroed && (split_cnt || tile_ctr) &&
+      cudaMemsetAsync(at<int32_t>(ws, L.splitcnt), 0, L.tilectr + 8 - L.splitcnt, st) !=
+          cudaSuccess)
     return MOE_ERR_CUDA;
   __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
   if (!g4) {
@@ -862,6 +870,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     if ((s = gateup_params(c, w, wl, wq, xn, xp, offsets, rr, h, split_part, split_cnt, err, p)) !=
         MOE_OK)
       return s;
+    p.tile_ctr = tile_ctr;
     s = launch_tc_bn<EPI_GATEUP>(bn, wq, pair_tiles(c), p, st);
     if (s != MOE_OK) return s;
     mk->mark(st);
@@ -871,6 +880,7 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
     if ((s = down_params(c, w, wl, wq, offsets, rr, gate, h, y, rows_bf16, ys, split_part,
                          split_cnt, err, p)) != MOE_OK)
       return s;
+    p.tile_ctr = tile_ctr ? tile_ctr + 1 : nullptr;
     s = launch_tc_bn<EPI_DOWN>(bn, wq, pair_tiles(c), p, st);
     mk->mark(st);
   }
@@ -1113,9 +1123,9 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
     if (aligned) return run_decode_layer(cfg, w, x, out, ws, logits_out, idx, counts, st);
   }
   mk->mark(st);
-  int32_t* split_cnt = split_k(cfg) ? at<int32_t>(ws, L.splitcnt) : nullptr;
-  if ((s = run_rmsnorm(cfg, w, x, xn, st, split_cnt, split_cnt ? split_counters() : 0)) !=
-      MOE_OK)
+  // the expert GEMMs' split-K and dynamic tile counters, zeroed by the RMSNorm
+  if ((s = run_rmsnorm(cfg, w, x, xn, st, at<int32_t>(ws, L.splitcnt),
+                       (int)((L.tilectr + 8 - L.splitcnt) / 4))) != MOE_OK)
     return s;
   mk->mark(st);
   if ((s = run_router(cfg, w, xn, part, L.ns, err, st)) != MOE_OK) return s;
