@@ -222,6 +222,23 @@ MOE_DEV void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int c0, int
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// The same copy with an L2 eviction policy (from l2_evict_first) for the source lines.
+MOE_DEV void tma_load_3d_hint(void* dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2,
+                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+      "l"(policy)
+      : "memory");
+}
+// L2 policy for data read exactly once: its lines are the first to be evicted, so
+// that they do not push out lines that later copies read again.
+MOE_DEV uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 // Bring `bytes` (a multiple of 16) of global memory at p into L2, asynchronously.
 MOE_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),

@@ -118,6 +118,7 @@ struct TileInfo {
   int slot0;          // routed: slot of the tile's first token
   int bt, ks;         // split-K: output tile and this work item's part of K
   int kb0, kb1;       // k-blocks [kb0, kb1) of this work item
+  int whole;          // the tile holds all of its group's rows (its weights are read once)
 };
 
 // Weight blocks (128 features x 64 k) per pipeline stage: gate and up for
@@ -271,6 +272,7 @@ MOE_DEV void decode_tile(const TcParams& p, const int* prefix, int BN, int TN, i
     ti.b_row = P.b_row_base + g * P.b_group_stride + ti.m0;
   }
   ti.rows = min(BN, seg_rows - ti.m0);
+  ti.whole = ti.m0 == 0 && seg_rows <= BN;
   ti.slot0 = seg_start + ti.m0;
   ti.out_seg = P.out_row_base + (size_t)seg_start + ti.m0;
 }
@@ -663,7 +665,18 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
       // GATEUP: the up matrix at the same features; wide DOWN: features +128
       const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
       const int n2 = (EPI == EPI_GATEUP) ? ti.n0 : ti.n0 + 128;
-      if (WQ == WQ_BF16) {
+      if (WQ == WQ_BF16 && DIRECT && ti.whole) {
+        // the weights of a group that fits one token tile are read by this tile
+        // only: first out of L2, after the lines that later token tiles re-read
+        const uint64_t pol = l2_evict_first();
+        tma_load_3d_hint(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g, pol);
+        tma_load_3d_hint(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g, pol);
+        if (NA == 2) {
+          tma_load_3d_hint(st + C::A_BYTES, m2, &full_bar[stage], n2, kb * 64, ti.g, pol);
+          tma_load_3d_hint(st + C::A_BYTES + 8192, m2, &full_bar[stage], n2 + 64, kb * 64, ti.g,
+                           pol);
+        }
+      } else if (WQ == WQ_BF16) {
         tma_load_3d(st, &P.tmA, &full_bar[stage], ti.n0, kb * 64, ti.g);
         tma_load_3d(st + 8192, &P.tmA, &full_bar[stage], ti.n0 + 64, kb * 64, ti.g);
         if (NA == 2) {
