@@ -823,6 +823,41 @@ __global__ void __launch_bounds__(256) k_gather_rows(const TA* __restrict__ xn,
   }
 }
 
+// The same gather token by token: xp[slot_of[t k + j]] = xn[t] for every kept
+// assignment (slot >= 0).  One warp per token reads its row once and writes it to
+// each of its (at most 32) slots, so that xn is read from memory once instead of
+// once per assignment; the rows written are those of k_gather_rows.
+template <typename TA>
+__global__ void __launch_bounds__(256) k_gather_rows_by_token(const TA* __restrict__ xn,
+                                                              const int32_t* __restrict__ slot_of,
+                                                              int T, int k, int d,
+                                                              TA* __restrict__ xp) {
+  pdl_wait();
+  pdl_trigger();
+  const int vec_per_row = d * (int)sizeof(TA) / 16;
+  const int warps = gridDim.x * 8;
+  const int lane = threadIdx.x & 31;
+  constexpr int U = 8;   // vectors per lane loaded before they are stored
+  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += warps) {
+    const int my_slot = lane < k ? slot_of[(size_t)t * k + lane] : -1;
+    const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * d);
+    for (int i0 = lane; i0 < vec_per_row; i0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + 32 * u < vec_per_row) v[u] = src[i0 + 32 * u];
+      for (int j = 0; j < k; ++j) {
+        const int sl = __shfl_sync(0xffffffffu, my_slot, j);
+        if (sl < 0) continue;
+        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)sl * d);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (i0 + 32 * u < vec_per_row) dst[i0 + 32 * u] = v[u];
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // a8: combine, VEC consecutive elements per thread.  out = residual + shared
 // experts (s ascending) + kept assignments (j ascending), summed in FP32.  The

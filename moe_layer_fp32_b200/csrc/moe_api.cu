@@ -658,6 +658,7 @@ struct RoutedRows {
   const int32_t* src;
   int src_k;
   const int32_t* dst;
+  const int32_t* slot_of = nullptr;   // [T, k] slot of each assignment (-1: dropped), if known
 };
 
 // Parameters of the grouped gate/up GEMM: the routed problem (rows gathered by the
@@ -857,7 +858,12 @@ moe_status run_ffn(const moe_config* c, const moe_weights* w, const void* xn,
           cudaSuccess)
     return MOE_ERR_CUDA;
   __nv_bfloat16* xp = at<__nv_bfloat16>(ws, L.xp);
-  if (!g4) {
+  if (!g4 && rr.slot_of && k <= 32) {
+    // token by token (each row of xn read once); 64 warps per SM
+    MOE_LAUNCH((k_gather_rows_by_token<__nv_bfloat16>), 8 * num_sms(), 256, 0, st,
+               static_cast<const __nv_bfloat16*>(xn), rr.slot_of, T, k, c->d, xp);
+    if ((s = check_launch()) != MOE_OK) return s;
+  } else if (!g4) {
     // 64 warps per SM, so that many rows are in flight at once
     MOE_LAUNCH((k_gather_rows<__nv_bfloat16>), 8 * num_sms(), 256, 0, st,
                static_cast<const __nv_bfloat16*>(xn), rr.src, offsets + c->E, rr.src_k, c->d,
@@ -1166,8 +1172,8 @@ moe_status layer_forward_impl(const moe_config* cfg, const moe_weights* w, const
       return s;
   }
   mk->mark(st);
-  if ((s = run_ffn(cfg, w, xn, offsets, RoutedRows{perm, cfg->k, perm}, gate, y, ys, ws, st, mk,
-                   true, y_bf16(cfg))) != MOE_OK)
+  if ((s = run_ffn(cfg, w, xn, offsets, RoutedRows{perm, cfg->k, perm, slot}, gate, y, ys, ws,
+                   st, mk, true, y_bf16(cfg))) != MOE_OK)
     return s;
   s = run_combine(cfg, y, y_bf16(cfg), slot, ys, x, out, st);
   mk->mark(st);
