@@ -67,7 +67,7 @@ def workload_name(sh, T):
              "qwen3_int4": "Qwen3-30B-A3B-shaped (int4 experts)",
              "qwen3_int8": "Qwen3-30B-A3B-shaped (int8 experts)",
              "qwen3_fp8": "Qwen3-30B-A3B-shaped (fp8 experts)", "v3": "DeepSeek-V3-shaped",
-             "tiny": "Tiny"}
+             "v3_e32": "DeepSeek-V3-shaped (32 experts)", "tiny": "Tiny"}
     kind = "decode" if T <= 64 else "prefill"
     return f"{names.get(sh.name, sh.name)} MoE layer forward, {kind} T={T}"
 

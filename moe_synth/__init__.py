@@ -105,6 +105,11 @@ PRESETS: Dict[str, LayerShape] = {
     # DeepSeek-V3-shaped layer: 1 shared expert, Zipf(1.1) select-mode bias
     "v3": LayerShape("v3", d=7168, E=256, k=8, f=2048, n_shared=1, bias_mode="select",
                      seed=4, tokens=(32, 256, 9440)),
+    # profiling case of the V3-shaped expert GEMMs: the same d, f, k, shared expert and
+    # select-mode bias over 32 experts (2.9 GB of weights), T = 1184 giving the same
+    # 296 rows per expert on average as the V3-shaped T = 9440 batch
+    "v3_e32": LayerShape("v3_e32", d=7168, E=32, k=8, f=2048, n_shared=1,
+                         bias_mode="select", seed=4, tokens=(1184,)),
 }
 
 
