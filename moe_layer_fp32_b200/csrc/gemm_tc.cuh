@@ -57,6 +57,8 @@ struct TcProblem {
   CUtensorMap tmA2;           // second weight matrix (up) for GATEUP
   CUtensorMap tmB;            // activations [R][K] bf16 (dims k, r), box (64, BN); with
                               // gather_rows: box (64, 1), rows fetched four at a time
+  CUtensorMap tmB64;          // bf16 direct tiles: the same rows, box (64, 64), for tiles
+                              // of at most 64 rows
   const int32_t* offsets;     // [G+1] segments (B rows and output rows), or nullptr
   int G;                      // groups
   int uniform_rows;           // rows per group when offsets == nullptr
@@ -193,6 +195,11 @@ struct TcConfig {
   static constexpr uint32_t IDESC = DIRECT            ? idesc_bf16(128, 128 * NA, false, !SMEM_W)
                                     : WQ == WQ_BF16 ? idesc_bf16(128, BN, true, false)
                                                     : idesc_bf16(128, BN, false, false);
+  // bf16 direct tiles of at most 64 rows: one M = 64 MMA per step over the first 64
+  // token rows (a 64-row copy), the accumulator in lanes 0..15 of each TMEM lane
+  // quadrant (row 16 q + i in lane 32 q + i)
+  static constexpr bool M64 = DIRECT && WQ == WQ_BF16;
+  static constexpr uint32_t IDESC_M64 = idesc_bf16(64, 128 * NA, false, true);
   // barriers + bookkeeping after the tiles
   // tile queue from the producer to the other roles
   static constexpr int TQ = 4;
@@ -658,9 +665,10 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
     auto issue_stage = [&](uint8_t* st, int stage, uint32_t phase, const TileInfo& ti,
                            const TcProblem& P, int kb, bool gather) {
       // gathered rows: only the tile's own (rounded up to 16), 128 B each
+      const bool m64 = C::M64 && ti.rows <= 64;
       mbar_arrive_expect_tx(&full_bar[stage],
                             gather ? C::TX_BYTES - C::B_BYTES + 128u * tile_n(ti.rows, BN)
-                                   : C::TX_BYTES);
+                                   : C::TX_BYTES - (m64 ? 64u * 128u : 0u));
       issued[stage] = (int)phase + 1;
       // GATEUP: the up matrix at the same features; wide DOWN: features +128
       const void* m2 = (EPI == EPI_GATEUP) ? (const void*)&P.tmA2 : (const void*)&P.tmA;
@@ -700,7 +708,9 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
           else tma_load_3d(scl + 256, s2, &full_bar[stage], n2, kb / 2, ti.g);
         }
       }
-      if (!gather) tma_load_2d(st + C::TOKEN_OFF, &P.tmB, &full_bar[stage], kb * 64, ti.b_row);
+      if (!gather)
+        tma_load_2d(st + C::TOKEN_OFF, m64 ? (const void*)&P.tmB64 : (const void*)&P.tmB,
+                    &full_bar[stage], kb * 64, ti.b_row);
     };
     int stage = 0;
     uint32_t phase = 0;
@@ -779,7 +789,9 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, p.err, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
-        const uint32_t idesc = DIRECT ? C::IDESC : idesc_with_n(C::IDESC, tile_n(ti.rows, BN));
+        const uint32_t idesc = (C::M64 && ti.rows <= 64) ? C::IDESC_M64
+                               : DIRECT ? C::IDESC
+                                        : idesc_with_n(C::IDESC, tile_n(ti.rows, BN));
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, p.err, abort_flag, p.wait_cycles)) { ok = false; break; }
           if (WQ != WQ_BF16 &&
@@ -805,7 +817,7 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
               if (NA == 2) tc_mma_f16_tmem_a(d_tmem + BN, a_tm + 32, xd, idesc, accum);
             } else if (DIRECT) {
               const uint64_t wd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
-              tc_mma_f16(d_tmem, xd, wd, C::IDESC, accum);   // N = 128 * NA at once
+              tc_mma_f16(d_tmem, xd, wd, idesc, accum);   // N = 128 * NA at once
             } else {
               const uint64_t wd = sw128_desc(st_addr + kk * 2048, 8192, 1024);
               tc_mma_f16(d_tmem, wd, xd, idesc, accum);
@@ -910,7 +922,8 @@ MOE_DEV bool tc_gemm_run(const TcParams& p, uint8_t* smem, const uint32_t* tmem_
         // accumulator wait so that the loads overlap the MMAs
         int r;
         float sc;
-        direct_row<EPI>(P, ti, q * 32 + lane, r, sc);
+        const bool m64 = C::M64 && ti.rows <= 64;
+        direct_row<EPI>(P, ti, m64 ? (lane < 16 ? q * 16 + lane : BN) : q * 32 + lane, r, sc);
         if (!mbar_wait(&tfull_bar[acc], acc_phase, p.err, abort_flag, p.wait_cycles, true)) break;
         tc_fence_after();
         direct_store<EPI, TN>(P, ti, r, sc, t_base, half, lane,

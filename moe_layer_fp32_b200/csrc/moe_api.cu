@@ -682,6 +682,9 @@ moe_status gateup_params(const moe_config* c, const moe_weights* w, const moe_we
   } else if (!map_rows(&P.tmB, xp, R, c->d, bn)) {
     return MOE_ERR_CUDA;
   }
+  // bf16 direct tiles: 64-row copies for the tiles of at most 64 rows
+  const bool m64_maps = bn == 128 && !g4 && wq == WQ_BF16;
+  if (m64_maps && !map_rows(&P.tmB64, xp, R, c->d, 64)) return MOE_ERR_CUDA;
   if (wq != WQ_BF16 && (!map_scales(&P.tmS, c, w->s_gate, c->E, c->d, c->f) ||
                         !map_scales(&P.tmS2, c, w->s_up, c->E, c->d, c->f)))
     return MOE_ERR_CUDA;
@@ -699,6 +702,7 @@ moe_status gateup_params(const moe_config* c, const moe_weights* w, const moe_we
     if (!map_expert(&Q.tmA, wq, wl.sh_gate, S, c->d, c->f)) return MOE_ERR_CUDA;
     if (!map_expert(&Q.tmA2, wq, wl.sh_up, S, c->d, c->f)) return MOE_ERR_CUDA;
     if (!map_rows(&Q.tmB, xn, T, c->d, bn)) return MOE_ERR_CUDA;
+    if (m64_maps && !map_rows(&Q.tmB64, xn, T, c->d, 64)) return MOE_ERR_CUDA;
     if (wq != WQ_BF16 && (!map_scales(&Q.tmS, c, w->sh_s_gate, S, c->d, c->f) ||
                           !map_scales(&Q.tmS2, c, w->sh_s_up, S, c->d, c->f)))
       return MOE_ERR_CUDA;
@@ -740,6 +744,8 @@ moe_status down_params(const moe_config* c, const moe_weights* w, const moe_weig
     P.tmS2 = P.tmS;
   }
   if (!map_rows(&P.tmB, h, R + S * T, c->f, bn)) return MOE_ERR_CUDA;
+  if (bn == 128 && wq == WQ_BF16 && !map_rows(&P.tmB64, h, R + S * T, c->f, 64))
+    return MOE_ERR_CUDA;
   P.offsets = offsets;
   P.G = c->E;
   P.N = c->d;
@@ -761,6 +767,7 @@ moe_status down_params(const moe_config* c, const moe_weights* w, const moe_weig
       Q.tmS2 = Q.tmS;
     }
     Q.tmB = P.tmB;
+    Q.tmB64 = P.tmB64;
     Q.offsets = nullptr;
     Q.G = S;
     Q.uniform_rows = T;
