@@ -520,19 +520,39 @@ def cpu_baseline(li_host, x_host, sh, T):
 
 
 # --------------------------------------------------------------------- traffic
-def read_traffic(kernel, sh, T):
-    """DRAM bytes per launch of this kernel from the committed ncu summary, if
-    that summary was taken on the current kernel source."""
+def code_of(text):
+    """CUDA source without its // comments, trailing blanks and empty lines: what
+    the compiler sees (the kernel sources hold no // inside string literals)."""
+    lines = []
+    for line in text.splitlines():
+        i = line.find("//")
+        if i >= 0:
+            line = line[:i]
+        line = line.rstrip()
+        if line:
+            lines.append(line)
+    return "\n".join(lines) + "\n"
+
+
+def kernel_source_digest():
+    """First 16 hex digits of the SHA-256 of the GEMM kernel sources' code
+    (common.cuh, then gemm_tc.cuh), comments excluded."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{sh.name}_T{T}.md")
-    if not os.path.exists(path):
-        return None
     src = os.path.join(ROOT, "moe_layer_fp32_b200", "csrc")
     h = hashlib.sha256()
     for f in ("common.cuh", "gemm_tc.cuh"):
-        with open(os.path.join(src, f), "rb") as fh:
-            h.update(fh.read())
-    digest = h.hexdigest()[:16]
+        with open(os.path.join(src, f)) as fh:
+            h.update(code_of(fh.read()).encode())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel, sh, T):
+    """DRAM bytes per launch of this kernel from the committed ncu summary, if
+    that summary was taken on the current kernel code."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{sh.name}_T{T}.md")
+    if not os.path.exists(path):
+        return None
+    digest = kernel_source_digest()
     vals = {}
     with open(path) as fh:
         for line in fh:

@@ -106,8 +106,8 @@ struct TcParams {
   int interleave;
   // Dynamic tile order (nullptr: static, tiles cta, cta + ncta, ...): each CTA takes
   // its first tile statically and every further one from this counter (zero when
-  // the launch starts), so that tiles run in index order whatever their costs and
-  // the tiles that share an expert's weights stay close in time (L2 reuse)
+  // the launch starts), so that tiles run in index order whatever their costs and no
+  // CTA is left with a run of expensive tiles at the end of the launch
   int32_t* tile_ctr;
 };
 

@@ -63,3 +63,12 @@ def test_tensor_peak_follows_the_timed_loop_length():
     assert v == 1610.9 and "burst" in label and "200 ms" in label
     v, label = R.tensor_peak(peaks, 5.0)
     assert v == 1393.5 and "sustained" in label
+
+
+def test_kernel_digest_ignores_comments_only():
+    """The traffic figures stay tied to the kernel code: a comment edit keeps the
+    digest, a code edit changes it."""
+    import bench
+    code = "int a = 1;  // one\n// a note\n\nint b = 2;\n"
+    assert bench.code_of(code) == bench.code_of("int a = 1;\nint b = 2;   // two\n")
+    assert bench.code_of(code) != bench.code_of("int a = 1;\nint b = 3;\n")
