@@ -225,6 +225,39 @@ def test_grouped_ffn_matches_oracle_per_assignment(name):
             assert np.all(np.abs(ysn[s] - rs) <= rel * bs + 1e-30)
 
 
+def test_direct_tile_row_boundaries():
+    """128-token tiles around the 64-row and 128-row boundaries: experts receiving
+    exactly 1, 63, 64, 65, 127, 128, 129 and 0 rows (k = 1, every token routed by
+    hand), so that tiles of at most 64 rows (M = 64 MMAs over a 64-row copy), full
+    and ragged 128-row tiles and a one-row tail all occur in both GEMMs; every row
+    within the bound of the per-assignment test."""
+    counts = [1, 63, 64, 65, 127, 128, 129, 0]
+    T = sum(counts)
+    sh = LayerShape("rows", d=256, E=len(counts), k=1, f=512, seed=7, tokens=(T,))
+    li, x, dli, dx = inputs_on_device(sh, T)
+    cfg = M.make_config(sh, T)
+    ws = M.alloc_workspace(cfg)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    perm = np.arange(T, dtype=np.int32)            # slot s holds token s (k = 1)
+    gates = np.random.default_rng(11).uniform(0.1, 1.0, T).astype(np.float32)
+    y = torch.zeros(T, sh.d, dtype=torch.float32, device="cuda")
+    M.moe_grouped_ffn(cfg, M.make_weights(dli), dx, tdev(offsets, torch.int32),
+                      tdev(perm, torch.int32), tdev(gates, torch.float32), y, None, ws)
+    assert M.moe_get_device_status(ws) == 0
+    y = y.cpu().numpy()
+    ex = O.weights_from_inputs(li)
+    xf = x.float().numpy().astype(np.float64)
+    rel = 2.0 ** -8   # bf16 h, FP32 sums (the per-assignment test's bound)
+    for e, (a0, a1) in enumerate(zip(offsets[:-1], offsets[1:])):
+        if a1 == a0:
+            continue
+        X = xf[a0:a1]
+        h = O.silu(X @ ex.get("gate", e)) * (X @ ex.get("up", e))
+        ref = gates[a0:a1, None] * (h @ ex.get("down", e))
+        bound = rel * gates[a0:a1, None] * (np.abs(h) @ np.abs(ex.get("down", e)))
+        assert np.all(np.abs(y[a0:a1] - ref) <= bound + 1e-30), (e, counts[e])
+
+
 # --------------------------------------------------------------------- a8
 def test_combine_sums_in_fixed_order():
     T, d, k, S = 33, 256, 3, 2
