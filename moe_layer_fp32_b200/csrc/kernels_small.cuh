@@ -133,6 +133,22 @@ MOE_DEV void unpack8(const uint4& u, float (&f)[8]) {
   for (int i = 0; i < 4; ++i) { f[2 * i] = __low2float(h[i]); f[2 * i + 1] = __high2float(h[i]); }
 }
 
+// bf16 of (f r) g, the product taken in double and rounded once (bf16_from_double),
+// computed in FP32 where that gives the same bf16: f is a bf16 value (exact in FP32),
+// r32 = fl32(r), and the two FP32 products carry a relative error below 3 * 2^-24 --
+// at most 3 units in the last place of y -- so y rounds to the same bf16 as the
+// double product unless its 16 low bits lie within 8 units of the rounding midpoint
+// 0x8000 (about 1 in 4000 values), or y is zero, subnormal, huge or not finite;
+// those take the double product.
+MOE_DEV __nv_bfloat16 bf16_of_scaled(float f, float g, double r, float r32) {
+  const float y = (f * r32) * g;
+  const uint32_t u = __float_as_uint(y);
+  const uint32_t low = u & 0xFFFFu, ex = (u >> 23) & 0xFFu;
+  if (ex > 1u && ex < 253u && (low < 0x8000u - 8u || low > 0x8000u + 8u))
+    return __float2bfloat16_rn(y);
+  return bf16_from_double(((double)f * r) * (double)g);
+}
+
 // One token row, vectorised: thread i < NT keeps up to MAXV 16-byte vectors of the
 // row in registers between the sum of squares and the scaling pass (d up to
 // NT * MAXV * 8).  `red` is a shared scratch of NT / 32 doubles.  Same arithmetic
@@ -167,6 +183,7 @@ MOE_DEV void rmsnorm_row_bf16v(const __nv_bfloat16* __restrict__ xrow,
 #pragma unroll
   for (int w = 0; w < NT / 32; ++w) tot += red[w];
   const double r = 1.0 / sqrt(tot / d + eps);
+  const float r32 = (float)r;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int v = threadIdx.x + i * NT;
@@ -179,7 +196,7 @@ MOE_DEV void rmsnorm_row_bf16v(const __nv_bfloat16* __restrict__ xrow,
       uint4 o;
       __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(&o);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) ob[j] = bf16_from_double(((double)f[j] * r) * (double)g[j]);
+      for (int j = 0; j < 8; ++j) ob[j] = bf16_of_scaled(f[j], g[j], r, r32);
       outr[v] = o;
     }
   }
